@@ -1,0 +1,225 @@
+/*
+ * poetx.h -- C ABI of libpoetx, the B200 (sm_100a) implementation of the POET-X
+ * orthogonal-equivalence linear layer.
+ *
+ * The layer (POET abstract: every weight is W = R W0 P with R, P learnable orthogonal
+ * and W0 fixed and random; POET-X technical summary, section 2):
+ *
+ *     y = (Pi_R^T G_R Pi_R) W0 (Pi_P^T G_P Pi_P) x
+ *
+ *   - G_P, G_R are block-diagonal with b x b blocks built by the Cayley-Neumann
+ *     parameterisation (section 2.4) from packed upper-triangular parameters theta;
+ *   - Pi_P, Pi_R are fixed random permutations applied through index maps, never as
+ *     matrices (section 2.2, permutation acceleration);
+ *   - the inner two permutations are merged once into W0' = Pi_R W0 Pi_P^T (section
+ *     2.2, permutation reduction), so a token row is processed input-centrically
+ *     (section 2.1) as
+ *         U = X[:, p_P];  V_j = U_j G_P,j^T;  W = V W0'^T;  Z_j = W_j G_R,j^T;
+ *         Y[:, p_R[i]] = Z[:, i]
+ *     and R W0 P is never formed.
+ *
+ * Conventions (the pages leave them open; these are the readings this library uses)
+ *   permutation   int32 vector p; (Pi x)_i = x[p[i]]; inverse inv[p[i]] = i.
+ *   blocks        block j covers coordinates [j*b, (j+1)*b) of the permuted space;
+ *                 n % b == 0 and m % b == 0.
+ *   theta         [nblk, b(b-1)/2] fp32, strict upper triangle row-major per block:
+ *                 idx(i,j) = i*b - i*(i+1)/2 + (j-i-1) for i < j; Q_ij = theta,
+ *                 Q_ji = -theta, Q_ii = 0.
+ *   CNP           G = (I + Q)(I + Q + ... + Q^k) = I + 2(Q + ... + Q^k) + Q^(k+1).
+ *   layouts       row-major: X [T, n], Y [T, m], W0 and W0' [m, n] (out x in),
+ *                 G [nblk, b, b], dG [nblk, b, b].
+ *   W0            frozen: the backward returns dX and dG (and, through
+ *                 poetx_cnp_bwd, dtheta) but no dW0.
+ *
+ * Precision
+ *   POETX_F32   everything fp32 (SIMT FFMA kernels).
+ *   POETX_BF16  activations, W0, W0' and G operands bf16 (tcgen05 tensor cores, fp32
+ *               accumulation in TMEM); theta, CNP, dG and dtheta fp32.  V, W, Z, dW,
+ *               dV, dU intermediates are stored in bf16.  Supported b: 128, 256, 512.
+ *
+ * Memory and streams
+ *   All pointers marked "device" are caller-owned device memory; the library never
+ *   allocates.  Scratch comes from (ws, ws_bytes); the *_workspace() queries return
+ *   the bytes a call needs.  Every device pointer must be 16-byte aligned.  All work is
+ *   enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *
+ * Errors
+ *   Every call returns a poetx_status.  Arguments are validated before anything is
+ *   launched; a failed validation launches nothing.  poetx_last_error() gives detail
+ *   text for the calling thread.  Launch failures map to POETX_ERR_CUDA.  Kernels that
+ *   wait on barriers give up after a time limit, record POETX_ERR_TIMEOUT in a device
+ *   flag and return; poetx_device_status() reads (and clears) that flag.
+ */
+#ifndef POETX_H
+#define POETX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum poetx_status {
+  POETX_OK = 0,
+  POETX_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad flag */
+  POETX_ERR_SHAPE = 2,       /* n % b or m % b nonzero, unsupported b or k */
+  POETX_ERR_DTYPE = 3,       /* dtype not POETX_F32 / POETX_BF16 */
+  POETX_ERR_ALIGN = 4,       /* a device pointer is not 16-byte aligned */
+  POETX_ERR_WORKSPACE = 5,   /* ws_bytes below what the call needs */
+  POETX_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+  POETX_ERR_TIMEOUT = 7      /* a kernel's bounded barrier wait ran out */
+} poetx_status;
+
+enum { POETX_F32 = 0, POETX_BF16 = 1 };
+
+/* Short description of a status code (static string). */
+const char* poetx_status_string(int status);
+
+/* Detail text of the last failed call on this thread ("" if none). */
+const char* poetx_last_error(void);
+
+/* Library version string. */
+const char* poetx_version(void);
+
+/*
+ * Seeded random permutation of {0..n-1} and its inverse, in HOST memory.
+ * POET-X section 2.2: the orthogonal factors carry fixed random permutations that are
+ * applied by index maps.  Generator: SplitMix64 (Steele, Lea & Flood 2014) from `seed`,
+ * Durstenfeld Fisher-Yates for i = n-1..1 with j = floor(r * (i+1) / 2^64).
+ *   perm, inv: caller-owned host arrays of n int32 (inv may be NULL).
+ *   Errors: POETX_ERR_INVALID_ARG if n < 0 or perm is NULL with n > 0.
+ */
+int poetx_make_perm(uint64_t seed, int32_t n, int32_t* perm, int32_t* inv);
+
+/*
+ * Permutation reduction (POET-X section 2.2): W0' = Pi_R W0 Pi_P^T, i.e.
+ * W0p[i, j] = W0[perm_R[i], perm_P[j]].  Run once per outer iteration.
+ *   W0   device [m, n] (dtype), read.      W0p  device [m, n] (dtype), written.
+ *   perm_R device int32 [m], perm_P device int32 [n].
+ *   Bit-exact copy.  Errors: INVALID_ARG, DTYPE, ALIGN, CUDA.
+ */
+int poetx_merge_perm(const void* W0, void* W0p, int32_t m, int32_t n, const int32_t* perm_R,
+                     const int32_t* perm_P, int dtype, void* stream);
+
+/*
+ * Index-map permutation of the columns of a row-major matrix (POET-X section 2.2,
+ * permutation acceleration): out[t, i] = in[t, idx[i]] for t < rows, i < cols.
+ * With idx = perm this applies Pi to every row; with idx = inv it applies Pi^T.
+ *   in, out device [rows, cols] (dtype), distinct buffers.  idx device int32 [cols].
+ *   Bit-exact.  Errors: INVALID_ARG, DTYPE, ALIGN, CUDA.
+ */
+int poetx_permute_cols(const void* in, void* out, const int32_t* idx, int32_t rows, int32_t cols,
+                       int dtype, void* stream);
+
+/*
+ * Scratch bytes needed by poetx_cnp_fwd / poetx_cnp_bwd for nblk blocks of size b with
+ * Neumann order k (the calls also accept less, down to one block's worth, and then work
+ * through the blocks in more chunks).  Returns 0 for invalid arguments.
+ */
+size_t poetx_cnp_workspace(int32_t nblk, int32_t b, int32_t k);
+
+/*
+ * Cayley-Neumann forward (POET-X section 2.4): for every block,
+ *   Q = skew(theta),  G = (I + Q)(I + Q + ... + Q^k).
+ *   theta   device fp32 [nblk, b(b-1)/2], read.
+ *   G       device fp32 [nblk, b, b], written.
+ *   G_bf16  device bf16 [nblk, b, b], written when non-NULL (the MMA operand copy,
+ *           round-to-nearest-even of G).
+ *   1 <= b <= 1024, 1 <= k <= 16.   fp32 throughout (SIMT FFMA).
+ *   Errors: INVALID_ARG, SHAPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b, int32_t k,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Cayley-Neumann backward (POET-X section 2.4, backward optimised the same way as the
+ * forward): dtheta = d<dG, G(theta)>/dtheta for the truncated polynomial as computed,
+ *   dtheta_idx(i,j) = dQ_ij - dQ_ji.
+ *   theta   device fp32 [nblk, b(b-1)/2], read.   dG device fp32 [nblk, b, b], read.
+ *   dtheta  device fp32 [nblk, b(b-1)/2], written (overwritten, not accumulated).
+ *   Errors: INVALID_ARG, SHAPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nblk, int32_t b,
+                  int32_t k, void* ws, size_t ws_bytes, void* stream);
+
+/* Shape, precision and index maps of one POET-X linear (index maps in device memory). */
+typedef struct poetx_linear_desc {
+  int32_t T;              /* tokens (rows of X and Y), >= 0 */
+  int32_t n;              /* input features */
+  int32_t m;              /* output features */
+  int32_t b;              /* block size of G_P and G_R */
+  int32_t dtype;          /* POETX_F32 or POETX_BF16 */
+  const int32_t* perm_P;  /* device int32 [n] */
+  const int32_t* inv_P;   /* device int32 [n] */
+  const int32_t* perm_R;  /* device int32 [m] */
+  const int32_t* inv_R;   /* device int32 [m] */
+} poetx_linear_desc;
+
+/* Scratch bytes of poetx_linear_fwd / poetx_linear_bwd.  The flags say which of the
+ * optional save buffers the call will get (a missing one is kept in scratch or
+ * recomputed).  Returns 0 for an invalid descriptor. */
+size_t poetx_linear_fwd_workspace(const poetx_linear_desc* d, int has_save_u, int has_save_w);
+size_t poetx_linear_bwd_workspace(const poetx_linear_desc* d, int has_save_u, int has_save_w);
+
+/*
+ * POET-X linear forward, input-centric with two index-map permutations.
+ *   x      device [T, n] (dtype), read.
+ *   G_P    device [n/b, b, b] (dtype: fp32 for POETX_F32, bf16 for POETX_BF16), read.
+ *   G_R    device [m/b, b, b] (same), read.
+ *   W0p    device [m, n] (dtype), the merged weight from poetx_merge_perm, read.
+ *   y      device [T, m] (dtype), written.
+ *   save_u device [T, n] or NULL: receives U = X[:, p_P] for the backward.
+ *   save_w device [T, m] or NULL: receives W = V W0'^T for the backward (POET-Xfast);
+ *          NULL together with NULL in the backward gives the recompute mode (POET-Xmem).
+ *   T = 0 is a no-op.  Errors: INVALID_ARG, SHAPE, DTYPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_linear_fwd(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
+                     const void* W0p, void* y, void* save_u, void* save_w, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * POET-X linear backward for the loss gradient dy (W0' frozen):
+ *   dZ = dY[:, p_R]; dW_j = dZ_j G_R,j; dG_R,j = dZ_j^T W_j; dV = dW W0';
+ *   dU_j = dV_j G_P,j; dG_P,j = dV_j^T U_j; dX[:, p_P[i]] = dU[:, i].
+ *   x, dy        device [T, n], [T, m] (dtype), read.
+ *   G_P, G_R, W0p  as in the forward, read.
+ *   save_u, save_w the forward's save buffers, or NULL to recompute U (a gather) and
+ *                W (block product + W0' GEMM) inside the call.
+ *   dx           device [T, n] (dtype), written.
+ *   dG_P, dG_R   device fp32 [n/b, b, b], [m/b, b, b]; overwritten when accumulate = 0,
+ *                added to when accumulate = 1 (micro-batch accumulation; dG is linear in
+ *                the tokens).  The token sums are reduced in a fixed order (no float
+ *                atomics), so results are identical from run to run.
+ *   Errors: INVALID_ARG, SHAPE, DTYPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, const void* G_P,
+                     const void* G_R, const void* W0p, const void* save_u, const void* save_w,
+                     void* dx, float* dG_P, float* dG_R, int accumulate, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * Reads and clears the device-side error flag that kernels with bounded barrier waits
+ * set on a timeout.  Synchronises the given stream first.  Returns POETX_OK or
+ * POETX_ERR_TIMEOUT (or POETX_ERR_CUDA if the synchronisation itself failed).
+ */
+int poetx_device_status(void* stream);
+
+/*
+ * Launch accounting and per-kernel timing.
+ *   poetx_launch_count() counts every kernel launch the library has made.
+ *   poetx_profile_begin(name) starts bracketing every launch of the kernel family
+ *   `name` ("gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm", ...) with
+ *   CUDA events on the launch stream (NULL or "" turns this off); poetx_profile_end()
+ *   synchronises those events and reports the number of bracketed launches and their
+ *   summed device time in milliseconds.  Events come from a fixed pool of 4096 pairs.
+ */
+uint64_t poetx_launch_count(void);
+int poetx_profile_begin(const char* name);
+int poetx_profile_end(int32_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POETX_H */

@@ -298,3 +298,28 @@ def full_step(x, W0, theta_P, theta_R, dy, perm_P, perm_R, b, k):
     dth_R = cnp_backward(theta_R, dG_R, b, k)
     return dict(W0p=W0p, G_P=G_P, G_R=G_R, y=Y, dx=dX, dG_P=dG_P, dG_R=dG_R,
                 dtheta_P=dth_P, dtheta_R=dth_R)
+
+
+def layer_block_grads(x, dy, W0p, G_P, G_R, perm_P, perm_R, j_R, j_P):
+    """dG_R,j_R and dG_P,j_P over all tokens, by their definitions, without forming the
+    other blocks' gradients (for spot checks at full size):
+        dG_R,j = dZ_j^T W_j   with W_j = V W0'[j-block rows]^T, V_i = U_i G_P,i^T
+        dG_P,j = dV_j^T U_j   with dV_j = dW W0'[:, j-block],  dW_i = dZ_i G_R,i
+    """
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    W0p = np.asarray(W0p, dtype=np.float64)
+    G_P = np.asarray(G_P, dtype=np.float64)
+    G_R = np.asarray(G_R, dtype=np.float64)
+    b = G_P.shape[1]
+    U = x[:, perm_P]
+    V = _block_apply(U, G_P, transpose=True)
+    rs = slice(j_R * b, (j_R + 1) * b)
+    W_j = V @ W0p[rs, :].T
+    dZ = dy[:, perm_R]
+    dG_R = dZ[:, rs].T @ W_j
+    dW = _block_apply(dZ, G_R, transpose=False)
+    ps = slice(j_P * b, (j_P + 1) * b)
+    dV_j = dW @ W0p[:, ps]
+    dG_P = dV_j.T @ U[:, ps]
+    return dG_P, dG_R

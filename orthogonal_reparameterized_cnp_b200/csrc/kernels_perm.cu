@@ -1,0 +1,140 @@
+// Index-map permutation kernels (POET-X technical summary, section 2.2: permutations are
+// applied by remapping indices, never as permutation matrices).
+//
+// out[r, c] = in[row_idx ? row_idx[r] : r, col_idx[c]]
+//
+// The permutation acts along the contiguous feature axis of a row-major matrix, so a
+// direct gather from global memory would touch a 32-byte sector per element.  Instead
+// each CTA stages whole source rows in shared memory with coalesced 16-byte loads and
+// writes the permuted row with coalesced 16-byte stores; the random access happens only
+// in shared memory.  HBM traffic is exactly one read and one write of the matrix.
+#include <cuda_bf16.h>
+
+#include "poetx_internal.h"
+
+namespace poetx {
+namespace {
+
+constexpr int kGatherThreads = 128;
+constexpr int kMaxSmemRowBytes = 200 * 1024;
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+template <typename E>
+__global__ void __launch_bounds__(kGatherThreads)
+    k_gather_rows_smem(const E* __restrict__ in, E* __restrict__ out,
+                       const int32_t* __restrict__ row_idx, const int32_t* __restrict__ col_idx,
+                       int rows, int cols, int64_t ld_in, int64_t ld_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  E* srow = reinterpret_cast<E*>(smem_raw);
+  constexpr int V = 16 / sizeof(E);  // elements per 16-byte vector
+  const unsigned ucols = (unsigned)cols;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    int sr = row_idx ? row_idx[r] : r;
+    sr = min(max(sr, 0), rows - 1);  // keep the read inside the matrix
+    const E* src = in + (int64_t)sr * ld_in;
+    const bool vin = (cols % V == 0) && ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+    if (vin) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      uint4* d4 = reinterpret_cast<uint4*>(srow);
+      for (int i = threadIdx.x; i < cols / V; i += blockDim.x) d4[i] = ldg_stream(s4 + i);
+    } else {
+      for (int i = threadIdx.x; i < cols; i += blockDim.x) srow[i] = src[i];
+    }
+    __syncthreads();
+    E* dst = out + (int64_t)r * ld_out;
+    const bool vout = (cols % V == 0) && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
+    if (vout) {
+      for (int c0 = threadIdx.x * V; c0 < cols; c0 += blockDim.x * V) {
+        E v[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          unsigned ci = (unsigned)__ldg(col_idx + c0 + e);
+          v[e] = srow[ci < ucols ? ci : ucols - 1];
+        }
+        *reinterpret_cast<uint4*>(dst + c0) = *reinterpret_cast<const uint4*>(v);
+      }
+    } else {
+      for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+        unsigned ci = (unsigned)__ldg(col_idx + c);
+        dst[c] = srow[ci < ucols ? ci : ucols - 1];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Rows too wide for shared memory: gather straight from global memory (L2 absorbs the
+// sector waste; only used beyond ~100k bf16 columns).
+template <typename E>
+__global__ void __launch_bounds__(256)
+    k_gather_rows_direct(const E* __restrict__ in, E* __restrict__ out,
+                         const int32_t* __restrict__ row_idx,
+                         const int32_t* __restrict__ col_idx, int rows, int cols, int64_t ld_in,
+                         int64_t ld_out) {
+  const unsigned ucols = (unsigned)cols;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    int sr = row_idx ? row_idx[r] : r;
+    sr = min(max(sr, 0), rows - 1);
+    const E* src = in + (int64_t)sr * ld_in;
+    E* dst = out + (int64_t)r * ld_out;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+      unsigned ci = (unsigned)__ldg(col_idx + c);
+      dst[c] = src[ci < ucols ? ci : ucols - 1];
+    }
+  }
+}
+
+template <typename E>
+cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
+                        const int32_t* col_idx, int rows, int cols, int64_t ld_in,
+                        int64_t ld_out, cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  const size_t row_bytes = ((size_t)cols * sizeof(E) + 15) & ~size_t(15);
+  const int sms = num_sms();
+  if (row_bytes <= (size_t)kMaxSmemRowBytes) {
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(k_gather_rows_smem<E>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kMaxSmemRowBytes);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    int per_sm = (int)(200 * 1024 / row_bytes);
+    per_sm = per_sm < 1 ? 1 : (per_sm > 16 ? 16 : per_sm);
+    int grid = sms * per_sm;
+    if (grid > rows) grid = rows;
+    begin_launch("permute", s);
+    k_gather_rows_smem<E><<<grid, kGatherThreads, row_bytes, s>>>(
+        static_cast<const E*>(in), static_cast<E*>(out), row_idx, col_idx, rows, cols, ld_in,
+        ld_out);
+    end_launch("permute", s);
+  } else {
+    int grid = sms * 8;
+    if (grid > rows) grid = rows;
+    begin_launch("permute", s);
+    k_gather_rows_direct<E><<<grid, 256, 0, s>>>(static_cast<const E*>(in), static_cast<E*>(out),
+                                                 row_idx, col_idx, rows, cols, ld_in, ld_out);
+    end_launch("permute", s);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gather(const void* in, void* out, const int32_t* row_idx,
+                          const int32_t* col_idx, int rows, int cols, int64_t ld_in,
+                          int64_t ld_out, int elem_bytes, cudaStream_t s) {
+  if (elem_bytes == 2)
+    return gather_impl<uint16_t>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+  return gather_impl<uint32_t>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+}
+
+}  // namespace poetx

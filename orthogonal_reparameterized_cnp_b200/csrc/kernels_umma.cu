@@ -1,0 +1,515 @@
+// tcgen05 (5th-generation tensor core) GEMM for sm_100a, fed by TMA.
+//
+//   D[M x N] = A[M x K] . B[N x K]^T      (bf16 operands, fp32 accumulation in TMEM)
+//
+// used for every dense contraction of the POET-X layer (technical summary sections
+// 2.1-2.3):
+//   * the batched block-diagonal products V_j = U_j G_j^T and dW_j = dZ_j G_j (one batch
+//     entry per b x b block; the sparse block-diagonal matrix is never formed),
+//   * the merged-weight products W = V W0'^T and dV = dW W0',
+//   * the block-gradient contractions dG_j = sum_t g_t^T h_t over tokens, split over the
+//     token axis into fixed partial sums.
+//
+// Structure: one persistent CTA per SM, 192 threads.
+//   warp 0      TMA producer (one lane): A/B k-chunks of 64 into a STAGES-deep smem ring
+//   warp 1      TMEM allocator + MMA issuer (one lane): 4 x (M=128, N=BN, K=16) per chunk
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, convert, store to global
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap the main loop
+// of tile t+1.  Operands may be K-major or MN-major (transposed) in global memory; both
+// are staged with the 128-byte swizzle the UMMA smem descriptors expect.
+//
+// Every mbarrier wait is bounded: after kWaitLimitNs the waiting role records
+// POETX_ERR_TIMEOUT in a device flag and leaves its loop; the CTA then drains its
+// outstanding TMA loads and MMAs (again with bounded waits), frees TMEM and returns.
+// No cluster multicast is used anywhere.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "poetx_internal.h"
+
+namespace poetx {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int kThreads = 192;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+struct Params {
+  int M, N, K, batch, ksplit, kcps, total_kc;
+  int tiles_m, tiles_n, num_items;
+  int a_boff_mn, a_boff_k, b_boff_mn, b_boff_k;
+  void* D;
+  int out_f32;
+  long long ldd, d_boff_col, d_boff, d_split;
+  int* err;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: false after a timeout (flag set) or when another CTA reported a failure.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  unsigned spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 63u) == 0) {
+      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        atomicCAS(err, 0, (int)POETX_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+// Short bounded wait used only while draining after a failure.
+__device__ __noinline__ void mbar_drain_wait(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 100000000ull) return;  // 100 ms
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 layout (version field = 1).
+//   K-major:  rows of 128 B (64 bf16 along K), 8-row core groups 1024 B apart (SBO);
+//             the K=16 slice kk starts kk*32 B into the row (LBO unused, set to 16 B).
+//   MN-major: rows of 128 B (64 bf16 along M/N), one row per K index; 8-K-row groups
+//             1024 B apart (SBO); 64-wide M/N groups LBO bytes apart.
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+__device__ __forceinline__ uint32_t make_idesc() {
+  return (1u << 4)                         // D format: f32
+         | (1u << 7)                       // A format: bf16
+         | (1u << 10)                      // B format: bf16
+         | ((A_MN ? 1u : 0u) << 15)        // A major
+         | ((B_MN ? 1u : 0u) << 16)        // B major
+         | ((uint32_t)(BN >> 3) << 17)     // N
+         | ((uint32_t)(kBM >> 4) << 24);   // M
+}
+
+struct Item {
+  int bz, split, tm, tn;
+};
+__device__ __forceinline__ Item decode(const Params& p, int item) {
+  Item it;
+  it.tm = item % p.tiles_m;
+  int r = item / p.tiles_m;
+  it.tn = r % p.tiles_n;
+  r /= p.tiles_n;
+  it.split = r % p.ksplit;
+  it.bz = r / p.ksplit;
+  return it;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_umma_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t sA = base;                          // STAGES x A_BYTES
+  const uint32_t sB = base + C::STAGES * C::A_BYTES;  // STAGES x B_BYTES
+  const uint32_t sBar = base + C::STAGES * C::STAGE_BYTES;
+  // barrier block: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, tmem slot
+  auto full_bar = [&](int s) { return sBar + 8u * s; };
+  auto empty_bar = [&](int s) { return sBar + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return sBar + 8u * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return sBar + 8u * (2 * C::STAGES + 2 + a); };
+  const uint32_t drain_bar = sBar + 8u * (2 * C::STAGES + 4);
+  const uint32_t tmem_slot = sBar + 8u * (2 * C::STAGES + 5);
+  unsigned char* generic_base = smem_raw + (base - raw);
+  volatile uint32_t* tmem_slot_ptr =
+      reinterpret_cast<volatile uint32_t*>(generic_base + (tmem_slot - base));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot_ptr;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int it = 0;
+    int last_round[8];
+    for (int s = 0; s < 8; ++s) last_round[s] = -1;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.num_items; item += gridDim.x) {
+      const Item w = decode(p, item);
+      const int m0 = w.tm * kBM, n0 = w.tn * BN;
+      const int kc0 = w.split * p.kcps;
+      const int kc1 = min(p.total_kc, kc0 + p.kcps);
+      for (int kc = kc0; kc < kc1; ++kc, ++it) {
+        const int s = it % C::STAGES, r = it / C::STAGES;
+        if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+        last_round[s] = r;
+        const int k = kc * kBK;
+        const uint32_t a_dst = sA + s * C::A_BYTES;
+        const uint32_t b_dst = sB + s * C::B_BYTES;
+        if (!A_MN) {
+          tma_load_2d(a_dst, &tmA, k + w.bz * p.a_boff_k, m0 + w.bz * p.a_boff_mn, full_bar(s));
+        } else {
+          tma_load_2d(a_dst, &tmA, m0 + w.bz * p.a_boff_mn, k + w.bz * p.a_boff_k, full_bar(s));
+          tma_load_2d(a_dst + 8192, &tmA, m0 + 64 + w.bz * p.a_boff_mn, k + w.bz * p.a_boff_k,
+                      full_bar(s));
+        }
+        if (!B_MN) {
+          tma_load_2d(b_dst, &tmB, k + w.bz * p.b_boff_k, n0 + w.bz * p.b_boff_mn, full_bar(s));
+        } else {
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i)
+            tma_load_2d(b_dst + i * 8192, &tmB, n0 + 64 * i + w.bz * p.b_boff_mn,
+                        k + w.bz * p.b_boff_k, full_bar(s));
+        }
+      }
+    }
+    if (!ok) {
+      // make sure no TMA write into this CTA's shared memory is still in flight
+      for (int s = 0; s < C::STAGES; ++s)
+        if (last_round[s] >= 0) mbar_drain_wait(full_bar(s), last_round[s] & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = make_idesc<BN, A_MN, B_MN>();
+    int it = 0, tcount = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.num_items; item += gridDim.x, ++tcount) {
+      const Item w = decode(p, item);
+      const int kc0 = w.split * p.kcps;
+      const int kc1 = min(p.total_kc, kc0 + p.kcps);
+      const int acc = tcount & 1, ra = tcount >> 1;
+      if (!mbar_wait(tempty_bar(acc), (ra & 1) ^ 1, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kc = kc0; kc < kc1; ++kc, ++it) {
+        const int s = it % C::STAGES, r = it / C::STAGES;
+        if (!mbar_wait(full_bar(s), r & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = sA + s * C::A_BYTES;
+        const uint32_t b_addr = sB + s * C::B_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t adesc = A_MN ? make_desc(a_addr + kk * 2048, 8192, 1024)
+                                      : make_desc(a_addr + kk * 32, 16, 1024);
+          const uint64_t bdesc = B_MN ? make_desc(b_addr + kk * 2048, 8192, 1024)
+                                      : make_desc(b_addr + kk * 32, 16, 1024);
+          umma_bf16(d_tmem, adesc, bdesc, idesc, (kc > kc0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(empty_bar(s));  // frees the smem slot once these MMAs have read it
+      }
+      if (!ok) break;
+      umma_commit(tfull_bar(acc));  // accumulator ready for the epilogue
+    }
+    // all MMAs issued by this thread complete before TMEM is released
+    umma_commit(drain_bar);
+    mbar_drain_wait(drain_bar, 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int tcount = 0;
+    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x, ++tcount) {
+      const Item w = decode(p, item);
+      const int acc = tcount & 1, ra = tcount >> 1;
+      // one lane waits so that the warp stays converged for the .sync.aligned loads
+      int ready = 0;
+      if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      const int row = w.tm * kBM + q * 32 + lane;
+      const int n0 = w.tn * BN;
+      const long long dbase = (long long)w.split * p.d_split + (long long)w.bz * p.d_boff +
+                              (long long)row * p.ldd + (long long)w.bz * p.d_boff_col;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), v);
+        tmem_wait_ld();
+        if (row < p.M && n0 + c < p.N) {
+          if (p.out_f32) {
+            float* dst = static_cast<float*>(p.D) + dbase + n0 + c;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<uint4*>(dst + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          } else {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + dbase + n0 + c;
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 o;
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+              o.x = *reinterpret_cast<uint32_t*>(&h0);
+              o.y = *reinterpret_cast<uint32_t*>(&h1);
+              o.z = *reinterpret_cast<uint32_t*>(&h2);
+              o.w = *reinterpret_cast<uint32_t*>(&h3);
+              *reinterpret_cast<uint4*>(dst + j) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const UmmaOperand& op, int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)op.cols, (cuuint64_t)op.rows};
+  cuuint64_t strides[1] = {(cuuint64_t)op.ld * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(op.ptr), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
+                     const char* family, cudaStream_t s) {
+  auto kern = k_umma_gemm<BN, A_MN, B_MN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<BN>::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  begin_launch(family, s);
+  kern<<<grid, kThreads, Cfg<BN>::SMEM_BYTES, s>>>(ma, mb, p);
+  end_launch(family, s);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
+                      bool a_mn, bool b_mn, const char* family, cudaStream_t s) {
+  if (!a_mn && !b_mn) return launch_t<BN, false, false>(ma, mb, p, grid, family, s);
+  if (!a_mn && b_mn) return launch_t<BN, false, true>(ma, mb, p, grid, family, s);
+  if (a_mn && b_mn) return launch_t<BN, true, true>(ma, mb, p, grid, family, s);
+  return launch_t<BN, true, false>(ma, mb, p, grid, family, s);
+}
+
+}  // namespace
+
+int umma_choose_ksplit(int M, int N, int K, int batch) {
+  const int BN = (N % 256 == 0) ? 256 : 128;
+  const int tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN) * batch;
+  const int total_kc = (K + kBK - 1) / kBK;
+  if (total_kc <= 0) return 1;
+  const int sms = num_sms();
+  int want = 1;
+  if (tiles < sms) want = (2 * sms + tiles - 1) / tiles;
+  int max_split = total_kc / 4;  // at least 4 k-chunks (256 along K) per split
+  if (max_split < 1) max_split = 1;
+  if (want > max_split) want = max_split;
+  const int kcps = (total_kc + want - 1) / want;
+  return (total_kc + kcps - 1) / kcps;  // every split non-empty
+}
+
+cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return cudaSuccess;
+  if (g.N % 128 != 0) return cudaErrorInvalidValue;
+  const int BN = (g.N % 256 == 0) ? 256 : 128;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, g.A, g.A.mn_major ? 64 : kBM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, g.B, g.B.mn_major ? 64 : BN)) return cudaErrorInvalidValue;
+  Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.batch = g.batch;
+  p.total_kc = (g.K + kBK - 1) / kBK;
+  if (p.total_kc <= 0) return cudaErrorInvalidValue;
+  int ks = g.ksplit < 1 ? 1 : g.ksplit;
+  if (ks > p.total_kc) ks = p.total_kc;
+  p.kcps = (p.total_kc + ks - 1) / ks;
+  p.ksplit = (p.total_kc + p.kcps - 1) / p.kcps;
+  if (p.ksplit != ks) return cudaErrorInvalidValue;  // caller sized its output for ks splits
+  p.tiles_m = (g.M + kBM - 1) / kBM;
+  p.tiles_n = (g.N + BN - 1) / BN;
+  const long long items = (long long)p.tiles_m * p.tiles_n * p.ksplit * p.batch;
+  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  p.num_items = (int)items;
+  p.a_boff_mn = (int)g.A.boff_mn;
+  p.a_boff_k = (int)g.A.boff_k;
+  p.b_boff_mn = (int)g.B.boff_mn;
+  p.b_boff_k = (int)g.B.boff_k;
+  p.D = g.D;
+  p.out_f32 = g.out_f32;
+  p.ldd = g.ldd;
+  p.d_boff_col = g.d_boff_col;
+  p.d_boff = g.d_boff;
+  p.d_split = g.d_split;
+  p.err = device_error_flag();
+  int grid = num_sms();
+  if (grid > p.num_items) grid = p.num_items;
+  if (BN == 256) return launch_bn<256>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, family, s);
+  return launch_bn<128>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, family, s);
+}
+
+}  // namespace poetx

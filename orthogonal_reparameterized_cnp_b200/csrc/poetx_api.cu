@@ -1,0 +1,814 @@
+// C ABI of libpoetx: argument validation, the permutation generator, scratch layout and
+// the launch sequences of the POET-X layer (POET-X technical summary, section 2).
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <initializer_list>
+#include <utility>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "poetx_internal.h"
+
+namespace poetx {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+int fail(int status, const std::string& msg) {
+  g_last_error = msg;
+  return status;
+}
+int cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return POETX_ERR_CUDA;
+}
+
+// Device-side error flag: kernels with bounded waits record POETX_ERR_TIMEOUT here.
+__device__ int g_device_error = 0;
+
+int* device_error_flag() {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 148;
+  }
+  return cache[dev];
+}
+
+// ------------------------------------------------------------------ launch accounting
+static std::atomic<uint64_t> g_launches{0};
+static std::mutex g_prof_mu;
+static std::string g_prof_family;
+static bool g_prof_on = false;
+static constexpr int kEventPairs = 4096;
+static std::vector<cudaEvent_t> g_ev_start, g_ev_stop;
+static int g_prof_used = 0;
+
+void begin_launch(const char* family, cudaStream_t s) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_prof_on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (g_prof_on && g_prof_family == family && g_prof_used < kEventPairs)
+    cudaEventRecord(g_ev_start[g_prof_used], s);
+}
+void end_launch(const char* family, cudaStream_t s) {
+  if (!g_prof_on) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (g_prof_on && g_prof_family == family && g_prof_used < kEventPairs)
+    cudaEventRecord(g_ev_stop[g_prof_used++], s);
+}
+
+// ------------------------------------------------------------------ helpers
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+size_t align_up(size_t v, size_t a = 256) { return (v + a - 1) / a * a; }
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+#define POETX_CUDA(call, what)                 \
+  do {                                         \
+    cudaError_t e_ = (call);                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+// ---- CNP polynomial coefficients ---------------------------------------------------
+// G = sum_{i=0..k+1} c_i Q^i with c = (1, 2, ..., 2, 1).  With S = Q^2 (symmetric):
+//   G = E(S) + Q F(S),  E = sum_j e_j S^j (e_j = c_{2j}),  F = sum_j f_j S^j (f_j = c_{2j+1})
+// E is symmetric and Q F skew, so G's upper triangle gives both halves.
+struct CnpPoly {
+  int d;          // highest power of S needed: floor((k+1)/2)
+  float e[10], f[10];
+};
+CnpPoly cnp_poly(int k) {
+  CnpPoly p;
+  p.d = (k + 1) / 2;
+  for (int j = 0; j <= p.d; ++j) {
+    auto c = [&](int i) -> float {
+      if (i < 0 || i > k + 1) return 0.f;
+      return (i == 0 || i == k + 1) ? 1.f : 2.f;
+    };
+    p.e[j] = c(2 * j);
+    p.f[j] = c(2 * j + 1);
+  }
+  return p;
+}
+
+// Matrices held per block in the CNP scratch (b x b fp32 each).
+int cnp_mats(int k, bool backward) {
+  const int d = (k + 1) / 2;
+  // forward: Q, P_1..P_d, F'
+  // backward adds: D, N_1..N_d, Pm, R, R2, T, T2, A
+  return backward ? 2 * d + 9 : d + 2;
+}
+
+constexpr size_t kCnpChunkTarget = 256ull << 20;  // bytes per scratch matrix
+
+size_t cnp_per_block(int b, int k, bool backward) {
+  return (size_t)cnp_mats(k, backward) * align_up((size_t)b * b * 4);
+}
+
+int cnp_validate(const void* theta, const void* out, int nblk, int b, int k) {
+  if (nblk < 0) return fail(POETX_ERR_INVALID_ARG, "nblk must be >= 0");
+  if (b < 1 || b > 1024) return fail(POETX_ERR_SHAPE, "block size b must be in [1, 1024]");
+  if (k < 1 || k > 16) return fail(POETX_ERR_SHAPE, "Neumann order k must be in [1, 16]");
+  if (nblk > 0 && (!theta || !out)) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  return POETX_OK;
+}
+
+// Runs fn(first_block, count, scratch) over chunks of blocks that fit in ws.
+template <typename Fn>
+int cnp_chunks(int nblk, int b, int k, bool backward, void* ws, size_t ws_bytes, Fn fn) {
+  const size_t per = cnp_per_block(b, k, backward);
+  size_t cap = ws_bytes / per;
+  if (cap < 1) return fail(POETX_ERR_WORKSPACE, "CNP scratch smaller than one block needs");
+  if (!ws) return fail(POETX_ERR_INVALID_ARG, "null scratch");
+  if (!aligned16(ws)) return fail(POETX_ERR_ALIGN, "scratch must be 16-byte aligned");
+  const size_t per_mat_cap = kCnpChunkTarget / ((size_t)b * b * 4);
+  if (cap > per_mat_cap && per_mat_cap >= 1) cap = per_mat_cap;
+  for (int b0 = 0; b0 < nblk; b0 += (int)cap) {
+    int cnt = nblk - b0 < (int)cap ? nblk - b0 : (int)cap;
+    int st = fn(b0, cnt);
+    if (st != POETX_OK) return st;
+  }
+  return POETX_OK;
+}
+
+SgemmArgs sq_gemm(const float* A, int tA, const float* B, int tB, float* C, int nb, int b,
+                  int mode) {
+  SgemmArgs g;
+  const int64_t bb = (int64_t)b * b;
+  g.A = A; g.lda = b; g.sA = bb; g.transA = tA;
+  g.B = B; g.ldb = b; g.sB = bb; g.transB = tB;
+  g.C = C; g.ldc = b; g.sC = bb;
+  g.M = b; g.N = b; g.K = b; g.batch = nb;
+  g.mode = mode;
+  return g;
+}
+
+}  // namespace
+}  // namespace poetx
+
+using namespace poetx;
+
+// ======================================================================= C ABI
+extern "C" {
+
+const char* poetx_status_string(int status) {
+  switch (status) {
+    case POETX_OK: return "ok";
+    case POETX_ERR_INVALID_ARG: return "invalid argument";
+    case POETX_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case POETX_ERR_DTYPE: return "unsupported dtype";
+    case POETX_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case POETX_ERR_WORKSPACE: return "workspace too small";
+    case POETX_ERR_CUDA: return "CUDA error";
+    case POETX_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* poetx_last_error(void) { return g_last_error.c_str(); }
+
+const char* poetx_version(void) { return "poetx 0.1.0 (sm_100a)"; }
+
+int poetx_make_perm(uint64_t seed, int32_t n, int32_t* perm, int32_t* inv) {
+  if (n < 0) return fail(POETX_ERR_INVALID_ARG, "n must be >= 0");
+  if (n > 0 && !perm) return fail(POETX_ERR_INVALID_ARG, "perm is NULL");
+  for (int32_t i = 0; i < n; ++i) perm[i] = i;
+  // SplitMix64 stream feeding Durstenfeld's Fisher-Yates; bounded draw by the high word
+  // of a 64x64 -> 128-bit product (Lemire's multiply-shift, no rejection).
+  uint64_t state = seed;
+  for (int32_t i = n - 1; i >= 1; --i) {
+    state += 0x9E3779B97F4A7C15ull;
+    uint64_t z = state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const uint64_t j = (uint64_t)(((unsigned __int128)z * (unsigned __int128)(uint64_t)(i + 1)) >> 64);
+    int32_t t = perm[i];
+    perm[i] = perm[j];
+    perm[j] = t;
+  }
+  if (inv)
+    for (int32_t i = 0; i < n; ++i) inv[perm[i]] = i;
+  return POETX_OK;
+}
+
+int poetx_merge_perm(const void* W0, void* W0p, int32_t m, int32_t n, const int32_t* perm_R,
+                     const int32_t* perm_P, int dtype, void* stream) {
+  if (m < 0 || n < 0) return fail(POETX_ERR_INVALID_ARG, "negative size");
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!W0 || !W0p || !perm_R || !perm_P) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (W0 == W0p) return fail(POETX_ERR_INVALID_ARG, "W0 and W0p must be distinct");
+  if (!aligned16(W0) || !aligned16(W0p) || !aligned16(perm_R) || !aligned16(perm_P))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  POETX_CUDA(launch_gather(W0, W0p, perm_R, perm_P, m, n, n, n, dtype == POETX_BF16 ? 2 : 4, s),
+             "merge_perm launch");
+  return POETX_OK;
+}
+
+int poetx_permute_cols(const void* in, void* out, const int32_t* idx, int32_t rows, int32_t cols,
+                       int dtype, void* stream) {
+  if (rows < 0 || cols < 0) return fail(POETX_ERR_INVALID_ARG, "negative size");
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (rows == 0 || cols == 0) return POETX_OK;
+  if (!in || !out || !idx) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (in == out) return fail(POETX_ERR_INVALID_ARG, "in and out must be distinct");
+  if (!aligned16(in) || !aligned16(out) || !aligned16(idx))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  POETX_CUDA(launch_gather(in, out, nullptr, idx, rows, cols, cols, cols,
+                           dtype == POETX_BF16 ? 2 : 4, static_cast<cudaStream_t>(stream)),
+             "permute launch");
+  return POETX_OK;
+}
+
+size_t poetx_cnp_workspace(int32_t nblk, int32_t b, int32_t k) {
+  if (nblk < 0 || b < 1 || b > 1024 || k < 1 || k > 16) return 0;
+  if (nblk == 0) return 0;
+  const size_t per_mat_cap = kCnpChunkTarget / ((size_t)b * b * 4);
+  size_t chunk = (size_t)nblk;
+  if (per_mat_cap >= 1 && chunk > per_mat_cap) chunk = per_mat_cap;
+  return chunk * cnp_per_block(b, k, true);
+}
+
+}  // extern "C"
+
+namespace {
+
+// P_1 = Q Q, P_p = S P_{p-1} (all symmetric), and F' = F - f_0 I = sum_{j>=1} f_j P_j
+// produced as the second output of the last power product.
+int cnp_powers(const float* Q, std::vector<float*>& Pw, float* Fp, const CnpPoly& P, int nb,
+               int b, cudaStream_t s) {
+  const int d = P.d;
+  for (int j = 1; j <= d; ++j) {
+    SgemmArgs g = (j == 1) ? sq_gemm(Q, 0, Q, 0, Pw[1], nb, b, SG_SYM)
+                           : sq_gemm(Pw[1], 0, Pw[j - 1], 0, Pw[j], nb, b, SG_SYM);
+    if (j == d) {
+      g.C2 = Fp;
+      g.alpha_c2 = P.f[d];
+      for (int t = 1; t < d; ++t) {
+        g.add[g.nadd] = Pw[t];
+        g.addc[g.nadd] = 0.f;
+        g.addc2[g.nadd] = P.f[t];
+        ++g.nadd;
+      }
+    }
+    POETX_CUDA(launch_sgemm(g, s), "cnp power product");
+  }
+  return POETX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b, int32_t k,
+                  void* ws, size_t ws_bytes, void* stream) {
+  int st = cnp_validate(theta, G, nblk, b, k);
+  if (st != POETX_OK) return st;
+  if (nblk == 0) return POETX_OK;
+  if (!aligned16(theta) || !aligned16(G) || (G_bf16 && !aligned16(G_bf16)))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CnpPoly P = cnp_poly(k);
+  const int d = P.d;
+  const int64_t bb = (int64_t)b * b, ntri = (int64_t)b * (b - 1) / 2;
+  return cnp_chunks(nblk, b, k, false, ws, ws_bytes, [&](int b0, int nb) -> int {
+    Carve cv(ws);
+    float* Q = static_cast<float*>(cv.take(bb * 4 * nb));
+    std::vector<float*> Pw(d + 1, nullptr);
+    for (int j = 1; j <= d; ++j) Pw[j] = static_cast<float*>(cv.take(bb * 4 * nb));
+    float* Fp = static_cast<float*>(cv.take(bb * 4 * nb));
+    POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
+    int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
+    if (st2 != POETX_OK) return st2;
+    // G = E + Q F with E = e_0 I + sum_j e_j P_j (symmetric) and Q F = Q F' + f_0 Q (skew):
+    // only upper tiles are multiplied; G_ji = E_ij - (QF)_ij.
+    SgemmArgs g = sq_gemm(Q, 0, Fp, 0, G + b0 * bb, nb, b, SG_SYMSKEW);
+    g.C_bf16 = G_bf16 ? static_cast<void*>(static_cast<uint16_t*>(G_bf16) + b0 * bb) : nullptr;
+    g.diag = P.e[0];
+    for (int j = 1; j <= d; ++j) {
+      g.add[g.nadd] = Pw[j];
+      g.addc[g.nadd] = P.e[j];
+      ++g.nadd;
+    }
+    g.skew_add = Q;
+    g.skew_c = P.f[0];
+    POETX_CUDA(launch_sgemm(g, s), "cnp G");
+    return POETX_OK;
+  });
+}
+
+int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nblk, int32_t b,
+                  int32_t k, void* ws, size_t ws_bytes, void* stream) {
+  int st = cnp_validate(theta, dtheta, nblk, b, k);
+  if (st != POETX_OK) return st;
+  if (nblk == 0) return POETX_OK;
+  if (!dG) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(theta) || !aligned16(dG) || !aligned16(dtheta))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const CnpPoly P = cnp_poly(k);
+  const int d = P.d;
+  const int64_t bb = (int64_t)b * b, ntri = (int64_t)b * (b - 1) / 2;
+  return cnp_chunks(nblk, b, k, true, ws, ws_bytes, [&](int b0, int nb) -> int {
+    Carve cv(ws);
+    auto mat = [&]() { return static_cast<float*>(cv.take(bb * 4 * nb)); };
+    float* Q = mat();
+    std::vector<float*> Pw(d + 1, nullptr), Nw(d + 1, nullptr);
+    for (int j = 1; j <= d; ++j) Pw[j] = mat();
+    float* Fp = mat();
+    float* D = mat();
+    for (int j = 1; j <= d; ++j) Nw[j] = mat();
+    float* Pm = mat();
+    float* R = mat();
+    float* R2 = mat();
+    float* T = mat();
+    float* T2 = mat();
+    float* A = mat();
+    const float* dg = dG + b0 * bb;
+    POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
+    int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
+    if (st2 != POETX_OK) return st2;
+    // D = Q dG; the adjoint reaching F is Q^T dG = -D.
+    POETX_CUDA(launch_sgemm(sq_gemm(Q, 0, dg, 0, D, nb, b, SG_FULL), s), "cnp D");
+    // N_j = M_j + M_j^T with M_j = e_j dG - f_j D  (upstream of S^j through E and F)
+    for (int j0 = 1; j0 <= d; j0 += 4) {
+      const int cnt = (d - j0 + 1) < 4 ? (d - j0 + 1) : 4;
+      const float* X[2] = {dg, D};
+      float* outs[4];
+      float coef[8];
+      for (int t = 0; t < cnt; ++t) {
+        outs[t] = Nw[j0 + t];
+        coef[t * 2 + 0] = P.e[j0 + t];
+        coef[t * 2 + 1] = -P.f[j0 + t];
+      }
+      POETX_CUDA(launch_symcomb(X, 2, outs, cnt, coef, nb, b, s), "cnp N");
+    }
+    // Y = dS + dS^T = sum_j sum_a S^a N_j S^(j-1-a), by a Horner recursion from the top
+    const float* Y = Nw[1];
+    if (d >= 2) {
+      const float* S = Pw[1];
+      SgemmArgs g = sq_gemm(Nw[d], 0, S, 0, Pm, nb, b, SG_FULL);  // Pm = N_d S
+      if (d >= 3) {  // R_{d-2} = N_{d-1} + Pm
+        g.C2 = R;
+        g.alpha_c2 = 1.f;
+        g.add[0] = Nw[d - 1];
+        g.addc[0] = 0.f;
+        g.addc2[0] = 1.f;
+        g.nadd = 1;
+      }
+      POETX_CUDA(launch_sgemm(g, s), "cnp N_d S");
+      {  // T_{d-2} = N_{d-1} + Pm + Pm^T
+        const float* X[2] = {Nw[d - 1], Pm};
+        float* outs[1] = {T};
+        float coef[2] = {0.5f, 1.f};
+        POETX_CUDA(launch_symcomb(X, 2, outs, 1, coef, nb, b, s), "cnp T");
+      }
+      float* Rc = R;
+      float* Rn = R2;
+      float* Tc = T;
+      float* Tn = T2;
+      for (int a = d - 3; a >= 0; --a) {
+        // R_a = N_{a+1} + R_{a+1} S
+        SgemmArgs gr = sq_gemm(Rc, 0, S, 0, Rn, nb, b, SG_FULL);
+        gr.add[0] = Nw[a + 1];
+        gr.addc[0] = 1.f;
+        gr.nadd = 1;
+        POETX_CUDA(launch_sgemm(gr, s), "cnp R");
+        // T_a = R_a + S T_{a+1}  (symmetric: upper tiles + mirror)
+        SgemmArgs gt = sq_gemm(S, 0, Tc, 0, Tn, nb, b, SG_SYM);
+        gt.add[0] = Rn;
+        gt.addc[0] = 1.f;
+        gt.nadd = 1;
+        POETX_CUDA(launch_sgemm(gt, s), "cnp T");
+        std::swap(Rc, Rn);
+        std::swap(Tc, Tn);
+      }
+      Y = Tc;
+    }
+    // A = f_0 dG + dG F' - Y Q  (skew part of A gives dtheta)
+    SgemmArgs ga = sq_gemm(dg, 0, Fp, 0, A, nb, b, SG_FULL);
+    ga.A2 = Y; ga.lda2 = b; ga.sA2 = bb;
+    ga.B2 = Q; ga.ldb2 = b; ga.sB2 = bb;
+    ga.K2 = b;
+    ga.alpha2 = -1.f;
+    ga.add[0] = dg;
+    ga.addc[0] = P.f[0];
+    ga.nadd = 1;
+    POETX_CUDA(launch_sgemm(ga, s), "cnp A");
+    POETX_CUDA(launch_pack_skew(A, dtheta + b0 * ntri, nb, b, s), "cnp pack");
+    return POETX_OK;
+  });
+}
+
+}  // extern "C"
+
+// ======================================================================= linear layer
+namespace {
+
+int linear_validate(const poetx_linear_desc* d) {
+  if (!d) return fail(POETX_ERR_INVALID_ARG, "descriptor is NULL");
+  if (d->T < 0 || d->n < 1 || d->m < 1 || d->b < 1)
+    return fail(POETX_ERR_INVALID_ARG, "sizes must be T >= 0 and n, m, b >= 1");
+  if (d->dtype != POETX_F32 && d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (d->n % d->b || d->m % d->b) return fail(POETX_ERR_SHAPE, "n and m must be multiples of b");
+  if (d->dtype == POETX_BF16 && d->b != 128 && d->b != 256 && d->b != 512)
+    return fail(POETX_ERR_SHAPE, "bf16 layer supports b in {128, 256, 512}");
+  if (d->dtype == POETX_F32 && d->b > 1024) return fail(POETX_ERR_SHAPE, "b must be <= 1024");
+  if (!d->perm_P || !d->inv_P || !d->perm_R || !d->inv_R)
+    return fail(POETX_ERR_INVALID_ARG, "index maps must be given");
+  if (!aligned16(d->perm_P) || !aligned16(d->inv_P) || !aligned16(d->perm_R) ||
+      !aligned16(d->inv_R))
+    return fail(POETX_ERR_ALIGN, "index maps must be 16-byte aligned");
+  return POETX_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(p)) return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  }
+  return POETX_OK;
+}
+
+int check_opt(const void* p) {
+  if (p && !aligned16(p)) return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  return POETX_OK;
+}
+
+struct FwdLayout {
+  size_t U, V, W, Z, total;
+};
+FwdLayout fwd_layout(const poetx_linear_desc* d, int has_u, int has_w) {
+  const size_t es = d->dtype == POETX_BF16 ? 2 : 4;
+  const size_t tn = (size_t)d->T * d->n * es, tm = (size_t)d->T * d->m * es;
+  FwdLayout L;
+  L.U = has_u ? 0 : align_up(tn);
+  L.V = align_up(tn);
+  L.W = has_w ? 0 : align_up(tm);
+  L.Z = align_up(tm);
+  L.total = L.U + L.V + L.W + L.Z;
+  return L;
+}
+
+struct BwdLayout {
+  size_t U, Vr, Wr, dZ, dW, dV, dU, partR, partP, total;
+  int ksR, ksP;
+};
+BwdLayout bwd_layout(const poetx_linear_desc* d, int has_u, int has_w) {
+  const size_t es = d->dtype == POETX_BF16 ? 2 : 4;
+  const size_t tn = (size_t)d->T * d->n * es, tm = (size_t)d->T * d->m * es;
+  const int nP = d->n / d->b, nR = d->m / d->b;
+  BwdLayout L;
+  L.U = has_u ? 0 : align_up(tn);
+  L.Vr = has_w ? 0 : align_up(tn);
+  L.Wr = has_w ? 0 : align_up(tm);
+  L.dZ = align_up(tm);
+  L.dW = align_up(tm);
+  L.dV = align_up(tn);
+  L.dU = align_up(tn);
+  L.ksR = L.ksP = 1;
+  L.partR = L.partP = 0;
+  if (d->dtype == POETX_BF16 && d->T > 0) {
+    L.ksR = umma_choose_ksplit(d->b, d->b, d->T, nR);
+    L.ksP = umma_choose_ksplit(d->b, d->b, d->T, nP);
+    L.partR = align_up((size_t)L.ksR * nR * d->b * d->b * 4);
+    L.partP = align_up((size_t)L.ksP * nP * d->b * d->b * 4);
+  }
+  L.total = L.U + L.Vr + L.Wr + L.dZ + L.dW + L.dV + L.dU + L.partR + L.partP;
+  return L;
+}
+
+// ---- fp32 building blocks (SIMT) --------------------------------------------------
+// out[:, j*b:(j+1)*b] = in[:, j*b:(j+1)*b] . (G_j^T if transposeG else G_j)
+cudaError_t f32_blockdiag(const float* in, const float* G, float* out, int T, int width, int b,
+                          bool transposeG, cudaStream_t s) {
+  SgemmArgs g;
+  g.A = in; g.lda = width; g.sA = b; g.transA = 0;
+  g.B = G; g.ldb = b; g.sB = (int64_t)b * b; g.transB = transposeG ? 1 : 0;
+  g.C = out; g.ldc = width; g.sC = b;
+  g.M = T; g.N = b; g.K = b; g.batch = width / b;
+  return launch_sgemm(g, s);
+}
+// dG_j (+)= A_j^T B_j over the token axis, A, B [T, width] row-major
+cudaError_t f32_block_grad(const float* A, const float* B, float* dG, int T, int width, int b,
+                           int accumulate, cudaStream_t s) {
+  SgemmArgs g;
+  g.A = A; g.lda = width; g.sA = b; g.transA = 1;
+  g.B = B; g.ldb = width; g.sB = b; g.transB = 0;
+  g.C = dG; g.ldc = b; g.sC = (int64_t)b * b;
+  g.M = b; g.N = b; g.K = T; g.batch = width / b;
+  if (accumulate) {
+    g.add[0] = dG;
+    g.addc[0] = 1.f;
+    g.nadd = 1;
+  }
+  return launch_sgemm(g, s);
+}
+
+// ---- bf16 building blocks (tcgen05) -----------------------------------------------
+UmmaOperand act_kmajor(const void* p, int T, int width, int64_t boff_k) {
+  UmmaOperand o;
+  o.ptr = p; o.rows = T; o.cols = width; o.ld = width; o.mn_major = 0; o.boff_k = boff_k;
+  return o;
+}
+UmmaOperand act_mnmajor(const void* p, int T, int width, int64_t boff_mn) {
+  UmmaOperand o;
+  o.ptr = p; o.rows = T; o.cols = width; o.ld = width; o.mn_major = 1; o.boff_mn = boff_mn;
+  return o;
+}
+cudaError_t bf16_blockdiag(const void* in, const void* G, void* out, int T, int width, int b,
+                           bool transposeG, cudaStream_t s) {
+  const int nblk = width / b;
+  UmmaGemm g;
+  g.A = act_kmajor(in, T, width, b);
+  UmmaOperand B;
+  B.ptr = G; B.rows = (int64_t)nblk * b; B.cols = b; B.ld = b;
+  if (!transposeG) {  // B[n=r][k=c] = G_j[r][c]: K-major
+    B.mn_major = 0; B.boff_mn = b;
+  } else {            // B[n=r][k=c] = G_j[c][r]: MN-major
+    B.mn_major = 1; B.boff_k = b;
+  }
+  g.B = B;
+  g.M = T; g.N = b; g.K = b; g.batch = nblk;
+  g.D = out; g.out_f32 = 0; g.ldd = width; g.d_boff_col = b;
+  // forward products use G^T (B K-major); backward products use G (B MN-major)
+  return launch_umma_gemm(g, "gemm_blockdiag", s);
+}
+cudaError_t bf16_block_grad(const void* A, const void* B, float* part, float* dG, int ks, int T,
+                            int width, int b, int accumulate, cudaStream_t s) {
+  const int nblk = width / b;
+  UmmaGemm g;
+  g.A = act_mnmajor(A, T, width, b);
+  g.B = act_mnmajor(B, T, width, b);
+  g.M = b; g.N = b; g.K = T; g.batch = nblk; g.ksplit = ks;
+  g.D = part; g.out_f32 = 1; g.ldd = b; g.d_boff = (int64_t)b * b;
+  g.d_split = (int64_t)nblk * b * b;
+  cudaError_t e = launch_umma_gemm(g, "gemm_dG", s);
+  if (e != cudaSuccess) return e;
+  return launch_split_reduce(part, ks, (int64_t)nblk * b * b, dG, (int64_t)nblk * b * b,
+                             accumulate, s);
+}
+cudaError_t bf16_w0(const void* in, const void* W0p, void* out, int T, int n, int m, bool forward,
+                    cudaStream_t s) {
+  UmmaGemm g;
+  if (forward) {  // W[T, m] = V[T, n] W0'^T : B[n=o][k=i] = W0'[o][i], K-major
+    g.A = act_kmajor(in, T, n, 0);
+    UmmaOperand B;
+    B.ptr = W0p; B.rows = m; B.cols = n; B.ld = n; B.mn_major = 0;
+    g.B = B;
+    g.M = T; g.N = m; g.K = n;
+    g.D = out; g.ldd = m;
+  } else {        // dV[T, n] = dW[T, m] W0' : B[n=i][k=o] = W0'[o][i], MN-major
+    g.A = act_kmajor(in, T, m, 0);
+    UmmaOperand B;
+    B.ptr = W0p; B.rows = m; B.cols = n; B.ld = n; B.mn_major = 1;
+    g.B = B;
+    g.M = T; g.N = n; g.K = m;
+    g.D = out; g.ldd = n;
+  }
+  g.batch = 1;
+  g.out_f32 = 0;
+  return launch_umma_gemm(g, "gemm_w0", s);
+}
+
+// Forward body shared by poetx_linear_fwd and the recompute path of the backward.
+// Writes U (if U != x-gather target), V, W; Z and y only when y != nullptr.
+int forward_body(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
+                 const void* W0p, void* y, void* U, void* V, void* W, void* Z, cudaStream_t s) {
+  const int T = d->T, n = d->n, m = d->m, b = d->b;
+  const bool bf = d->dtype == POETX_BF16;
+  const int es = bf ? 2 : 4;
+  POETX_CUDA(launch_gather(x, U, nullptr, d->perm_P, T, n, n, n, es, s), "gather x");
+  if (bf) {
+    POETX_CUDA(bf16_blockdiag(U, G_P, V, T, n, b, false, s), "blockdiag G_P");
+    POETX_CUDA(bf16_w0(V, W0p, W, T, n, m, true, s), "W0' gemm");
+    if (y) {
+      POETX_CUDA(bf16_blockdiag(W, G_R, Z, T, m, b, false, s), "blockdiag G_R");
+      POETX_CUDA(launch_gather(Z, y, nullptr, d->inv_R, T, m, m, m, es, s), "scatter y");
+    }
+  } else {
+    POETX_CUDA(f32_blockdiag((const float*)U, (const float*)G_P, (float*)V, T, n, b, true, s),
+               "blockdiag G_P");
+    SgemmArgs g;
+    g.A = (const float*)V; g.lda = n;
+    g.B = (const float*)W0p; g.ldb = n; g.transB = 1;
+    g.C = (float*)W; g.ldc = m;
+    g.M = T; g.N = m; g.K = n; g.batch = 1;
+    POETX_CUDA(launch_sgemm(g, s), "W0' gemm");
+    if (y) {
+      POETX_CUDA(f32_blockdiag((const float*)W, (const float*)G_R, (float*)Z, T, m, b, true, s),
+                 "blockdiag G_R");
+      POETX_CUDA(launch_gather(Z, y, nullptr, d->inv_R, T, m, m, m, es, s), "scatter y");
+    }
+  }
+  return POETX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t poetx_linear_fwd_workspace(const poetx_linear_desc* d, int has_save_u, int has_save_w) {
+  if (!d || d->T < 0 || d->n < 1 || d->m < 1 || d->b < 1) return 0;
+  return fwd_layout(d, has_save_u, has_save_w).total;
+}
+
+size_t poetx_linear_bwd_workspace(const poetx_linear_desc* d, int has_save_u, int has_save_w) {
+  if (!d || d->T < 0 || d->n < 1 || d->m < 1 || d->b < 1) return 0;
+  return bwd_layout(d, has_save_u, has_save_w).total;
+}
+
+int poetx_linear_fwd(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
+                     const void* W0p, void* y, void* save_u, void* save_w, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int st = linear_validate(d);
+  if (st != POETX_OK) return st;
+  if (d->T == 0) return POETX_OK;
+  if ((st = check_ptrs({x, G_P, G_R, W0p, y})) != POETX_OK) return st;
+  if ((st = check_opt(save_u)) != POETX_OK || (st = check_opt(save_w)) != POETX_OK) return st;
+  const FwdLayout L = fwd_layout(d, save_u != nullptr, save_w != nullptr);
+  if (ws_bytes < L.total) return fail(POETX_ERR_WORKSPACE, "forward scratch too small");
+  if (L.total && !ws) return fail(POETX_ERR_INVALID_ARG, "scratch is NULL");
+  if ((st = check_opt(ws)) != POETX_OK) return st;
+  Carve cv(ws);
+  void* U = save_u ? save_u : cv.take(L.U);
+  void* V = cv.take(L.V);
+  void* W = save_w ? save_w : cv.take(L.W);
+  void* Z = cv.take(L.Z);
+  return forward_body(d, x, G_P, G_R, W0p, y, U, V, W, Z, static_cast<cudaStream_t>(stream));
+}
+
+int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, const void* G_P,
+                     const void* G_R, const void* W0p, const void* save_u, const void* save_w,
+                     void* dx, float* dG_P, float* dG_R, int accumulate, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int st = linear_validate(d);
+  if (st != POETX_OK) return st;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(POETX_ERR_INVALID_ARG, "accumulate must be 0 or 1");
+  if ((st = check_ptrs({dG_P, dG_R})) != POETX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int T = d->T, n = d->n, m = d->m, b = d->b;
+  const int nP = n / b, nR = m / b;
+  if (T == 0) {  // empty token set: dG = 0 (or unchanged when accumulating)
+    if (!accumulate) {
+      POETX_CUDA(launch_split_reduce(nullptr, 0, 0, dG_P, (int64_t)nP * b * b, 0, s), "zero dG");
+      POETX_CUDA(launch_split_reduce(nullptr, 0, 0, dG_R, (int64_t)nR * b * b, 0, s), "zero dG");
+    }
+    return POETX_OK;
+  }
+  if ((st = check_ptrs({dy, G_P, G_R, W0p, dx})) != POETX_OK) return st;
+  if ((st = check_opt(save_u)) != POETX_OK || (st = check_opt(save_w)) != POETX_OK) return st;
+  if (!save_u || !save_w)
+    if ((st = check_ptrs({x})) != POETX_OK) return st;
+  const BwdLayout L = bwd_layout(d, save_u != nullptr, save_w != nullptr);
+  if (ws_bytes < L.total) return fail(POETX_ERR_WORKSPACE, "backward scratch too small");
+  if (L.total && !ws) return fail(POETX_ERR_INVALID_ARG, "scratch is NULL");
+  if ((st = check_opt(ws)) != POETX_OK) return st;
+  const bool bf = d->dtype == POETX_BF16;
+  const int es = bf ? 2 : 4;
+  Carve cv(ws);
+  void* U = save_u ? const_cast<void*>(save_u) : cv.take(L.U);
+  void* Vr = save_w ? nullptr : cv.take(L.Vr);
+  void* W = save_w ? const_cast<void*>(save_w) : cv.take(L.Wr);
+  void* dZ = cv.take(L.dZ);
+  void* dW = cv.take(L.dW);
+  void* dV = cv.take(L.dV);
+  void* dU = cv.take(L.dU);
+  float* partR = static_cast<float*>(cv.take(L.partR));
+  float* partP = static_cast<float*>(cv.take(L.partP));
+  // recompute what the forward did not save (POET-X section 2.5, checkpointing)
+  if (!save_w) {
+    st = forward_body(d, x, G_P, G_R, W0p, nullptr, U, Vr, W, nullptr, s);
+    if (st != POETX_OK) return st;
+  } else if (!save_u) {
+    POETX_CUDA(launch_gather(x, U, nullptr, d->perm_P, T, n, n, n, es, s), "gather x");
+  }
+  // B1: dZ = dY[:, p_R]; dW_j = dZ_j G_R,j; dG_R,j = dZ_j^T W_j
+  POETX_CUDA(launch_gather(dy, dZ, nullptr, d->perm_R, T, m, m, m, es, s), "gather dy");
+  if (bf) {
+    POETX_CUDA(bf16_blockdiag(dZ, G_R, dW, T, m, b, true, s), "blockdiag G_R^T");
+    POETX_CUDA(bf16_block_grad(dZ, W, partR, dG_R, L.ksR, T, m, b, accumulate, s), "dG_R");
+    // B2: dV = dW W0'
+    POETX_CUDA(bf16_w0(dW, W0p, dV, T, n, m, false, s), "W0' gemm (backward)");
+    // B3: dU_j = dV_j G_P,j; dG_P,j = dV_j^T U_j; dX[:, p_P[i]] = dU[:, i]
+    POETX_CUDA(bf16_blockdiag(dV, G_P, dU, T, n, b, true, s), "blockdiag G_P^T");
+    POETX_CUDA(bf16_block_grad(dV, U, partP, dG_P, L.ksP, T, n, b, accumulate, s), "dG_P");
+  } else {
+    POETX_CUDA(f32_blockdiag((const float*)dZ, (const float*)G_R, (float*)dW, T, m, b, false, s),
+               "blockdiag G_R^T");
+    POETX_CUDA(f32_block_grad((const float*)dZ, (const float*)W, dG_R, T, m, b, accumulate, s),
+               "dG_R");
+    SgemmArgs g;
+    g.A = (const float*)dW; g.lda = m;
+    g.B = (const float*)W0p; g.ldb = n; g.transB = 0;
+    g.C = (float*)dV; g.ldc = n;
+    g.M = T; g.N = n; g.K = m; g.batch = 1;
+    POETX_CUDA(launch_sgemm(g, s), "W0' gemm (backward)");
+    POETX_CUDA(f32_blockdiag((const float*)dV, (const float*)G_P, (float*)dU, T, n, b, false, s),
+               "blockdiag G_P^T");
+    POETX_CUDA(f32_block_grad((const float*)dV, (const float*)U, dG_P, T, n, b, accumulate, s),
+               "dG_P");
+  }
+  POETX_CUDA(launch_gather(dU, dx, nullptr, d->inv_P, T, n, n, n, es, s), "scatter dx");
+  return POETX_OK;
+}
+
+int poetx_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int* flag = device_error_flag();
+  if (!flag) return fail(POETX_ERR_CUDA, "device error flag unavailable");
+  int v = 0;
+  e = cudaMemcpy(&v, flag, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device flag");
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(v, "a kernel's bounded wait timed out");
+  }
+  return POETX_OK;
+}
+
+uint64_t poetx_launch_count(void) { return g_launches.load(); }
+
+int poetx_profile_begin(const char* name) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!name || !*name) {
+    g_prof_on = false;
+    return POETX_OK;
+  }
+  if (g_ev_start.empty()) {
+    g_ev_start.resize(kEventPairs);
+    g_ev_stop.resize(kEventPairs);
+    for (int i = 0; i < kEventPairs; ++i) {
+      cudaError_t e1 = cudaEventCreate(&g_ev_start[i]);
+      cudaError_t e2 = cudaEventCreate(&g_ev_stop[i]);
+      if (e1 != cudaSuccess || e2 != cudaSuccess) {
+        g_ev_start.clear();
+        g_ev_stop.clear();
+        return cuda_fail(e1 != cudaSuccess ? e1 : e2, "event create");
+      }
+    }
+  }
+  g_prof_family = name;
+  g_prof_used = 0;
+  g_prof_on = true;
+  return POETX_OK;
+}
+
+int poetx_profile_end(int32_t* launches, double* total_ms) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  double tot = 0.0;
+  for (int i = 0; i < g_prof_used; ++i) {
+    cudaError_t e = cudaEventSynchronize(g_ev_stop[i]);
+    if (e != cudaSuccess) return cuda_fail(e, "event synchronize");
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, g_ev_start[i], g_ev_stop[i]);
+    if (e != cudaSuccess) return cuda_fail(e, "event elapsed");
+    tot += ms;
+  }
+  if (launches) *launches = g_prof_used;
+  if (total_ms) *total_ms = tot;
+  return POETX_OK;
+}
+
+}  // extern "C"

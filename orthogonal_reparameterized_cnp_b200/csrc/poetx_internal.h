@@ -1,0 +1,119 @@
+// Internal declarations shared by the libpoetx translation units (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/poetx.h"
+
+namespace poetx {
+
+// ---- error reporting -------------------------------------------------------------
+void set_error(const std::string& msg);
+int fail(int status, const std::string& msg);
+int cuda_fail(cudaError_t e, const char* what);
+
+// Launch accounting: every kernel launch goes through begin_launch/end_launch, which
+// count it and, when the profiler watches that kernel family, bracket it with events.
+void begin_launch(const char* family, cudaStream_t s);
+void end_launch(const char* family, cudaStream_t s);
+
+// Device error flag (set by kernels whose bounded waits time out).
+int* device_error_flag();
+
+// Number of SMs of the current device.
+int num_sms();
+
+// ---- permutation / gather kernels (kernels_perm.cu) ------------------------------
+// out[r, c] = in[row_idx ? row_idx[r] : r, col_idx[c]]
+cudaError_t launch_gather(const void* in, void* out, const int32_t* row_idx,
+                          const int32_t* col_idx, int rows, int cols, int64_t ld_in,
+                          int64_t ld_out, int elem_bytes, cudaStream_t s);
+
+// ---- fp32 SIMT batched GEMM (kernels_sgemm.cu) -----------------------------------
+enum SgemmMode { SG_FULL = 0, SG_SYM = 1, SG_SYMSKEW = 2 };
+
+struct SgemmArgs {
+  // acc = op(A) op(B) + alpha2 * op(A2) op(B2)
+  // sym  = diag * delta_ij + sum_t addc[t] * add[t][i, j]
+  // skew = alpha * acc + skew_c * skew_add[i, j]
+  // FULL / SYM:  C = skew + sym (SYM: upper tiles computed, C_ji = C_ij)
+  // SYMSKEW:     C_ij = sym + skew, C_ji = sym - skew, C_ii = sym (upper tiles computed)
+  // C2 (optional, FULL / SYM only) = alpha_c2 * acc + diag2 * delta + sum addc2[t] add[t]
+  const float* A = nullptr;
+  int64_t lda = 0, sA = 0;
+  const float* B = nullptr;
+  int64_t ldb = 0, sB = 0;
+  int transA = 0, transB = 0;
+  const float* A2 = nullptr;
+  int64_t lda2 = 0, sA2 = 0;
+  const float* B2 = nullptr;
+  int64_t ldb2 = 0, sB2 = 0;
+  int transA2 = 0, transB2 = 0;
+  int K2 = 0;
+  float alpha2 = 1.f;
+  float* C = nullptr;
+  int64_t ldc = 0, sC = 0;  // also the layout of add[], skew_add and C2
+  void* C_bf16 = nullptr;   // optional bf16 copy of C
+  float* C2 = nullptr;
+  float alpha_c2 = 0.f, diag2 = 0.f;
+  float addc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int M = 0, N = 0, K = 0, batch = 0;
+  float alpha = 1.f;
+  int nadd = 0;
+  const float* add[8] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  float addc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const float* skew_add = nullptr;
+  float skew_c = 0.f;
+  float diag = 0.f;
+  int mode = SG_FULL;
+};
+cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s);
+
+// ---- CNP elementwise kernels (kernels_sgemm.cu) -----------------------------------
+// Q = skew(theta) for nblk blocks of size b.
+cudaError_t launch_theta_to_Q(const float* theta, float* Q, int nblk, int b, cudaStream_t s);
+// out_o = sum_s coef[o][s] * (X_s + X_s^T) for o < nout (symmetric outputs), s < nin.
+cudaError_t launch_symcomb(const float* const* X, int nin, float* const* out, int nout,
+                           const float* coef /* [nout][nin] row-major */, int nblk, int b,
+                           cudaStream_t s);
+// dtheta_idx(i,j) = A_ij - A_ji for i < j.
+cudaError_t launch_pack_skew(const float* A, float* dtheta, int nblk, int b, cudaStream_t s);
+// dst[j] = (accumulate ? dst[j] : 0) + sum_s src[s * stride + j], s < nsplit (fixed order).
+cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, float* dst,
+                                int64_t count, int accumulate, cudaStream_t s);
+// fp32 -> bf16 (round to nearest even)
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s);
+
+// ---- tcgen05 GEMM (kernels_umma.cu) ----------------------------------------------
+// D[M x N] = A[M x K] . B[N x K]^T per batch entry, bf16 operands, fp32 accumulation.
+// Operand X is K-major when X[row, k] is contiguous in k, MN-major when contiguous in
+// the row index.  Each operand is a 2-D row-major bf16 matrix in global memory plus
+// per-batch coordinate offsets.
+struct UmmaOperand {
+  const void* ptr = nullptr;  // base of the row-major 2-D matrix
+  int64_t rows = 0, cols = 0; // extent of the 2-D matrix
+  int64_t ld = 0;             // row stride in elements
+  int mn_major = 0;           // 0: rows index M/N and cols index K; 1: rows index K
+  int64_t boff_mn = 0;        // per-batch offset added to the M (or N) coordinate
+  int64_t boff_k = 0;         // per-batch offset added to the K coordinate
+};
+struct UmmaGemm {
+  UmmaOperand A, B;
+  int M = 0, N = 0, K = 0, batch = 1;
+  int ksplit = 1;             // split of K into ksplit partial sums (fp32 output only)
+  void* D = nullptr;          // output base
+  int out_f32 = 0;            // 0: bf16 output, 1: fp32 output
+  int64_t ldd = 0;            // row stride of D in elements
+  int64_t d_boff_col = 0;     // per-batch column offset of D
+  int64_t d_boff = 0;         // per-batch element offset of D
+  int64_t d_split = 0;        // per-split element offset of D
+};
+cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t s);
+// ksplit the launcher would choose for the given problem (used to size scratch).
+int umma_choose_ksplit(int M, int N, int K, int batch);
+
+}  // namespace poetx

@@ -1,0 +1,327 @@
+"""Thin ctypes binding of libpoetx (the C ABI declared in include/poetx.h).
+
+Argument marshalling only: tensors are passed as raw device pointers, the stream as the
+torch stream handle.  Every step of the layer runs in the library's CUDA kernels; there is
+no fallback.  A missing library or a call without a CUDA device raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpoetx.so")
+
+POETX_OK = 0
+POETX_ERR_INVALID_ARG = 1
+POETX_ERR_SHAPE = 2
+POETX_ERR_DTYPE = 3
+POETX_ERR_ALIGN = 4
+POETX_ERR_WORKSPACE = 5
+POETX_ERR_CUDA = 6
+POETX_ERR_TIMEOUT = 7
+
+POETX_F32 = 0
+POETX_BF16 = 1
+
+_c_int = ctypes.c_int
+_c_i32 = ctypes.c_int32
+_c_u64 = ctypes.c_uint64
+_c_size = ctypes.c_size_t
+_vp = ctypes.c_void_p
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+
+class LinearDesc(ctypes.Structure):
+    _fields_ = [("T", _c_i32), ("n", _c_i32), ("m", _c_i32), ("b", _c_i32), ("dtype", _c_i32),
+                ("perm_P", _vp), ("inv_P", _vp), ("perm_R", _vp), ("inv_R", _vp)]
+
+
+# name -> (restype, argtypes); the same list is checked against include/poetx.h by the tests
+SIGNATURES = {
+    "poetx_status_string": (ctypes.c_char_p, [_c_int]),
+    "poetx_last_error": (ctypes.c_char_p, []),
+    "poetx_version": (ctypes.c_char_p, []),
+    "poetx_make_perm": (_c_int, [_c_u64, _c_i32, _i32p, _i32p]),
+    "poetx_merge_perm": (_c_int, [_vp, _vp, _c_i32, _c_i32, _vp, _vp, _c_int, _vp]),
+    "poetx_permute_cols": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
+    "poetx_cnp_workspace": (_c_size, [_c_i32, _c_i32, _c_i32]),
+    "poetx_cnp_fwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
+    "poetx_cnp_bwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
+    "poetx_linear_fwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
+    "poetx_linear_bwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
+    "poetx_linear_fwd": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _c_size, _vp]),
+    "poetx_linear_bwd": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp, _vp, _c_int, _vp, _c_size, _vp]),
+    "poetx_device_status": (_c_int, [_vp]),
+    "poetx_launch_count": (_c_u64, []),
+    "poetx_profile_begin": (_c_int, [ctypes.c_char_p]),
+    "poetx_profile_end": (_c_int, [_i32p, ctypes.POINTER(ctypes.c_double)]),
+}
+
+_lib = None
+
+
+class PoetxError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        lib = _load()
+        super().__init__(f"{where}: {lib.poetx_status_string(status).decode()} "
+                         f"({status}): {lib.poetx_last_error().decode()}")
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libpoetx.so not built ({LIB_PATH}); run "
+                               "`python -m orthogonal_reparameterized_cnp_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def lib():
+    return _load()
+
+
+def _check(status: int, where: str):
+    if status != POETX_OK:
+        raise PoetxError(status, where)
+
+
+# ------------------------------------------------------------------------ helpers
+def _ptr(t) -> int | None:
+    """Device pointer of a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return POETX_F32
+    if t.dtype == torch.bfloat16:
+        return POETX_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------------ host calls
+def make_perm(seed: int, n: int):
+    """Seeded permutation and its inverse (numpy int32), computed by the library."""
+    L = _load()
+    perm = np.empty(n, dtype=np.int32)
+    inv = np.empty(n, dtype=np.int32)
+    _check(L.poetx_make_perm(seed & ((1 << 64) - 1), n,
+                             perm.ctypes.data_as(_i32p), inv.ctypes.data_as(_i32p)),
+           "poetx_make_perm")
+    return perm, inv
+
+
+def cnp_workspace(nblk: int, b: int, k: int) -> int:
+    return int(_load().poetx_cnp_workspace(nblk, b, k))
+
+
+def linear_desc(T, n, m, b, dtype_code, perm_P, inv_P, perm_R, inv_R) -> LinearDesc:
+    return LinearDesc(T, n, m, b, dtype_code, _ptr(perm_P), _ptr(inv_P), _ptr(perm_R),
+                      _ptr(inv_R))
+
+
+def linear_fwd_workspace(desc: LinearDesc, has_save_u=True, has_save_w=True) -> int:
+    return int(_load().poetx_linear_fwd_workspace(ctypes.byref(desc), int(has_save_u),
+                                                  int(has_save_w)))
+
+
+def linear_bwd_workspace(desc: LinearDesc, has_save_u=True, has_save_w=True) -> int:
+    return int(_load().poetx_linear_bwd_workspace(ctypes.byref(desc), int(has_save_u),
+                                                  int(has_save_w)))
+
+
+def launch_count() -> int:
+    return int(_load().poetx_launch_count())
+
+
+def profile_begin(name: str | None):
+    _check(_load().poetx_profile_begin(name.encode() if name else None), "poetx_profile_begin")
+
+
+def profile_end():
+    n = ctypes.c_int32(0)
+    ms = ctypes.c_double(0.0)
+    _check(_load().poetx_profile_end(ctypes.byref(n), ctypes.byref(ms)), "poetx_profile_end")
+    return int(n.value), float(ms.value)
+
+
+# ------------------------------------------------------------------------ device calls
+def _require_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        raise RuntimeError("libpoetx needs a CUDA device (sm_100a); none is available")
+
+
+def merge_perm(W0, W0p, perm_R, perm_P, stream=None):
+    _require_cuda()
+    m, n = W0.shape
+    _check(_load().poetx_merge_perm(_ptr(W0), _ptr(W0p), m, n, _ptr(perm_R), _ptr(perm_P),
+                                    _dtype_code(W0), _stream(stream)), "poetx_merge_perm")
+
+
+def permute_cols(x, out, idx, stream=None):
+    _require_cuda()
+    rows, cols = x.shape
+    _check(_load().poetx_permute_cols(_ptr(x), _ptr(out), _ptr(idx), rows, cols, _dtype_code(x),
+                                      _stream(stream)), "poetx_permute_cols")
+
+
+def cnp_fwd(theta, G, G_bf16, b: int, k: int, ws, stream=None):
+    _require_cuda()
+    nblk = theta.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_cnp_fwd(_ptr(theta), _ptr(G), _ptr(G_bf16), nblk, b, k, _ptr(ws),
+                                 ws_bytes, _stream(stream)), "poetx_cnp_fwd")
+
+
+def cnp_bwd(theta, dG, dtheta, b: int, k: int, ws, stream=None):
+    _require_cuda()
+    nblk = theta.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_cnp_bwd(_ptr(theta), _ptr(dG), _ptr(dtheta), nblk, b, k, _ptr(ws),
+                                 ws_bytes, _stream(stream)), "poetx_cnp_bwd")
+
+
+def linear_fwd(desc: LinearDesc, x, G_P, G_R, W0p, y, save_u, save_w, ws, stream=None):
+    _require_cuda()
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_linear_fwd(ctypes.byref(desc), _ptr(x), _ptr(G_P), _ptr(G_R),
+                                    _ptr(W0p), _ptr(y), _ptr(save_u), _ptr(save_w), _ptr(ws),
+                                    ws_bytes, _stream(stream)), "poetx_linear_fwd")
+
+
+def linear_bwd(desc: LinearDesc, x, dy, G_P, G_R, W0p, save_u, save_w, dx, dG_P, dG_R,
+               accumulate: int, ws, stream=None):
+    _require_cuda()
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_linear_bwd(ctypes.byref(desc), _ptr(x), _ptr(dy), _ptr(G_P), _ptr(G_R),
+                                    _ptr(W0p), _ptr(save_u), _ptr(save_w), _ptr(dx), _ptr(dG_P),
+                                    _ptr(dG_R), int(accumulate), _ptr(ws), ws_bytes,
+                                    _stream(stream)), "poetx_linear_bwd")
+
+
+def device_status(stream=None) -> int:
+    _require_cuda()
+    return int(_load().poetx_device_status(_stream(stream)))
+
+
+# ------------------------------------------------------------------------ a layer object
+@dataclass
+class PoetxLinearState:
+    """Device buffers of one POET-X linear for a fixed token count (allocated by torch)."""
+    T: int
+    n: int
+    m: int
+    b: int
+    k: int
+    dtype: str
+
+
+class PoetxLinear:
+    """One POET-X linear on the GPU: merged weight, CNP blocks, forward and backward.
+
+    All buffers are torch tensors on the current device; every computation is a libpoetx
+    call.  ``theta`` holds the input-side blocks first, then the output-side blocks.
+    """
+
+    def __init__(self, W0, theta_P, theta_R, perm_P, perm_R, b: int, k: int, T: int,
+                 save_activations: bool = True):
+        import torch
+        _require_cuda()
+        dev = W0.device
+        self.m, self.n = W0.shape
+        self.b, self.k, self.T = b, k, T
+        self.bf16 = W0.dtype == torch.bfloat16
+        self.nP, self.nR = self.n // b, self.m // b
+        nblk = self.nP + self.nR
+        ntri = b * (b - 1) // 2
+        i32 = dict(dtype=torch.int32, device=dev)
+        pP = torch.as_tensor(np.asarray(perm_P, dtype=np.int32), **i32)
+        pR = torch.as_tensor(np.asarray(perm_R, dtype=np.int32), **i32)
+        self.perm_P, self.perm_R = pP, pR
+        self.inv_P = torch.empty_like(pP)
+        self.inv_P[pP.long()] = torch.arange(self.n, **i32)
+        self.inv_R = torch.empty_like(pR)
+        self.inv_R[pR.long()] = torch.arange(self.m, **i32)
+        self.W0 = W0
+        self.W0p = torch.empty_like(W0)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.theta = torch.empty((nblk, ntri), **f32)
+        self.theta[: self.nP] = theta_P
+        self.theta[self.nP:] = theta_R
+        self.G = torch.empty((nblk, b, b), **f32)
+        self.G_lp = torch.empty((nblk, b, b), dtype=W0.dtype, device=dev) if self.bf16 else None
+        self.dG = torch.empty((nblk, b, b), **f32)
+        self.dtheta = torch.empty((nblk, ntri), **f32)
+        self.cnp_ws = torch.empty(max(cnp_workspace(nblk, b, k), 16), dtype=torch.uint8,
+                                  device=dev)
+        self.desc = linear_desc(T, self.n, self.m, b, POETX_BF16 if self.bf16 else POETX_F32,
+                                self.perm_P, self.inv_P, self.perm_R, self.inv_R)
+        act = W0.dtype
+        self.save = save_activations
+        if save_activations:
+            self.U = torch.empty((T, self.n), dtype=act, device=dev)
+            self.Wsave = torch.empty((T, self.m), dtype=act, device=dev)
+        else:
+            self.U = self.Wsave = None
+        fwd_ws = linear_fwd_workspace(self.desc, self.save, self.save)
+        bwd_ws = linear_bwd_workspace(self.desc, self.save, self.save)
+        self.ws = torch.empty(max(fwd_ws, bwd_ws, 16), dtype=torch.uint8, device=dev)
+
+    def G_ops(self):
+        G = self.G_lp if self.bf16 else self.G
+        return G[: self.nP], G[self.nP:]
+
+    def merge(self, stream=None):
+        merge_perm(self.W0, self.W0p, self.perm_R, self.perm_P, stream)
+
+    def cnp_forward(self, stream=None):
+        cnp_fwd(self.theta, self.G, self.G_lp, self.b, self.k, self.cnp_ws, stream)
+
+    def forward(self, x, y, stream=None):
+        GP, GR = self.G_ops()
+        linear_fwd(self.desc, x, GP, GR, self.W0p, y, self.U, self.Wsave, self.ws, stream)
+
+    def backward(self, x, dy, dx, accumulate=0, stream=None):
+        GP, GR = self.G_ops()
+        linear_bwd(self.desc, x, dy, GP, GR, self.W0p, self.U, self.Wsave, dx,
+                   self.dG[: self.nP], self.dG[self.nP:], accumulate, self.ws, stream)
+
+    def cnp_backward(self, stream=None):
+        cnp_bwd(self.theta, self.dG, self.dtheta, self.b, self.k, self.cnp_ws, stream)
+
+    def step(self, x, dy, y, dx, stream=None):
+        """One pass of the whole path: merge, CNP forward, layer forward and backward,
+        CNP backward."""
+        self.merge(stream)
+        self.cnp_forward(stream)
+        self.forward(x, y, stream)
+        self.backward(x, dy, dx, 0, stream)
+        self.cnp_backward(stream)

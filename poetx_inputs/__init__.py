@@ -119,12 +119,22 @@ def layer_inputs(s: LayerShape) -> LayerInputs:
 
 
 def cnp_inputs(config_id: int, linear_id: int, nblk: int, b: int, std_theta: float = 0.01,
-               std_dG: float = 1.0):
-    """theta [nblk, b(b-1)/2] and an upstream gradient dG [nblk, b, b], both fp32."""
+               std_dG: float = 1.0, chunk_blocks: int = 256):
+    """theta [nblk, b(b-1)/2] and an upstream gradient dG [nblk, b, b], both fp32.
+
+    Drawn in chunks of blocks from one stream per tensor (the same values as a single
+    draw), so large block counts never hold a float64 copy of the whole tensor.
+    """
     ntri = b * (b - 1) // 2
-    theta = draw(config_id, linear_id, "theta_P", (nblk, ntri), std_theta, "f32")
-    dG = draw(config_id, linear_id, "dG", (nblk, b, b), std_dG, "f32")
-    return theta, dG
+    out = []
+    for name, shape, std in [("theta_P", (ntri,), std_theta), ("dG", (b, b), std_dG)]:
+        g = _rng(config_id, linear_id, TENSOR_IDS[name])
+        a = np.empty((nblk,) + shape, dtype=np.float32)
+        for c0 in range(0, nblk, chunk_blocks):
+            c1 = min(nblk, c0 + chunk_blocks)
+            a[c0:c1] = (g.standard_normal(size=(c1 - c0,) + shape) * std).astype(np.float32)
+        out.append(a)
+    return out[0], out[1]
 
 
 # ---------------------------------------------------------------- named workloads

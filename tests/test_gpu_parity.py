@@ -1,0 +1,326 @@
+"""GPU parity: libpoetx (through its C ABI) against the float64 oracle on the same seeded
+inputs.
+
+Bars: permutations / index maps / merged weight bit-exact; CNP fp32 max-abs <= 1e-5 on G
+and dtheta; fp32 layer normalised max error <= 1e-5; bf16 layer outputs and gradients
+normalised max error <= 2e-2 (normalised = max|gpu - ref| / max|ref| per tensor).
+"""
+import numpy as np
+import pytest
+
+from oracle import poetx_ref as ref
+from poetx_inputs import (LayerShape, cnp_inputs, cnp_sweep_blocks, layer_inputs,
+                          workload_llama13b_block, workload_llama1b_attn, workload_llama8b_up,
+                          workload_small_fp32)
+
+from .gpu_harness import host, norm_max_err, run_layer, tensor
+
+pytestmark = pytest.mark.gpu
+
+CNP_ABS = 1e-5
+F32_NORM = 1e-5
+BF16_NORM = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    P.lib()  # fails loudly if the library is missing
+    yield
+
+
+def _P():
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    return P
+
+
+# ------------------------------------------------------------------ index maps
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rows,cols", [(1, 8), (7, 24), (300, 2048), (33, 14336), (5, 13824)])
+def test_permute_cols_bit_exact(dtype, rows, cols):
+    import torch
+    P = _P()
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    rng = np.random.default_rng(rows * 7 + cols)
+    a = rng.standard_normal((rows, cols)).astype(np.float32)
+    perm, inv = P.make_perm(rows * 1000 + cols, cols)
+    x = tensor(a, tdt)
+    out = torch.empty_like(x)
+    back = torch.empty_like(x)
+    P.permute_cols(x, out, tensor(perm, torch.int32))
+    P.permute_cols(out, back, tensor(inv, torch.int32))
+    torch.cuda.synchronize()
+    xs = x.cpu()
+    assert torch.equal(out.cpu(), xs[:, torch.from_numpy(perm.astype(np.int64))])
+    assert torch.equal(back.cpu(), xs)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("m,n", [(12, 8), (2048, 2048), (14336, 4096)])
+def test_merge_perm_bit_exact(dtype, m, n):
+    import torch
+    P = _P()
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    W0 = tensor(np.random.default_rng(m + n).standard_normal((m, n)).astype(np.float32), tdt)
+    pR, _ = P.make_perm(11 + m, m)
+    pP, _ = P.make_perm(13 + n, n)
+    W0p = torch.empty_like(W0)
+    P.merge_perm(W0, W0p, tensor(pR, torch.int32), tensor(pP, torch.int32))
+    torch.cuda.synchronize()
+    expect = ref.merge_perm(W0.cpu().float().numpy(), pR.astype(np.int64), pP.astype(np.int64))
+    assert np.array_equal(W0p.cpu().float().numpy(), expect)
+
+
+# ------------------------------------------------------------------ CNP
+def _cnp_gpu(theta, dG, b, k, with_bf16=False, ws_blocks=None):
+    import torch
+    P = _P()
+    nblk = theta.shape[0]
+    th = tensor(theta, torch.float32)
+    G = torch.empty((nblk, b, b), dtype=torch.float32, device="cuda")
+    Gb = torch.empty((nblk, b, b), dtype=torch.bfloat16, device="cuda") if with_bf16 else None
+    ws_bytes = P.cnp_workspace(nblk if ws_blocks is None else ws_blocks, b, k)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    P.cnp_fwd(th, G, Gb, b, k, ws)
+    dth = None
+    if dG is not None:
+        dth_t = torch.empty_like(th)
+        P.cnp_bwd(th, tensor(dG, torch.float32), dth_t, b, k, ws)
+        dth = dth_t
+    torch.cuda.synchronize()
+    assert P.device_status() == P.POETX_OK
+    return G, Gb, dth
+
+
+@pytest.mark.parametrize("b,k", [(2, 1), (2, 4), (3, 2), (5, 3), (8, 4), (17, 5), (32, 4),
+                                 (64, 2), (64, 6), (100, 4), (128, 4), (256, 4), (256, 7),
+                                 (512, 4), (1024, 2)])
+def test_cnp_matches_oracle(b, k):
+    nblk = 3 if b <= 256 else 2
+    rng = np.random.default_rng(b * 31 + k)
+    theta = (rng.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    dG = rng.standard_normal((nblk, b, b)).astype(np.float32)
+    G, Gb, dth = _cnp_gpu(theta, dG, b, k, with_bf16=True)
+    G_ref = ref.cnp_forward(theta, b, k)
+    assert np.abs(host(G) - G_ref).max() <= CNP_ABS
+    dth_ref = ref.cnp_backward(theta, dG, b, k)
+    assert np.abs(host(dth) - dth_ref).max() <= CNP_ABS
+    # the bf16 copy is the round-to-nearest-even of the fp32 G
+    import torch
+    assert torch.equal(Gb.cpu(), G.cpu().to(torch.bfloat16))
+
+
+def test_cnp_zero_theta_is_exact_identity():
+    import torch
+    for b in [4, 64, 256]:
+        theta = np.zeros((3, b * (b - 1) // 2), dtype=np.float32)
+        G, Gb, _ = _cnp_gpu(theta, None, b, 4, with_bf16=True)
+        eye = torch.eye(b).expand(3, b, b)
+        assert torch.equal(G.cpu(), eye)
+        assert torch.equal(Gb.cpu(), eye.to(torch.bfloat16))
+
+
+def test_cnp_small_workspace_chunks_blocks():
+    # one block's worth of scratch forces a chunk per block; results must not change
+    b, k, nblk = 64, 4, 5
+    rng = np.random.default_rng(5)
+    theta = (rng.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    dG = rng.standard_normal((nblk, b, b)).astype(np.float32)
+    G1, _, d1 = _cnp_gpu(theta, dG, b, k)
+    G2, _, d2 = _cnp_gpu(theta, dG, b, k, ws_blocks=1)
+    import torch
+    assert torch.equal(G1.cpu(), G2.cpu()) and torch.equal(d1.cpu(), d2.cpu())
+
+
+@pytest.mark.parametrize("b", [64, 128, 256, 512])
+@pytest.mark.parametrize("k", [2, 4, 6])
+def test_cnp_sweep_sampled(b, k):
+    """CNP sweep: all 7 linears x 32 layers of Llama-8B shapes on both sides (full block
+    count); the oracle checks the first, the last and randomly chosen blocks."""
+    nblk = cnp_sweep_blocks(b)
+    theta, dG = cnp_inputs(4, b * 10 + k, nblk, b)
+    G, _, dth = _cnp_gpu(theta, dG, b, k)
+    nsamp = {64: 24, 128: 12, 256: 6, 512: 3}[b]
+    rng = np.random.default_rng(b + k)
+    idx = sorted({0, nblk - 1, *rng.choice(nblk, nsamp, replace=False).tolist()})
+    G_h = G[idx].cpu().double().numpy()
+    d_h = dth[idx].cpu().double().numpy()
+    G_ref = ref.cnp_forward(theta[idx], b, k)
+    d_ref = ref.cnp_backward(theta[idx], dG[idx], b, k)
+    assert np.abs(G_h - G_ref).max() <= CNP_ABS
+    assert np.abs(d_h - d_ref).max() <= CNP_ABS
+
+
+# ------------------------------------------------------------------ layer, fp32
+def _check_full(out, s, inp, tol):
+    W0p = ref.merge_perm(inp.W0, out["perm_R"].astype(np.int64), out["perm_P"].astype(np.int64))
+    assert np.array_equal(out["W0p"], W0p)
+    o = ref.full_step(inp.x, inp.W0, inp.theta_P, inp.theta_R, inp.dy,
+                      out["perm_P"].astype(np.int64), out["perm_R"].astype(np.int64), s.b, s.k)
+    errs = {key: norm_max_err(out[key], o[key])
+            for key in ["y", "dx", "dG_P", "dG_R", "dtheta_P", "dtheta_R"]}
+    bad = {kk: v for kk, v in errs.items() if not v <= tol}
+    assert not bad, f"normalised max errors above {tol}: {errs}"
+    G_ref = np.concatenate([o["G_P"], o["G_R"]])
+    assert np.abs(out["G"] - G_ref).max() <= CNP_ABS
+    return errs
+
+
+def test_layer_fp32_small_config():
+    s = workload_small_fp32()
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    _check_full(out, s, inp, F32_NORM)
+
+
+@pytest.mark.parametrize("n,m,b,k,T", [(8, 12, 2, 1, 5), (12, 8, 4, 3, 3), (16, 24, 8, 4, 70),
+                                       (96, 64, 32, 2, 129), (256, 128, 64, 4, 1)])
+def test_layer_fp32_small_shapes(n, m, b, k, T):
+    s = LayerShape(f"fp32-{n}x{m}", T=T, n=n, m=m, b=b, k=k, dtype="f32", config_id=100 + b,
+                   std_theta=0.05)
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    _check_full(out, s, inp, F32_NORM)
+
+
+# ------------------------------------------------------------------ layer, bf16
+@pytest.mark.parametrize("n,m,b,T", [(256, 256, 128, 300), (512, 256, 256, 129), (256, 768, 128, 1),
+                                     (1024, 512, 512, 200), (384, 640, 128, 513)])
+def test_layer_bf16_small_shapes(n, m, b, T):
+    s = LayerShape(f"bf16-{n}x{m}", T=T, n=n, m=m, b=b, k=4, dtype="bf16", config_id=200 + b)
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    _check_full(out, s, inp, BF16_NORM)
+
+
+def test_layer_bf16_llama1b_full():
+    """n = m = 2048, b = 256, k = 4, T = 8192: every output against the full oracle."""
+    s = workload_llama1b_attn()
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    _check_full(out, s, inp, BF16_NORM)
+
+
+def test_recompute_mode_matches_saved_mode():
+    s = LayerShape("bf16-recompute", T=777, n=512, m=768, b=256, k=4, dtype="bf16", config_id=300)
+    inp = layer_inputs(s)
+    a = run_layer(inp, save=True)
+    b_ = run_layer(inp, save=False)
+    for key in ["y", "dx", "dG_P", "dG_R", "dtheta_P", "dtheta_R"]:
+        assert np.array_equal(a[key], b_[key]), key
+
+
+def test_runs_are_deterministic():
+    s = LayerShape("bf16-det", T=1000, n=512, m=512, b=128, k=4, dtype="bf16", config_id=301)
+    inp = layer_inputs(s)
+    a = run_layer(inp)
+    b_ = run_layer(inp)
+    for key in ["y", "dx", "dG_P", "dG_R", "dtheta_P", "dtheta_R"]:
+        assert np.array_equal(a[key], b_[key]), key
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_micro_batch_accumulation(dtype):
+    import torch
+    P = _P()
+    b = 128 if dtype == "bf16" else 16
+    s = LayerShape("acc", T=400, n=256, m=384, b=b, k=4, dtype=dtype, config_id=302)
+    inp = layer_inputs(s)
+    full = run_layer(inp)
+    layer = full["layer"]
+    act = layer.W0.dtype
+    x = tensor(inp.x, act)
+    dy = tensor(inp.dy, act)
+    y = torch.empty((s.T, s.m), dtype=act, device="cuda")
+    dx = torch.empty((s.T, s.n), dtype=act, device="cuda")
+    # split the tokens into two micro-batches sharing the same layer buffers
+    halves = [(0, 150), (150, 400)]
+    dG_sum = None
+    for i, (t0, t1) in enumerate(halves):
+        sub = P.PoetxLinear(layer.W0, layer.theta[: layer.nP], layer.theta[layer.nP:],
+                            full["perm_P"], full["perm_R"], s.b, s.k, t1 - t0)
+        sub.merge()
+        sub.cnp_forward()
+        sub.forward(x[t0:t1].contiguous(), y[t0:t1])
+        if dG_sum is not None:
+            sub.dG.copy_(dG_sum)
+        sub.backward(x[t0:t1].contiguous(), dy[t0:t1].contiguous(), dx[t0:t1], accumulate=int(i > 0))
+        dG_sum = sub.dG.clone()
+    torch.cuda.synchronize()
+    tol = 1e-6 if dtype == "f32" else 1e-5
+    assert np.abs(host(dG_sum) - host(layer.dG)).max() <= tol * max(1.0, np.abs(host(layer.dG)).max())
+
+
+def test_empty_token_set():
+    import torch
+    P = _P()
+    s = LayerShape("empty", T=0, n=256, m=256, b=128, k=4, dtype="bf16", config_id=303)
+    W0 = tensor(np.zeros((256, 256), np.float32), torch.bfloat16)
+    th = torch.zeros((2, 128 * 127 // 2), dtype=torch.float32, device="cuda")
+    pP, _ = P.make_perm(1, 256)
+    pR, _ = P.make_perm(2, 256)
+    layer = P.PoetxLinear(W0, th, th, pP, pR, 128, 4, 0)
+    layer.merge()
+    layer.cnp_forward()
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    layer.forward(x, y)
+    layer.dG.fill_(7.0)
+    layer.backward(x, y, x)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(layer.dG).item() == 0
+
+
+# ------------------------------------------------------------------ full-size, sampled
+def _sampled_checks(out, s, inp, rows, tol=BF16_NORM):
+    pP = out["perm_P"].astype(np.int64)
+    pR = out["perm_R"].astype(np.int64)
+    W0p = ref.merge_perm(inp.W0, pR, pP)
+    G_P = ref.cnp_forward(inp.theta_P, s.b, s.k)
+    G_R = ref.cnp_forward(inp.theta_R, s.b, s.k)
+    y_ref = ref.layer_forward_rows(inp.x[rows], W0p, G_P, G_R, pP, pR)
+    dx_ref = ref.layer_backward_dx_rows(inp.dy[rows], W0p, G_P, G_R, pP, pR)
+    assert norm_max_err(out["y"][rows], y_ref) <= tol
+    assert norm_max_err(out["dx"][rows], dx_ref) <= tol
+    assert np.abs(out["G"] - np.concatenate([G_P, G_R])).max() <= CNP_ABS
+    # <dY, Y> = <dX, X> = sum <dG_P, G_P> = sum <dG_R, G_R> (linearity in each factor)
+    L = float(np.sum(inp.dy.astype(np.float64) * out["y"]))
+    G_used = out.get("G_lp", out["G"])
+    nP = s.n // s.b
+    for v in [float(np.sum(inp.x.astype(np.float64) * out["dx"])),
+              float(np.sum(out["dG_P"] * G_used[:nP])),
+              float(np.sum(out["dG_R"] * G_used[nP:]))]:
+        assert abs(v - L) <= tol * abs(L)
+    return W0p, G_P, G_R
+
+
+def test_layer_bf16_llama8b_up_sampled():
+    """n = 4096 -> m = 14336, b = 256, T = 16384: sampled rows of y and dX, the inner
+    product identities, and the first/last blocks' dG over all tokens."""
+    s = workload_llama8b_up()
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    rng = np.random.default_rng(3)
+    rows = np.sort(np.concatenate([[0, s.T - 1], rng.choice(s.T, 62, replace=False)]))
+    W0p, G_P, G_R = _sampled_checks(out, s, inp, rows)
+    pP = out["perm_P"].astype(np.int64)
+    pR = out["perm_R"].astype(np.int64)
+    jR, jP = s.m // s.b - 1, 0
+    gP, gR = ref.layer_block_grads(inp.x, inp.dy, W0p, G_P, G_R, pP, pR, jR, jP)
+    assert norm_max_err(out["dG_R"][jR], gR) <= BF16_NORM
+    assert norm_max_err(out["dG_P"][jP], gP) <= BF16_NORM
+    dthR = ref.cnp_backward(inp.theta_R[jR:jR + 1], gR[None], s.b, s.k)[0]
+    assert norm_max_err(out["dtheta_R"][jR], dthR) <= BF16_NORM
+
+
+@pytest.mark.parametrize("idx", range(7))
+def test_layer_bf16_llama13b_block_sampled(idx):
+    s = workload_llama13b_block()[idx]
+    inp = layer_inputs(s)
+    out = run_layer(inp)
+    rng = np.random.default_rng(idx)
+    rows = np.sort(np.concatenate([[0, s.T - 1], rng.choice(s.T, 30, replace=False)]))
+    _sampled_checks(out, s, inp, rows)

@@ -384,3 +384,15 @@ def test_pins_catch_planted_mistakes():
     t = 0.5
     G_flip = ref.cnp_block(-ref.theta_to_Q(np.array([t]), 2), 4)
     assert not np.array_equal(G_flip, np.array([[0.625, 0.78125], [-0.78125, 0.625]]))
+
+
+def test_block_grads_helper_matches_full_backward():
+    n, m, b, k, T = 32, 48, 8, 4, 11
+    x, W0, tP, tR, dy, pP, pR = _small_layer(n, m, b, k, T, 23)
+    W0p = ref.merge_perm(W0, pR, pP)
+    GP, GR = ref.cnp_forward(tP, b, k), ref.cnp_forward(tR, b, k)
+    _, dGP, dGR = ref.layer_backward(x, dy, W0p, GP, GR, pP, pR)
+    for jR, jP in [(0, 0), (5, 3), (2, 1)]:
+        gP, gR = ref.layer_block_grads(x, dy, W0p, GP, GR, pP, pR, jR, jP)
+        assert np.allclose(gP, dGP[jP], rtol=0, atol=1e-13)
+        assert np.allclose(gR, dGR[jR], rtol=0, atol=1e-13)
