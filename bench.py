@@ -272,6 +272,24 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ multi-rank timing
+def max_over_ranks(local_ms: float, dist=None, device=None) -> float:
+    """The step region's device time as the maximum over ranks (replicas run in lock-step
+    between barriers; the slowest rank defines the job's time)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or \
+            dist.get_world_size() == 1:
+        return float(local_ms)
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: tokens processed by all ranks / slowest rank's time."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_poetx(args):
     import torch
@@ -340,7 +358,9 @@ def run_poetx(args):
 
     # timed region
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    uuid = str(getattr(props, "uuid", "") or "")
+    gpu_id = (uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if uuid else str(local)
+    sampler = ClockSampler(gpu_id)
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
@@ -359,14 +379,11 @@ def run_poetx(args):
     barrier()
     clocks = sampler.stop()
     elapsed_ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, dist if world > 1 else None, dev)
     if P.device_status(stream) != P.POETX_OK:
         raise RuntimeError("device status not OK after the timed region")
     ms_per_step = max_ms / args.steps
-    value = world * s.T * args.steps / (max_ms / 1e3)
+    value = job_tokens_per_s(world, s.T, args.steps, max_ms)
 
     # roofline of the dominant kernel family
     peaks, peak_src = load_peaks()
@@ -434,14 +451,11 @@ def run_poetx(args):
             e2e_step(i)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e_ms = float(te.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
         h2d = hx[0].numel() * hx[0].element_size() + hdy[0].numel() * hdy[0].element_size() + \
             hth.numel() * 4
         d2h = hy.numel() * hy.element_size() + hdx.numel() * hdx.element_size() + hdth.numel() * 4
-        e2e = {"value": world * s.T * args.e2e_steps / (e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_tokens_per_s(world, s.T, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps}
 

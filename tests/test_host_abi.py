@@ -1,0 +1,127 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every symbol the
+header declares with the binding's signatures, generates the same permutations as the
+oracle's independent generator, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import poetx_ref as ref
+from orthogonal_reparameterized_cnp_b200 import poetx as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "poetx.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(poetx_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = P.lib()
+    names = _declared_functions()
+    assert len(names) >= 15
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(P.SIGNATURES) == names  # the binding declares exactly the header's calls
+
+
+def test_status_strings_and_version():
+    lib = P.lib()
+    for st in range(8):
+        assert lib.poetx_status_string(st)
+    assert lib.poetx_status_string(99) == b"unknown status"
+    assert b"sm_100a" in lib.poetx_version()
+
+
+@pytest.mark.parametrize("seed,n", [(0, 4), (1, 1), (0, 0), (12345, 2048), (2 ** 64 - 1, 5120),
+                                    ((2 << 32) | (0 << 8) | 1, 14336)])
+def test_perm_generator_bit_exact_against_oracle(seed, n):
+    p, inv = P.make_perm(seed, n)
+    q, jnv = ref.make_perm(seed, n)
+    assert np.array_equal(p, q) and np.array_equal(inv, jnv)
+
+
+def test_make_perm_rejects_bad_arguments():
+    lib = P.lib()
+    assert lib.poetx_make_perm(0, -1, None, None) == P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_make_perm(0, 3, None, None) == P.POETX_ERR_INVALID_ARG
+    assert b"perm" in lib.poetx_last_error()
+
+
+def test_cnp_validation_before_launch():
+    lib = P.lib()
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.poetx_cnp_fwd(fake, fake, None, 2, 0, 4, fake, 1 << 20, None) == P.POETX_ERR_SHAPE
+    assert lib.poetx_cnp_fwd(fake, fake, None, 2, 8, 0, fake, 1 << 20, None) == P.POETX_ERR_SHAPE
+    assert lib.poetx_cnp_fwd(fake, fake, None, 2, 8, 17, fake, 1 << 20, None) == P.POETX_ERR_SHAPE
+    assert lib.poetx_cnp_fwd(None, fake, None, 2, 8, 4, fake, 1 << 20, None) == \
+        P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_cnp_fwd(fake, fake, None, -1, 8, 4, fake, 1 << 20, None) == \
+        P.POETX_ERR_INVALID_ARG
+    odd = ctypes.c_void_p(0x10004)
+    assert lib.poetx_cnp_fwd(odd, fake, None, 2, 8, 4, fake, 1 << 20, None) == P.POETX_ERR_ALIGN
+    # scratch below one block's need
+    assert lib.poetx_cnp_fwd(fake, fake, None, 2, 64, 4, fake, 1024, None) == \
+        P.POETX_ERR_WORKSPACE
+    assert lib.poetx_cnp_bwd(fake, None, fake, 2, 8, 4, fake, 1 << 20, None) == \
+        P.POETX_ERR_INVALID_ARG
+    # nothing to do is fine
+    assert lib.poetx_cnp_fwd(None, None, None, 0, 8, 4, None, 0, None) == P.POETX_OK
+
+
+def test_cnp_workspace_query():
+    assert P.cnp_workspace(16, 256, 4) >= 16 * 4 * 256 * 256 * 4
+    assert P.cnp_workspace(0, 256, 4) == 0
+    assert P.cnp_workspace(4, 0, 4) == 0
+    # large block counts are processed in chunks: the query stays bounded
+    assert P.cnp_workspace(44032, 64, 6) < 8 << 30
+
+
+def _desc(T=64, n=512, m=256, b=128, dtype=P.POETX_BF16, maps=True):
+    fake = 0x20000 if maps else None
+    return P.LinearDesc(T, n, m, b, dtype, fake, fake, fake, fake)
+
+
+def test_linear_validation_before_launch():
+    lib = P.lib()
+    f = ctypes.c_void_p(0x30000)
+    ws = ctypes.c_void_p(0x40000)
+    big = 1 << 40
+
+    def fwd(d, x=f, ws_bytes=big):
+        return lib.poetx_linear_fwd(ctypes.byref(d), x, f, f, f, f, None, None, ws, ws_bytes, None)
+
+    assert lib.poetx_linear_fwd(None, f, f, f, f, f, None, None, ws, big, None) == \
+        P.POETX_ERR_INVALID_ARG
+    assert fwd(_desc(n=500)) == P.POETX_ERR_SHAPE               # n % b
+    assert fwd(_desc(b=64)) == P.POETX_ERR_SHAPE                # bf16 b outside {128,256,512}
+    assert fwd(_desc(dtype=7)) == P.POETX_ERR_DTYPE
+    assert fwd(_desc(maps=False)) == P.POETX_ERR_INVALID_ARG
+    assert fwd(_desc(), x=None) == P.POETX_ERR_INVALID_ARG
+    assert fwd(_desc(), x=ctypes.c_void_p(0x30002)) == P.POETX_ERR_ALIGN
+    assert fwd(_desc(), ws_bytes=16) == P.POETX_ERR_WORKSPACE
+    assert fwd(_desc(T=0)) == P.POETX_OK                        # empty token set: no-op
+    assert fwd(_desc(T=-1)) == P.POETX_ERR_INVALID_ARG
+    d = _desc()
+    assert lib.poetx_linear_bwd(ctypes.byref(d), f, f, f, f, f, f, f, f, f, f, 2, ws, big, None) \
+        == P.POETX_ERR_INVALID_ARG                              # accumulate not 0/1
+    assert lib.poetx_linear_bwd(ctypes.byref(d), f, f, f, f, f, f, f, f, None, f, 0, ws, big,
+                                None) == P.POETX_ERR_INVALID_ARG
+
+
+def test_linear_workspace_queries():
+    d = _desc(T=8192, n=2048, m=2048, b=256)
+    fs = P.linear_fwd_workspace(d, True, True)
+    assert fs >= 2 * 8192 * 2048 * 2          # V and Z scratch
+    assert P.linear_fwd_workspace(d, False, False) >= fs + 2 * 8192 * 2048 * 2
+    assert P.linear_bwd_workspace(d, False, False) > P.linear_bwd_workspace(d, True, True)
+
+
+def test_profile_and_launch_counter_without_launches():
+    n0 = P.launch_count()
+    assert P.launch_count() == n0
