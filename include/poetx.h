@@ -133,6 +133,29 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
                   void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Cayley-Neumann forward without a caller scratch buffer.  The papers have no
+ * counterpart: this entry point exists for callers that cannot allocate device memory
+ * where they need G (a host framework that owns all device memory in its own pool and
+ * exposes none to this call site, or a loop that must not call cudaMalloc because it
+ * would synchronise the device).  Same arguments and result as poetx_cnp_fwd, minus
+ * (ws, ws_bytes).
+ *   Scratch: a fixed 32 MiB array of the library's own device memory, present on every
+ *   GPU that loads the library until the process exits.  One block's scratch must fit
+ *   it (poetx_cnp_workspace(1, b, k) <= 32 MiB: every k for b <= 512); larger b returns
+ *   POETX_ERR_WORKSPACE with a message.  Any number of blocks is processed in chunks.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any
+ *   stream capture.  The call allocates nothing and calls no allocating routine.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's
+ *   contents; nothing in it needs to start at zero (each intermediate is fully written
+ *   before it is read).  Calls whose GPU work overlaps (e.g. on two streams) race on
+ *   the array: order them on one stream or with events.
+ *   Errors: INVALID_ARG, SHAPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_cnp_fwd_static(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b,
+                         int32_t k, void* stream);
+
+/*
  * Cayley-Neumann backward (POET-X section 2.4, backward optimised the same way as the
  * forward): dtheta = d<dG, G(theta)>/dtheta for the truncated polynomial as computed,
  *   dtheta_idx(i,j) = dQ_ij - dQ_ji.

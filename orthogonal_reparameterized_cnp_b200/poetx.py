@@ -51,6 +51,7 @@ SIGNATURES = {
     "poetx_cnp_workspace": (_c_size, [_c_i32, _c_i32, _c_i32]),
     "poetx_cnp_fwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
     "poetx_cnp_bwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
+    "poetx_cnp_fwd_static": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp]),
     "poetx_linear_fwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
     "poetx_linear_bwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
     "poetx_linear_fwd": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -199,6 +200,15 @@ def cnp_fwd(theta, G, G_bf16, b: int, k: int, ws, stream=None):
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_load().poetx_cnp_fwd(_ptr(theta), _ptr(G), _ptr(G_bf16), nblk, b, k, _ptr(ws),
                                  ws_bytes, _stream(stream)), "poetx_cnp_fwd")
+
+
+def cnp_fwd_static(theta, G, G_bf16, b: int, k: int, stream=None):
+    """CNP forward with the library's fixed device scratch (no caller buffer; see the
+    header for the size limit and the sharing rules)."""
+    _require_cuda()
+    nblk = theta.shape[0]
+    _check(_load().poetx_cnp_fwd_static(_ptr(theta), _ptr(G), _ptr(G_bf16), nblk, b, k,
+                                        _stream(stream)), "poetx_cnp_fwd_static")
 
 
 def cnp_bwd(theta, dG, dtheta, b: int, k: int, ws, stream=None):
