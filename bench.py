@@ -391,7 +391,9 @@ def run_poetx(args):
     w = work.get(dominant)
     roof = None
     if w is not None:
-        per_launch_steps = dom_launches / args.steps
+        # launches of the family per step (exact, from the profiled pre-pass); the event
+        # pool may bracket fewer launches than the timed region makes
+        per_launch_steps = breakdown[dominant]["launches_per_step"]
         if w["bound"] == "tensor":
             achieved = w["flops"] / per_launch_steps / (avg_launch_ms / 1e3) / 1e12 \
                 if per_launch_steps else 0.0

@@ -235,7 +235,8 @@ int poetx_device_status(void* stream);
  *   `name` ("gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm", ...) with
  *   CUDA events on the launch stream (NULL or "" turns this off); poetx_profile_end()
  *   synchronises those events and reports the number of bracketed launches and their
- *   summed device time in milliseconds.  Events come from a fixed pool of 4096 pairs.
+ *   summed device time in milliseconds.  Events come from a fixed pool of 32768 pairs;
+ *   launches beyond it are not bracketed (the count reports how many were).
  */
 uint64_t poetx_launch_count(void);
 int poetx_profile_begin(const char* name);

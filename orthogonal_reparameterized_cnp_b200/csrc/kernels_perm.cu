@@ -70,6 +70,102 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
+// Pipelined variant for rows whose byte size is a multiple of 16: batches of R rows are
+// copied into shared memory with cp.async (two buffers: the next batch lands while the
+// current one is gathered), and each thread keeps the index map of the output vectors it
+// owns in registers for the CTA's whole life.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+constexpr int kPipeThreads = 256;
+
+template <typename E, int MAXV>
+__global__ void __launch_bounds__(kPipeThreads)
+    k_gather_rows_pipe(const E* __restrict__ in, E* __restrict__ out,
+                       const int32_t* __restrict__ row_idx, const int32_t* __restrict__ col_idx,
+                       int rows, int cols, int64_t ld_in, int64_t ld_out, int R) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int V = 16 / sizeof(E);
+  const int nvec = cols / V;                    // 16-byte vectors per row
+  const int row_elems = cols;                   // elements per staged row
+  E* buf[2] = {reinterpret_cast<E*>(smem_raw),
+               reinterpret_cast<E*>(smem_raw) + (size_t)R * row_elems};
+  const unsigned ucols = (unsigned)cols;
+
+  // index map of the output vectors this thread owns (v = tid + j * blockDim.x), two
+  // 16-bit column indices per register (cols <= 65535 on this path)
+  uint32_t idx[MAXV][V / 2];
+  int myv = 0;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int v = threadIdx.x + j * kPipeThreads;
+    if (v < nvec) {
+      ++myv;
+#pragma unroll
+      for (int e = 0; e < V; e += 2) {
+        unsigned c0 = (unsigned)__ldg(col_idx + v * V + e);
+        unsigned c1 = (unsigned)__ldg(col_idx + v * V + e + 1);
+        c0 = c0 < ucols ? c0 : ucols - 1;
+        c1 = c1 < ucols ? c1 : ucols - 1;
+        idx[j][e / 2] = c0 | (c1 << 16);
+      }
+    }
+  }
+
+  const int nbatch = (rows + R - 1) / R;
+  auto issue = [&](int batch, E* dst) {
+    const int r0 = batch * R;
+    const int nr = min(R, rows - r0);
+    for (int i = threadIdx.x; i < nr * nvec; i += kPipeThreads) {
+      const int rr = i / nvec, vv = i - rr * nvec;
+      int sr = row_idx ? row_idx[r0 + rr] : r0 + rr;
+      sr = min(max(sr, 0), rows - 1);
+      cp_async16(dst + (size_t)rr * row_elems + vv * V, in + (int64_t)sr * ld_in + vv * V);
+    }
+  };
+
+  int batch = blockIdx.x;
+  int it = 0;
+  if (batch < nbatch) issue(batch, buf[0]);
+  cp_async_commit();
+  for (; batch < nbatch; batch += gridDim.x, ++it) {
+    const int next = batch + gridDim.x;
+    if (next < nbatch) issue(next, buf[(it + 1) & 1]);
+    cp_async_commit();
+    cp_async_wait1();
+    __syncthreads();
+    const E* src = buf[it & 1];
+    const int r0 = batch * R;
+    const int nr = min(R, rows - r0);
+    for (int rr = 0; rr < nr; ++rr) {
+      const E* srow = src + (size_t)rr * row_elems;
+      E* drow = out + (int64_t)(r0 + rr) * ld_out;
+#pragma unroll
+      for (int j = 0; j < MAXV; ++j) {
+        if (j < myv) {
+          E v[V];
+#pragma unroll
+          for (int e = 0; e < V; e += 2) {
+            v[e] = srow[idx[j][e / 2] & 0xFFFFu];
+            v[e + 1] = srow[idx[j][e / 2] >> 16];
+          }
+          *reinterpret_cast<uint4*>(drow + (threadIdx.x + j * kPipeThreads) * V) =
+              *reinterpret_cast<const uint4*>(v);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // Rows too wide for shared memory: gather straight from global memory (L2 absorbs the
 // sector waste; only used beyond ~100k bf16 columns).
 template <typename E>
@@ -91,6 +187,30 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+template <typename E, int MAXV>
+cudaError_t pipe_launch(const void* in, void* out, const int32_t* row_idx, const int32_t* col_idx,
+                        int rows, int cols, int64_t ld_in, int64_t ld_out, cudaStream_t s) {
+  const size_t row_bytes = (size_t)cols * sizeof(E);
+  // R rows per batch: ~32 KB per buffer, two buffers per CTA
+  int R = (int)((32 * 1024) / row_bytes);
+  R = R < 1 ? 1 : (R > 16 ? 16 : R);
+  const size_t smem = 2 * (size_t)R * row_bytes;
+  cudaError_t e = cudaFuncSetAttribute(k_gather_rows_pipe<E, MAXV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+  if (e != cudaSuccess) return e;
+  const int nbatch = (rows + R - 1) / R;
+  int per_sm = (int)((200 * 1024) / (smem + 1024));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+  int grid = num_sms() * per_sm;
+  if (grid > nbatch) grid = nbatch;
+  begin_launch("permute", s);
+  k_gather_rows_pipe<E, MAXV><<<grid, kPipeThreads, smem, s>>>(
+      static_cast<const E*>(in), static_cast<E*>(out), row_idx, col_idx, rows, cols, ld_in,
+      ld_out, R);
+  end_launch("permute", s);
+  return cudaGetLastError();
+}
+
 template <typename E>
 cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
                         const int32_t* col_idx, int rows, int cols, int64_t ld_in,
@@ -98,6 +218,18 @@ cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
   if (rows <= 0 || cols <= 0) return cudaSuccess;
   const size_t row_bytes = ((size_t)cols * sizeof(E) + 15) & ~size_t(15);
   const int sms = num_sms();
+  constexpr int V = 16 / sizeof(E);
+  const bool vec_ok = (cols % V == 0) && (ld_in % V == 0) && (ld_out % V == 0) &&
+                      ((reinterpret_cast<uintptr_t>(in) & 15) == 0) &&
+                      ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+  const int nvec = cols / V;
+  if (vec_ok && cols <= 65535 && nvec <= 8 * kPipeThreads && 2 * row_bytes <= 96 * 1024) {
+    const int need = (nvec + kPipeThreads - 1) / kPipeThreads;
+    if (need <= 1) return pipe_launch<E, 1>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+    if (need <= 2) return pipe_launch<E, 2>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+    if (need <= 4) return pipe_launch<E, 4>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+    return pipe_launch<E, 8>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
+  }
   if (row_bytes <= (size_t)kMaxSmemRowBytes) {
     static bool attr_set = false;
     if (!attr_set) {

@@ -14,7 +14,6 @@ namespace poetx {
 namespace {
 
 constexpr int kThreads = 256;  // 16 x 16 thread grid
-constexpr int kBK = 16;
 
 struct SgemmDev {
   const float* A;
@@ -50,32 +49,34 @@ struct SgemmDev {
 };
 
 // Thread (tx, ty) owns rows g*(16*VEC) + ty*VEC + v and the same pattern of columns.
-template <int TM>
+template <int TM, int BK>
 struct Tile {
   static constexpr int VEC = TM < 4 ? TM : 4;
   static constexpr int NG = TM / VEC;
   static constexpr int BM = 16 * TM;
-  static constexpr int LOADS = BM * kBK / kThreads;  // elements per thread per operand tile
+  static constexpr int LOADS = BM * BK / kThreads;  // elements per thread per operand tile
+  // the mirror half of SYM / SYMSKEW tiles is staged in smem when it fits the A buffers
+  static constexpr bool STAGE = (BM * (BM + 1)) <= 2 * BK * (BM + 4);
 };
 
-template <int TM>
-__device__ __forceinline__ void load_tile_regs(float (&r)[Tile<TM>::LOADS], const float* X,
+template <int TM, int BK>
+__device__ __forceinline__ void load_tile_regs(float (&r)[Tile<TM, BK>::LOADS], const float* X,
                                                int64_t ldx, int trans, int row0, int k0,
                                                int rows, int kdim, float scale, bool is_b) {
-  // Loads the (BM x kBK) tile of op(X) (for A) or the (kBK x BN) tile of op(B), as
-  // element (row, k) with row in [row0, row0+BM), k in [k0, k0+kBK).
+  // Loads the (BM x BK) tile of op(X) (for A) or the (BK x BN) tile of op(B), as
+  // element (row, k) with row in [row0, row0+BM), k in [k0, k0+BK).
   // A: op(A)[i][k] = trans ? X[k*ld + i] : X[i*ld + k]
   // B: op(B)[k][j] = trans ? X[j*ld + k] : X[k*ld + j]   (j plays the role of row)
-  constexpr int BM = Tile<TM>::BM;
+  constexpr int BM = Tile<TM, BK>::BM;
   const int tid = threadIdx.x;
   const bool k_contig = is_b ? (trans != 0) : (trans == 0);
 #pragma unroll
-  for (int l = 0; l < Tile<TM>::LOADS; ++l) {
+  for (int l = 0; l < Tile<TM, BK>::LOADS; ++l) {
     int idx = tid + l * kThreads;
     int i, k;
     if (k_contig) {
-      i = idx / kBK;
-      k = idx % kBK;
+      i = idx / BK;
+      k = idx % BK;
     } else {
       k = idx / BM;
       i = idx % BM;
@@ -90,20 +91,20 @@ __device__ __forceinline__ void load_tile_regs(float (&r)[Tile<TM>::LOADS], cons
   }
 }
 
-template <int TM>
-__device__ __forceinline__ void store_tile_smem(const float (&r)[Tile<TM>::LOADS],
-                                                float (*S)[Tile<TM>::BM + 4], int trans,
+template <int TM, int BK>
+__device__ __forceinline__ void store_tile_smem(const float (&r)[Tile<TM, BK>::LOADS],
+                                                float (*S)[Tile<TM, BK>::BM + 4], int trans,
                                                 bool is_b) {
-  constexpr int BM = Tile<TM>::BM;
+  constexpr int BM = Tile<TM, BK>::BM;
   const int tid = threadIdx.x;
   const bool k_contig = is_b ? (trans != 0) : (trans == 0);
 #pragma unroll
-  for (int l = 0; l < Tile<TM>::LOADS; ++l) {
+  for (int l = 0; l < Tile<TM, BK>::LOADS; ++l) {
     int idx = tid + l * kThreads;
     int i, k;
     if (k_contig) {
-      i = idx / kBK;
-      k = idx % kBK;
+      i = idx / BK;
+      k = idx % BK;
     } else {
       k = idx / BM;
       i = idx % BM;
@@ -112,12 +113,12 @@ __device__ __forceinline__ void store_tile_smem(const float (&r)[Tile<TM>::LOADS
   }
 }
 
-template <int TM>
-__global__ void __launch_bounds__(kThreads) k_sgemm(SgemmDev p) {
-  using TL = Tile<TM>;
+template <int TM, int BK>
+__global__ void __launch_bounds__(kThreads, TM <= 4 ? 2 : 1) k_sgemm(SgemmDev p) {
+  using TL = Tile<TM, BK>;
   constexpr int BM = TL::BM, VEC = TL::VEC, NG = TL::NG;
-  __shared__ __align__(16) float As[2][kBK][BM + 4];
-  __shared__ __align__(16) float Bs[2][kBK][BM + 4];
+  __shared__ __align__(16) float As[2][BK][BM + 4];
+  __shared__ __align__(16) float Bs[2][BK][BM + 4];
 
   const int tile_lin = blockIdx.x;
   const int bz = tile_lin / p.tiles_per_batch;
@@ -144,27 +145,29 @@ __global__ void __launch_bounds__(kThreads) k_sgemm(SgemmDev p) {
     for (int c = 0; c < TM; ++c) acc[a][c] = 0.f;
 
   float ra[TL::LOADS], rb[TL::LOADS];
-  const int nk1 = (p.K + kBK - 1) / kBK;
-  const int nk2 = p.A2 ? (p.K2 + kBK - 1) / kBK : 0;
+  const int nk1 = (p.K + BK - 1) / BK;
+  const int nk2 = p.A2 ? (p.K2 + BK - 1) / BK : 0;
   const int nkt = nk1 + nk2;
 
   auto load = [&](int kt) {
     if (kt < nk1) {
-      load_tile_regs<TM>(ra, p.A + bz * p.sA, p.lda, p.transA, m0, kt * kBK, p.M, p.K, 1.f,
-                         false);
-      load_tile_regs<TM>(rb, p.B + bz * p.sB, p.ldb, p.transB, n0, kt * kBK, p.N, p.K, 1.f, true);
+      load_tile_regs<TM, BK>(ra, p.A + bz * p.sA, p.lda, p.transA, m0, kt * BK, p.M, p.K, 1.f,
+                             false);
+      load_tile_regs<TM, BK>(rb, p.B + bz * p.sB, p.ldb, p.transB, n0, kt * BK, p.N, p.K, 1.f,
+                             true);
     } else {
-      int k2 = (kt - nk1) * kBK;
-      load_tile_regs<TM>(ra, p.A2 + bz * p.sA2, p.lda2, p.transA2, m0, k2, p.M, p.K2, p.alpha2,
-                         false);
-      load_tile_regs<TM>(rb, p.B2 + bz * p.sB2, p.ldb2, p.transB2, n0, k2, p.N, p.K2, 1.f, true);
+      int k2 = (kt - nk1) * BK;
+      load_tile_regs<TM, BK>(ra, p.A2 + bz * p.sA2, p.lda2, p.transA2, m0, k2, p.M, p.K2,
+                             p.alpha2, false);
+      load_tile_regs<TM, BK>(rb, p.B2 + bz * p.sB2, p.ldb2, p.transB2, n0, k2, p.N, p.K2, 1.f,
+                             true);
     }
   };
   auto store = [&](int kt, int buf) {
     int ta = kt < nk1 ? p.transA : p.transA2;
     int tb = kt < nk1 ? p.transB : p.transB2;
-    store_tile_smem<TM>(ra, As[buf], ta, false);
-    store_tile_smem<TM>(rb, Bs[buf], tb, true);
+    store_tile_smem<TM, BK>(ra, As[buf], ta, false);
+    store_tile_smem<TM, BK>(rb, Bs[buf], tb, true);
   };
 
   if (nkt > 0) {
@@ -176,7 +179,7 @@ __global__ void __launch_bounds__(kThreads) k_sgemm(SgemmDev p) {
     const int buf = kt & 1;
     if (kt + 1 < nkt) load(kt + 1);
 #pragma unroll
-    for (int k = 0; k < kBK; ++k) {
+    for (int k = 0; k < BK; ++k) {
       float a[TM], b[TM];
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
@@ -207,19 +210,25 @@ __global__ void __launch_bounds__(kThreads) k_sgemm(SgemmDev p) {
   float* C = p.C + boff;
   __nv_bfloat16* Cb = p.Cb ? p.Cb + boff : nullptr;
   float* C2 = p.C2 ? p.C2 + boff : nullptr;
+  const bool structured = p.mode != SG_FULL;
+  // mirror half staged in smem (coalesced transposed store), when the tile fits
+  constexpr bool STAGE = TL::STAGE;
+  float (*Ms)[BM + 1] = reinterpret_cast<float (*)[BM + 1]>(&As[0][0][0]);
+  float (*Ms2)[BM + 1] = reinterpret_cast<float (*)[BM + 1]>(&Bs[0][0][0]);
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
     for (int vi = 0; vi < VEC; ++vi) {
-      const int i = m0 + gi * 16 * VEC + ty * VEC + vi;
-      if (i >= p.M) continue;
+      const int il = gi * 16 * VEC + ty * VEC + vi;
+      const int i = m0 + il;
 #pragma unroll
       for (int gj = 0; gj < NG; ++gj)
 #pragma unroll
         for (int vj = 0; vj < VEC; ++vj) {
-          const int j = n0 + gj * 16 * VEC + tx * VEC + vj;
-          if (j >= p.N) continue;
-          if (p.mode != SG_FULL && I == J && i > j) continue;  // mirror of (j, i)
+          const int jl = gj * 16 * VEC + tx * VEC + vj;
+          const int j = n0 + jl;
+          if (i >= p.M || j >= p.N) continue;
+          if (structured && I == J && i > j) continue;  // mirror of (j, i)
           const int64_t ij = (int64_t)i * p.ldc + j;
           const float a = acc[gi * VEC + vi][gj * VEC + vj];
           float sym = (i == j) ? p.diag : 0.f;
@@ -231,33 +240,273 @@ __global__ void __launch_bounds__(kThreads) k_sgemm(SgemmDev p) {
           }
           float skew = p.alpha * a;
           if (p.skew_add) skew += p.skew_c * p.skew_add[boff + ij];
-          const int64_t ji = (int64_t)j * p.ldc + i;
+          float v, vm, v2 = 0.f;
           if (p.mode == SG_SYMSKEW) {
-            if (i == j) {
-              C[ij] = sym;
-              if (Cb) Cb[ij] = __float2bfloat16_rn(sym);
-            } else {
-              C[ij] = sym + skew;
-              C[ji] = sym - skew;
-              if (Cb) {
-                Cb[ij] = __float2bfloat16_rn(sym + skew);
-                Cb[ji] = __float2bfloat16_rn(sym - skew);
-              }
-            }
+            v = (i == j) ? sym : sym + skew;   // G_ij = E_ij + O_ij (O_ii = 0)
+            vm = sym - skew;                   // G_ji = E_ij - O_ij
           } else {
-            const float v = skew + sym;
-            C[ij] = v;
-            if (Cb) Cb[ij] = __float2bfloat16_rn(v);
-            const float v2 = p.alpha_c2 * a + sym2;
-            if (C2) C2[ij] = v2;
-            if (p.mode == SG_SYM && i != j) {
-              C[ji] = v;
-              if (Cb) Cb[ji] = __float2bfloat16_rn(v);
+            v = skew + sym;
+            vm = v;
+            v2 = p.alpha_c2 * a + sym2;
+          }
+          C[ij] = v;
+          if (Cb) Cb[ij] = __float2bfloat16_rn(v);
+          if (C2 && !(p.mode == SG_SYMSKEW)) C2[ij] = v2;
+          if (structured && i != j) {
+            if constexpr (STAGE) {
+              Ms[il][jl] = vm;
+              if (C2) Ms2[il][jl] = v2;
+            } else {
+              const int64_t ji = (int64_t)j * p.ldc + i;
+              C[ji] = vm;
+              if (Cb) Cb[ji] = __float2bfloat16_rn(vm);
               if (C2) C2[ji] = v2;
             }
           }
         }
     }
+  if constexpr (STAGE) {
+    if (structured) {
+      __syncthreads();
+      // C[n0 + jl][m0 + il] = Ms[il][jl] for the strictly-upper part of the tile
+      for (int e = threadIdx.x; e < BM * BM; e += kThreads) {
+        const int jl = e / BM, il = e - jl * BM;
+        const int i = m0 + il, j = n0 + jl;
+        if (i >= p.M || j >= p.N) continue;
+        if (I == J && il >= jl) continue;
+        const int64_t ji = (int64_t)j * p.ldc + i;
+        const float vm = Ms[il][jl];
+        C[ji] = vm;
+        if (Cb) Cb[ji] = __float2bfloat16_rn(vm);
+        if (C2) C2[ji] = Ms2[il][jl];
+      }
+    }
+  }
+}
+
+// ---- square-block products (b % 64 == 0, no transposes): the CNP's workhorse ---------
+// 64 x 64 output tile per CTA, 128 threads, thread (tx = tid & 15, ty = tid >> 4) owns rows
+// ty*8 .. ty*8+7 and columns tx*4 .. tx*4+3.  K tiles of 16, register-prefetched.  No
+// bounds checks: every tile is full.  A symmetric or skew A (a_sym = +-1) is read by rows
+// as its own transpose, so both operands go to shared memory with 16-byte stores.
+constexpr int kMMThreads = 128;
+constexpr int kMMBK = 16;
+constexpr int kMMLD = 64 + 4;
+
+struct MMSmem {
+  float As[2][kMMBK][kMMLD];
+  float Bs[2][kMMBK][kMMLD];
+};
+constexpr int kMMStage = 2 * 64 * 65;  // two 64 x 65 staging tiles for the mirror half
+constexpr int kMMSmemFloats =
+    (int)(sizeof(MMSmem) / 4) > kMMStage ? (int)(sizeof(MMSmem) / 4) : kMMStage;
+
+__device__ __forceinline__ float4 ldg4(const float* p) {
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+
+template <int KT_UNUSED = 0>
+__global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym, int a2_sym) {
+  __shared__ __align__(16) float smem[kMMSmemFloats];
+  MMSmem& S = *reinterpret_cast<MMSmem*>(smem);
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+
+  const int bz = blockIdx.x / p.tiles_per_batch;
+  int t = blockIdx.x - bz * p.tiles_per_batch;
+  int I, J;
+  if (p.mode == SG_FULL) {
+    I = t / p.tiles_n;
+    J = t - I * p.tiles_n;
+  } else {
+    I = 0;
+    while (t >= p.nt - I) {
+      t -= p.nt - I;
+      ++I;
+    }
+    J = I + t;
+  }
+  const int m0 = I * 64, n0 = J * 64;
+  const int b = p.ldc;  // square blocks: ld = b for every operand
+
+  float acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+
+  const int nk1 = p.K / kMMBK;
+  const int nk2 = p.A2 ? p.K2 / kMMBK : 0;
+  const int nkt = nk1 + nk2;
+
+  float4 ra[2], rb[2];
+  // global -> registers for k tile kt
+  auto load = [&](int kt) {
+    const bool first = kt < nk1;
+    const float* A = first ? p.A + bz * p.sA : p.A2 + bz * p.sA2;
+    const float* B = first ? p.B + bz * p.sB : p.B2 + bz * p.sB2;
+    const int k0 = (first ? kt : kt - nk1) * kMMBK;
+    const int sym = first ? a_sym : a2_sym;
+    const float sc = first ? 1.f : p.alpha2;
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      const int f = tid + l * kMMThreads;  // 0..255
+      // B tile: 16 rows (k) x 64 cols, 16 float4 per row
+      const int br = f >> 4, bc = (f & 15) * 4;
+      rb[l] = ldg4(B + (int64_t)(k0 + br) * b + n0 + bc);
+      float4 a;
+      if (sym != 0) {  // As[k][i] = sym * A[k][i]: rows of A are its transpose's columns
+        a = ldg4(A + (int64_t)(k0 + br) * b + m0 + bc);
+        const float s2 = sc * (float)sym;
+        a.x *= s2; a.y *= s2; a.z *= s2; a.w *= s2;
+      } else {         // As[k][i] = A[i][k]: 64 rows x 4 float4 of k
+        const int ar = f >> 2, ac = (f & 3) * 4;
+        a = ldg4(A + (int64_t)(m0 + ar) * b + k0 + ac);
+        a.x *= sc; a.y *= sc; a.z *= sc; a.w *= sc;
+      }
+      ra[l] = a;
+    }
+  };
+  auto store = [&](int kt, int buf) {
+    const int sym = kt < nk1 ? a_sym : a2_sym;
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      const int f = tid + l * kMMThreads;
+      const int br = f >> 4, bc = (f & 15) * 4;
+      *reinterpret_cast<float4*>(&S.Bs[buf][br][bc]) = rb[l];
+      if (sym != 0) {
+        *reinterpret_cast<float4*>(&S.As[buf][br][bc]) = ra[l];
+      } else {
+        const int ar = f >> 2, ac = (f & 3) * 4;
+        S.As[buf][ac + 0][ar] = ra[l].x;
+        S.As[buf][ac + 1][ar] = ra[l].y;
+        S.As[buf][ac + 2][ar] = ra[l].z;
+        S.As[buf][ac + 3][ar] = ra[l].w;
+      }
+    }
+  };
+
+  if (nkt > 0) {
+    load(0);
+    store(0, 0);
+  }
+  __syncthreads();
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nkt) load(kt + 1);
+#pragma unroll
+    for (int k = 0; k < kMMBK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&S.As[buf][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&S.As[buf][k][ty * 8 + 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&S.Bs[buf][k][tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+    }
+    if (kt + 1 < nkt) store(kt + 1, buf ^ 1);
+    __syncthreads();
+  }
+
+  // ---- epilogue (same semantics as k_sgemm)
+  const int64_t boff = (int64_t)bz * p.sC;
+  float* C = p.C + boff;
+  __nv_bfloat16* Cb = p.Cb ? p.Cb + boff : nullptr;
+  float* C2 = p.C2 ? p.C2 + boff : nullptr;
+  const bool structured = p.mode != SG_FULL;
+  float (*Ms)[65] = reinterpret_cast<float (*)[65]>(smem);
+  float (*Ms2)[65] = reinterpret_cast<float (*)[65]>(smem + 64 * 65);
+  const int jl0 = tx * 4;
+  const int j0 = n0 + jl0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int il = ty * 8 + r;
+    const int i = m0 + il;
+    const int64_t row = (int64_t)i * b;
+    float sym[4] = {0.f, 0.f, 0.f, 0.f}, sym2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (i == j0 + c) {
+        sym[c] = p.diag;
+        sym2[c] = p.diag2;
+      }
+    for (int q = 0; q < p.nadd; ++q) {
+      const float4 x = ldg4(p.add[q] + boff + row + j0);
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        sym[c] += p.addc[q] * xs[c];
+        sym2[c] += p.addc2[q] * xs[c];
+      }
+    }
+    float skew[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) skew[c] = p.alpha * acc[r][c];
+    if (p.skew_add) {
+      const float4 x = ldg4(p.skew_add + boff + row + j0);
+      skew[0] += p.skew_c * x.x; skew[1] += p.skew_c * x.y;
+      skew[2] += p.skew_c * x.z; skew[3] += p.skew_c * x.w;
+    }
+    float v[4], vm[4], v2[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + c;
+      if (p.mode == SG_SYMSKEW) {
+        v[c] = (i == j) ? sym[c] : sym[c] + skew[c];
+        vm[c] = sym[c] - skew[c];
+      } else {
+        v[c] = skew[c] + sym[c];
+        vm[c] = v[c];
+      }
+      v2[c] = p.alpha_c2 * acc[r][c] + sym2[c];
+    }
+    // in diagonal tiles of structured outputs only the upper triangle is written here
+    if (structured && I == J) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = j0 + c;
+        if (i <= j) {
+          C[row + j] = v[c];
+          if (Cb) Cb[row + j] = __float2bfloat16_rn(v[c]);
+          if (C2) C2[row + j] = v2[c];
+        }
+      }
+    } else {
+      *reinterpret_cast<float4*>(C + row + j0) = make_float4(v[0], v[1], v[2], v[3]);
+      if (Cb) {
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t*>(&h0);
+        o.y = *reinterpret_cast<uint32_t*>(&h1);
+        *reinterpret_cast<uint2*>(Cb + row + j0) = o;
+      }
+      if (C2) *reinterpret_cast<float4*>(C2 + row + j0) = make_float4(v2[0], v2[1], v2[2], v2[3]);
+    }
+    if (structured) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        Ms[il][jl0 + c] = vm[c];
+        if (C2) Ms2[il][jl0 + c] = v2[c];
+      }
+    }
+  }
+  if (structured) {
+    // the main loop ended with a barrier, so the staging tiles may overwrite As/Bs; one
+    // more barrier makes every thread's staged values visible
+    __syncthreads();
+    for (int e = tid; e < 64 * 64; e += kMMThreads) {
+      const int jl = e >> 6, il = e & 63;
+      if (I == J && il >= jl) continue;
+      const int64_t ji = (int64_t)(n0 + jl) * b + m0 + il;
+      const float vmv = Ms[il][jl];
+      C[ji] = vmv;
+      if (Cb) Cb[ji] = __float2bfloat16_rn(vmv);
+      if (C2) C2[ji] = Ms2[il][jl];
+    }
+  }
 }
 
 // ---- tile-pair elementwise kernels (32 x 32 tiles, I <= J) --------------------------
@@ -405,10 +654,58 @@ __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __re
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+SgemmDev make_dev(const SgemmArgs& a) {
+  SgemmDev p;
+  p.A = a.A; p.lda = a.lda; p.sA = a.sA;
+  p.B = a.B; p.ldb = a.ldb; p.sB = a.sB;
+  p.transA = a.transA; p.transB = a.transB;
+  p.A2 = a.A2; p.lda2 = a.lda2; p.sA2 = a.sA2;
+  p.B2 = a.B2; p.ldb2 = a.ldb2; p.sB2 = a.sB2;
+  p.transA2 = a.transA2; p.transB2 = a.transB2;
+  p.K2 = a.K2; p.alpha2 = a.alpha2;
+  p.C = a.C; p.ldc = a.ldc; p.sC = a.sC;
+  p.Cb = static_cast<__nv_bfloat16*>(a.C_bf16);
+  p.C2 = a.C2; p.alpha_c2 = a.alpha_c2; p.diag2 = a.diag2;
+  p.M = a.M; p.N = a.N; p.K = a.K; p.batch = a.batch;
+  p.alpha = a.alpha;
+  p.nadd = a.nadd;
+  for (int q = 0; q < 8; ++q) {
+    p.add[q] = a.add[q];
+    p.addc[q] = a.addc[q];
+    p.addc2[q] = a.addc2[q];
+  }
+  p.skew_add = a.skew_add;
+  p.skew_c = a.skew_c;
+  p.diag = a.diag;
+  p.mode = a.mode;
+  return p;
+}
+
+cudaError_t launch_cnp_mm(const SgemmArgs& a, cudaStream_t s) {
+  SgemmDev p = make_dev(a);
+  const int nt = a.M / 64;
+  p.nt = nt;
+  p.tiles_n = nt;
+  p.tiles_per_batch = a.mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
+  const int64_t grid = (int64_t)p.tiles_per_batch * a.batch;
+  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  begin_launch("cnp_sgemm", s);
+  k_cnp_mm<0><<<(unsigned)grid, kMMThreads, 0, s>>>(p, a.a_sym, a.a2_sym);
+  end_launch("cnp_sgemm", s);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s) {
   if (a.batch <= 0 || a.M <= 0 || a.N <= 0) return cudaSuccess;
+  // square b x b blocks with b % 64 == 0 and no transposed operand: the lean kernel
+  const int bsq = a.M;
+  const bool square = a.M == a.N && a.K == bsq && (!a.A2 || a.K2 == bsq) && bsq % 64 == 0 &&
+                      a.lda == bsq && a.ldb == bsq && a.ldc == bsq &&
+                      (!a.A2 || (a.lda2 == bsq && a.ldb2 == bsq)) && !a.transA && !a.transB &&
+                      !a.transA2 && !a.transB2 && a.nadd <= 8;
+  if (square) return launch_cnp_mm(a, s);
   SgemmDev p;
   p.A = a.A; p.lda = a.lda; p.sA = a.sA;
   p.B = a.B; p.ldb = a.ldb; p.sB = a.sB;
@@ -451,11 +748,11 @@ cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s) {
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
   begin_launch("cnp_sgemm", s);
   if (TM == 8)
-    k_sgemm<8><<<(unsigned)grid, kThreads, 0, s>>>(p);
+    k_sgemm<8, 16><<<(unsigned)grid, kThreads, 0, s>>>(p);
   else if (TM == 4)
-    k_sgemm<4><<<(unsigned)grid, kThreads, 0, s>>>(p);
+    k_sgemm<4, 32><<<(unsigned)grid, kThreads, 0, s>>>(p);
   else
-    k_sgemm<2><<<(unsigned)grid, kThreads, 0, s>>>(p);
+    k_sgemm<2, 32><<<(unsigned)grid, kThreads, 0, s>>>(p);
   end_launch("cnp_sgemm", s);
   return cudaGetLastError();
 }

@@ -62,7 +62,7 @@ static std::atomic<uint64_t> g_launches{0};
 static std::mutex g_prof_mu;
 static std::string g_prof_family;
 static bool g_prof_on = false;
-static constexpr int kEventPairs = 4096;
+static constexpr int kEventPairs = 32768;
 static std::vector<cudaEvent_t> g_ev_start, g_ev_stop;
 static int g_prof_used = 0;
 
@@ -278,6 +278,7 @@ int cnp_powers(const float* Q, std::vector<float*>& Pw, float* Fp, const CnpPoly
   for (int j = 1; j <= d; ++j) {
     SgemmArgs g = (j == 1) ? sq_gemm(Q, 0, Q, 0, Pw[1], nb, b, SG_SYM)
                            : sq_gemm(Pw[1], 0, Pw[j - 1], 0, Pw[j], nb, b, SG_SYM);
+    g.a_sym = (j == 1) ? -1 : 1;  // Q is skew, S symmetric
     if (j == d) {
       g.C2 = Fp;
       g.alpha_c2 = P.f[d];
@@ -320,6 +321,7 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
     // G = E + Q F with E = e_0 I + sum_j e_j P_j (symmetric) and Q F = Q F' + f_0 Q (skew):
     // only upper tiles are multiplied; G_ji = E_ij - (QF)_ij.
     SgemmArgs g = sq_gemm(Q, 0, Fp, 0, G + b0 * bb, nb, b, SG_SYMSKEW);
+    g.a_sym = -1;
     g.C_bf16 = G_bf16 ? static_cast<void*>(static_cast<uint16_t*>(G_bf16) + b0 * bb) : nullptr;
     g.diag = P.e[0];
     for (int j = 1; j <= d; ++j) {
@@ -366,7 +368,11 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
     if (st2 != POETX_OK) return st2;
     // D = Q dG; the adjoint reaching F is Q^T dG = -D.
-    POETX_CUDA(launch_sgemm(sq_gemm(Q, 0, dg, 0, D, nb, b, SG_FULL), s), "cnp D");
+    {
+      SgemmArgs gd = sq_gemm(Q, 0, dg, 0, D, nb, b, SG_FULL);
+      gd.a_sym = -1;
+      POETX_CUDA(launch_sgemm(gd, s), "cnp D");
+    }
     // N_j = M_j + M_j^T with M_j = e_j dG - f_j D  (upstream of S^j through E and F)
     for (int j0 = 1; j0 <= d; j0 += 4) {
       const int cnt = (d - j0 + 1) < 4 ? (d - j0 + 1) : 4;
@@ -385,6 +391,7 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     if (d >= 2) {
       const float* S = Pw[1];
       SgemmArgs g = sq_gemm(Nw[d], 0, S, 0, Pm, nb, b, SG_FULL);  // Pm = N_d S
+      g.a_sym = 1;
       if (d >= 3) {  // R_{d-2} = N_{d-1} + Pm
         g.C2 = R;
         g.alpha_c2 = 1.f;
@@ -413,6 +420,7 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
         POETX_CUDA(launch_sgemm(gr, s), "cnp R");
         // T_a = R_a + S T_{a+1}  (symmetric: upper tiles + mirror)
         SgemmArgs gt = sq_gemm(S, 0, Tc, 0, Tn, nb, b, SG_SYM);
+        gt.a_sym = 1;
         gt.add[0] = Rn;
         gt.addc[0] = 1.f;
         gt.nadd = 1;
@@ -428,6 +436,7 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     ga.B2 = Q; ga.ldb2 = b; ga.sB2 = bb;
     ga.K2 = b;
     ga.alpha2 = -1.f;
+    ga.a2_sym = 1;  // Y is symmetric
     ga.add[0] = dg;
     ga.addc[0] = P.f[0];
     ga.nadd = 1;

@@ -70,6 +70,9 @@ struct SgemmArgs {
   float skew_c = 0.f;
   float diag = 0.f;
   int mode = SG_FULL;
+  // structure of A and A2 when known: 0 general, +1 symmetric, -1 skew-symmetric (lets
+  // the square-block kernel read them already transposed)
+  int a_sym = 0, a2_sym = 0;
 };
 cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s);
 
