@@ -298,17 +298,36 @@ struct MMSmem {
   float Bs[2][kMMBK][kMMLD];
 };
 constexpr int kMMStage = 2 * 64 * 65;  // two 64 x 65 staging tiles for the mirror half
-constexpr int kMMSmemFloats =
-    (int)(sizeof(MMSmem) / 4) > kMMStage ? (int)(sizeof(MMSmem) / 4) : kMMStage;
+constexpr int kMMStages = 4;            // cp.async ring depth of the row-operand path
+constexpr int kMMStageFloats = 2 * kMMBK * kMMLD;
+constexpr int kMMSmemFloats = kMMStages * kMMStageFloats > kMMStage
+                                  ? kMMStages * kMMStageFloats : kMMStage;
+
+__device__ __forceinline__ void mm_cp_async16(float* smem_dst, const float* gsrc) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void mm_cp_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void mm_cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ float4 ldg4(const float* p) {
   return __ldg(reinterpret_cast<const float4*>(p));
 }
 
-template <int KT_UNUSED = 0>
+// ROWS: every A operand of the launch is readable by rows (symmetric, skew, or given as
+// its transpose), so A and B tiles stream through a 4-deep cp.async ring; the sign of a
+// skew operand and alpha2 = -1 are applied to the accumulators (acc_scale below).
+// !ROWS: register-staged loads with a transposing store for a general A.
+template <bool ROWS>
 __global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym, int a2_sym) {
   __shared__ __align__(16) float smem[kMMSmemFloats];
   MMSmem& S = *reinterpret_cast<MMSmem*>(smem);
+  (void)S;
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
 
@@ -339,6 +358,69 @@ __global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym,
   const int nk2 = p.A2 ? p.K2 / kMMBK : 0;
   const int nkt = nk1 + nk2;
 
+  // multiplier that turns the accumulators into op(A) op(B) + alpha2 op(A2) op(B2)
+  float acc_scale = 1.f;
+  if constexpr (ROWS) {
+    const float s1 = a_sym < 0 ? -1.f : 1.f;
+    const float s2 = a2_sym < 0 ? -1.f : 1.f;
+    const float boundary = s1 * s2 * p.alpha2;  // applied before the second product
+    acc_scale = nk2 > 0 ? s2 * p.alpha2 : s1;
+    auto As_ = [&](int st) {
+      return reinterpret_cast<float (*)[kMMLD]>(smem + st * kMMStageFloats);
+    };
+    auto Bs_ = [&](int st) {
+      return reinterpret_cast<float (*)[kMMLD]>(smem + st * kMMStageFloats + kMMBK * kMMLD);
+    };
+    auto issue = [&](int kt) {
+      if (kt < nkt) {
+        const bool first = kt < nk1;
+        const float* A = first ? p.A + bz * p.sA : p.A2 + bz * p.sA2;
+        const float* B = first ? p.B + bz * p.sB : p.B2 + bz * p.sB2;
+        const int k0 = (first ? kt : kt - nk1) * kMMBK;
+        const int st = kt % kMMStages;
+        float (*As)[kMMLD] = As_(st);
+        float (*Bs)[kMMLD] = Bs_(st);
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+          const int f = tid + l * kMMThreads;
+          const int r = f >> 4, c4 = (f & 15) * 4;
+          mm_cp_async16(&As[r][c4], A + (int64_t)(k0 + r) * b + m0 + c4);
+          mm_cp_async16(&Bs[r][c4], B + (int64_t)(k0 + r) * b + n0 + c4);
+        }
+      }
+      mm_cp_commit();
+    };
+#pragma unroll
+    for (int st = 0; st < kMMStages - 1; ++st) issue(st);
+    for (int kt = 0; kt < nkt; ++kt) {
+      mm_cp_wait<kMMStages - 2>();
+      __syncthreads();
+      issue(kt + kMMStages - 1);
+      if (nk2 > 0 && kt == nk1) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] *= boundary;
+      }
+      const int st = kt % kMMStages;
+      float (*As)[kMMLD] = As_(st);
+      float (*Bs)[kMMLD] = Bs_(st);
+#pragma unroll
+      for (int k = 0; k < kMMBK; ++k) {
+        const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 8]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&As[k][ty * 8 + 4]);
+        const float4 bv = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+      }
+    }
+    mm_cp_wait<0>();
+    __syncthreads();
+  } else {
   float4 ra[2], rb[2];
   // global -> registers for k tile kt
   auto load = [&](int kt) {
@@ -346,7 +428,7 @@ __global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym,
     const float* A = first ? p.A + bz * p.sA : p.A2 + bz * p.sA2;
     const float* B = first ? p.B + bz * p.sB : p.B2 + bz * p.sB2;
     const int k0 = (first ? kt : kt - nk1) * kMMBK;
-    const int sym = first ? a_sym : a2_sym;
+    const int sym = (first ? a_sym : a2_sym) == 2 ? 1 : (first ? a_sym : a2_sym);
     const float sc = first ? 1.f : p.alpha2;
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
@@ -409,6 +491,7 @@ __global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym,
     if (kt + 1 < nkt) store(kt + 1, buf ^ 1);
     __syncthreads();
   }
+  }  // !ROWS
 
   // ---- epilogue (same semantics as k_sgemm)
   const int64_t boff = (int64_t)bz * p.sC;
@@ -441,6 +524,8 @@ __global__ void __launch_bounds__(kMMThreads, 4) k_cnp_mm(SgemmDev p, int a_sym,
         sym2[c] += p.addc2[q] * xs[c];
       }
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] *= acc_scale;
     float skew[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) skew[c] = p.alpha * acc[r][c];
@@ -558,6 +643,7 @@ struct SymcombDev {
   float* out[4];
   float coef[4][4];
   int nin, nout;
+  float* tout;  // optional: tout = X[0]^T
 };
 
 __global__ void __launch_bounds__(256) k_symcomb(SymcombDev p, int b, int nt, int pairs) {
@@ -583,6 +669,15 @@ __global__ void __launch_bounds__(256) k_symcomb(SymcombDev p, int b, int nt, in
     for (int r = ty; r < 32; r += 8) {
       float v = ta[r][tx] + tb[tx][r];  // (X + X^T)[I*32 + r, J*32 + tx]
       for (int o = 0; o < p.nout; ++o) acc[o][r][tx] += p.coef[o][s] * v;
+    }
+    if (s == 0 && p.tout) {  // transposed copy: tout(I,J) = X(J,I)^T, tout(J,I) = X(I,J)^T
+      float* y = p.tout + base;
+      for (int r = ty; r < 32; r += 8) {
+        int i = I * 32 + r, j = J * 32 + tx;
+        if (i < b && j < b) y[(int64_t)i * b + j] = tb[tx][r];
+        int i2 = J * 32 + r, j2 = I * 32 + tx;
+        if (I != J && i2 < b && j2 < b) y[(int64_t)i2 * b + j2] = ta[tx][r];
+      }
     }
   }
   __syncthreads();
@@ -689,8 +784,12 @@ cudaError_t launch_cnp_mm(const SgemmArgs& a, cudaStream_t s) {
   p.tiles_per_batch = a.mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
   const int64_t grid = (int64_t)p.tiles_per_batch * a.batch;
   if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+  const bool rows = a.a_sym != 0 && (!a.A2 || (a.a2_sym != 0 && (a.alpha2 == 1.f || a.alpha2 == -1.f)));
   begin_launch("cnp_sgemm", s);
-  k_cnp_mm<0><<<(unsigned)grid, kMMThreads, 0, s>>>(p, a.a_sym, a.a2_sym);
+  if (rows)
+    k_cnp_mm<true><<<(unsigned)grid, kMMThreads, 0, s>>>(p, a.a_sym, a.a2_sym);
+  else
+    k_cnp_mm<false><<<(unsigned)grid, kMMThreads, 0, s>>>(p, a.a_sym, a.a2_sym);
   end_launch("cnp_sgemm", s);
   return cudaGetLastError();
 }
@@ -706,6 +805,12 @@ cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s) {
                       (!a.A2 || (a.lda2 == bsq && a.ldb2 == bsq)) && !a.transA && !a.transB &&
                       !a.transA2 && !a.transB2 && a.nadd <= 8;
   if (square) return launch_cnp_mm(a, s);
+  if (a.a_sym == 2 || a.a2_sym == 2) {  // operand given as its transpose
+    SgemmArgs t = a;
+    if (t.a_sym == 2) { t.transA = !t.transA; t.a_sym = 0; }
+    if (t.a2_sym == 2) { t.transA2 = !t.transA2; t.a2_sym = 0; }
+    return launch_sgemm(t, s);
+  }
   SgemmDev p;
   p.A = a.A; p.lda = a.lda; p.sA = a.sA;
   p.B = a.B; p.ldb = a.ldb; p.sB = a.sB;
@@ -767,10 +872,11 @@ cudaError_t launch_theta_to_Q(const float* theta, float* Q, int nblk, int b, cud
 }
 
 cudaError_t launch_symcomb(const float* const* X, int nin, float* const* out, int nout,
-                           const float* coef, int nblk, int b, cudaStream_t s) {
+                           const float* coef, int nblk, int b, cudaStream_t s, float* tout) {
   if (nblk <= 0) return cudaSuccess;
   if (nin < 1 || nin > 4 || nout < 1 || nout > 4) return cudaErrorInvalidValue;
   SymcombDev p;
+  p.tout = tout;
   for (int i = 0; i < 4; ++i) {
     p.X[i] = i < nin ? X[i] : nullptr;
     p.out[i] = i < nout ? out[i] : nullptr;

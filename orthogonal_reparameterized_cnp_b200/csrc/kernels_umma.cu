@@ -35,18 +35,24 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one swizzle row
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 2 control warps + 8 epilogue warps
+constexpr int kEpiWarps = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
-template <int BN>
+// B_RES: the B operand of a whole item (K <= 256) stays in shared memory while the CTA
+// works through consecutive items that share it (the block-diagonal products: one G_j
+// for many token tiles); only A streams through the ring.
+template <int BN, bool B_RES>
 struct Cfg {
   static constexpr int A_BYTES = kBM * kBK * 2;
-  static constexpr int B_BYTES = BN * kBK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int B_BYTES = BN * kBK * 2;  // one K chunk of B
+  static constexpr int STAGES = B_RES ? (BN == 256 ? 4 : 6) : (BN == 256 ? 4 : 6);
+  static constexpr int KCH_RES = 4;             // resident K chunks (K <= 256)
+  static constexpr int RING_BYTES = B_RES ? STAGES * A_BYTES : STAGES * (A_BYTES + B_BYTES);
+  static constexpr int BRES_BYTES = B_RES ? KCH_RES * B_BYTES : 0;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BRES_BYTES + BAR_BYTES;
 };
 
 struct Params {
@@ -169,6 +175,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+        "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]),
+        "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]),
+        "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]), "=r"(v[49]),
+        "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+        "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]),
+        "=r"(v[62]), "=r"(v[63])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -213,30 +239,60 @@ __device__ __forceinline__ Item decode(const Params& p, int item) {
   return it;
 }
 
-template <int BN, bool A_MN, bool B_MN>
+// Items a CTA works on: round-robin (item = blockIdx.x + q * gridDim.x), or, in B_RES
+// mode, one contiguous range so that consecutive items share their B operand.
+struct Range {
+  int first, last, step;
+};
+__device__ __forceinline__ Range my_items(const Params& p, bool contiguous) {
+  Range r;
+  if (contiguous) {
+    r.first = (int)(((long long)blockIdx.x * p.num_items) / gridDim.x);
+    r.last = (int)(((long long)(blockIdx.x + 1) * p.num_items) / gridDim.x);
+    r.step = 1;
+  } else {
+    r.first = blockIdx.x;
+    r.last = p.num_items;
+    r.step = gridDim.x;
+  }
+  return r;
+}
+__device__ __forceinline__ int b_key(const Params& p, int item) {
+  const Item w = decode(p, item);
+  return (w.bz * p.ksplit + w.split) * p.tiles_n + w.tn;
+}
+
+template <int BN, bool A_MN, bool B_MN, bool B_RES>
 __global__ void __launch_bounds__(kThreads, 1)
     k_umma_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, B_RES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sA = base;                          // STAGES x A_BYTES
-  const uint32_t sB = base + C::STAGES * C::A_BYTES;  // STAGES x B_BYTES
-  const uint32_t sBar = base + C::STAGES * C::STAGE_BYTES;
-  // barrier block: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, tmem slot
+  const uint32_t sA = base;                                   // STAGES x A_BYTES
+  const uint32_t sB = base + C::STAGES * C::A_BYTES;          // ring B (or resident B)
+  const uint32_t sBar = base + C::RING_BYTES + C::BRES_BYTES;
+  // barrier block: full[S], empty[S], tfull[2], tempty[2], drain, bfull, bempty, tmem slot
   auto full_bar = [&](int s) { return sBar + 8u * s; };
   auto empty_bar = [&](int s) { return sBar + 8u * (C::STAGES + s); };
   auto tfull_bar = [&](int a) { return sBar + 8u * (2 * C::STAGES + a); };
   auto tempty_bar = [&](int a) { return sBar + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t drain_bar = sBar + 8u * (2 * C::STAGES + 4);
-  const uint32_t tmem_slot = sBar + 8u * (2 * C::STAGES + 5);
+  const uint32_t bfull_bar = sBar + 8u * (2 * C::STAGES + 5);
+  const uint32_t bempty_bar = sBar + 8u * (2 * C::STAGES + 6);
+  const uint32_t tmem_slot = sBar + 8u * (2 * C::STAGES + 7);
   unsigned char* generic_base = smem_raw + (base - raw);
   volatile uint32_t* tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t*>(generic_base + (tmem_slot - base));
+  // address of B chunk kc for ring stage s (or of resident chunk kc)
+  auto b_addr_of = [&](int s, int kc) -> uint32_t {
+    return B_RES ? sB + (uint32_t)kc * C::B_BYTES : sB + (uint32_t)s * C::B_BYTES;
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const Range rng = my_items(p, B_RES);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -245,9 +301,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);
+      mbar_init(tempty_bar(a), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(bfull_bar, 1);
+    mbar_init(bempty_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
@@ -266,23 +324,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     int last_round[8];
     for (int s = 0; s < 8; ++s) last_round[s] = -1;
+    int brun = -1, cur_key = -1;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.num_items; item += gridDim.x) {
+    for (int item = rng.first; ok && item < rng.last; item += rng.step) {
       const Item w = decode(p, item);
       const int m0 = w.tm * kBM, n0 = w.tn * BN;
       const int kc0 = w.split * p.kcps;
       const int kc1 = min(p.total_kc, kc0 + p.kcps);
+      if (B_RES) {
+        const int key = b_key(p, item);
+        if (key != cur_key) {
+          ++brun;
+          if (!mbar_wait(bempty_bar, (brun & 1) ^ 1, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bfull_bar, (uint32_t)(kc1 - kc0) * C::B_BYTES);
+          for (int kc = kc0; kc < kc1; ++kc) {
+            const int k = kc * kBK;
+            const uint32_t b_dst = b_addr_of(0, kc - kc0);
+            if (!B_MN) {
+              tma_load_2d(b_dst, &tmB, k + w.bz * p.b_boff_k, n0 + w.bz * p.b_boff_mn, bfull_bar);
+            } else {
+#pragma unroll
+              for (int i = 0; i < BN / 64; ++i)
+                tma_load_2d(b_dst + i * 8192, &tmB, n0 + 64 * i + w.bz * p.b_boff_mn,
+                            k + w.bz * p.b_boff_k, bfull_bar);
+            }
+          }
+          cur_key = key;
+        }
+      }
       for (int kc = kc0; kc < kc1; ++kc, ++it) {
         const int s = it % C::STAGES, r = it / C::STAGES;
         if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+        mbar_expect_tx(full_bar(s), B_RES ? C::A_BYTES : C::A_BYTES + C::B_BYTES);
         last_round[s] = r;
         const int k = kc * kBK;
         const uint32_t a_dst = sA + s * C::A_BYTES;
-        const uint32_t b_dst = sB + s * C::B_BYTES;
         if (!A_MN) {
           tma_load_2d(a_dst, &tmA, k + w.bz * p.a_boff_k, m0 + w.bz * p.a_boff_mn, full_bar(s));
         } else {
@@ -290,13 +372,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(a_dst + 8192, &tmA, m0 + 64 + w.bz * p.a_boff_mn, k + w.bz * p.a_boff_k,
                       full_bar(s));
         }
-        if (!B_MN) {
-          tma_load_2d(b_dst, &tmB, k + w.bz * p.b_boff_k, n0 + w.bz * p.b_boff_mn, full_bar(s));
-        } else {
+        if (!B_RES) {
+          const uint32_t b_dst = b_addr_of(s, 0);
+          if (!B_MN) {
+            tma_load_2d(b_dst, &tmB, k + w.bz * p.b_boff_k, n0 + w.bz * p.b_boff_mn, full_bar(s));
+          } else {
 #pragma unroll
-          for (int i = 0; i < BN / 64; ++i)
-            tma_load_2d(b_dst + i * 8192, &tmB, n0 + 64 * i + w.bz * p.b_boff_mn,
-                        k + w.bz * p.b_boff_k, full_bar(s));
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_2d(b_dst + i * 8192, &tmB, n0 + 64 * i + w.bz * p.b_boff_mn,
+                          k + w.bz * p.b_boff_k, full_bar(s));
+          }
         }
       }
     }
@@ -304,17 +389,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       // make sure no TMA write into this CTA's shared memory is still in flight
       for (int s = 0; s < C::STAGES; ++s)
         if (last_round[s] >= 0) mbar_drain_wait(full_bar(s), last_round[s] & 1);
+      if (B_RES && brun >= 0) mbar_drain_wait(bfull_bar, brun & 1);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = make_idesc<BN, A_MN, B_MN>();
     int it = 0, tcount = 0;
+    int brun = -1, cur_key = -1;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.num_items; item += gridDim.x, ++tcount) {
+    for (int item = rng.first; ok && item < rng.last; item += rng.step, ++tcount) {
       const Item w = decode(p, item);
       const int kc0 = w.split * p.kcps;
       const int kc1 = min(p.total_kc, kc0 + p.kcps);
       const int acc = tcount & 1, ra = tcount >> 1;
+      int key = -1;
+      if (B_RES) {
+        key = b_key(p, item);
+        if (key != cur_key) {
+          ++brun;
+          if (!mbar_wait(bfull_bar, brun & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          cur_key = key;
+        }
+      }
       if (!mbar_wait(tempty_bar(acc), (ra & 1) ^ 1, p.err)) {
         ok = false;
         break;
@@ -329,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t a_addr = sA + s * C::A_BYTES;
-        const uint32_t b_addr = sB + s * C::B_BYTES;
+        const uint32_t b_addr = b_addr_of(s, kc - kc0);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t adesc = A_MN ? make_desc(a_addr + kk * 2048, 8192, 1024)
@@ -338,19 +437,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       : make_desc(b_addr + kk * 32, 16, 1024);
           umma_bf16(d_tmem, adesc, bdesc, idesc, (kc > kc0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(empty_bar(s));  // frees the smem slot once these MMAs have read it
+        umma_commit(empty_bar(s));  // frees the A (and ring B) slot once read
       }
       if (!ok) break;
       umma_commit(tfull_bar(acc));  // accumulator ready for the epilogue
+      if (B_RES) {
+        const int nxt = item + rng.step;
+        if (nxt >= rng.last || b_key(p, nxt) != key) umma_commit(bempty_bar);  // B reusable
+      }
     }
     // all MMAs issued by this thread complete before TMEM is released
     umma_commit(drain_bar);
     mbar_drain_wait(drain_bar, 0);
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // warp w drains TMEM lane quadrant (w % 4) and column half (w - 2) / 4 of each tile,
+    // 64 columns per tcgen05.ld
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int HALF = BN / 2;
     int tcount = 0;
-    for (int item = blockIdx.x; item < p.num_items; item += gridDim.x, ++tcount) {
+    for (int item = rng.first; item < rng.last; item += rng.step, ++tcount) {
       const Item w = decode(p, item);
       const int acc = tcount & 1, ra = tcount >> 1;
       // one lane waits so that the warp stays converged for the .sync.aligned loads
@@ -364,30 +471,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long dbase = (long long)w.split * p.d_split + (long long)w.bz * p.d_boff +
                               (long long)row * p.ldd + (long long)w.bz * p.d_boff_col;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), v);
+      for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+        uint32_t v[64];
+        tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), v);
         tmem_wait_ld();
-        if (row < p.M && n0 + c < p.N) {
-          if (p.out_f32) {
-            float* dst = static_cast<float*>(p.D) + dbase + n0 + c;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<uint4*>(dst + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-          } else {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + dbase + n0 + c;
+        for (int h = 0; h < 64; h += 32) {
+          if (row < p.M && n0 + c + h < p.N) {
+            if (p.out_f32) {
+              float* dst = static_cast<float*>(p.D) + dbase + n0 + c + h;
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              uint4 o;
-              __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-              __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-              __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-              o.x = *reinterpret_cast<uint32_t*>(&h0);
-              o.y = *reinterpret_cast<uint32_t*>(&h1);
-              o.z = *reinterpret_cast<uint32_t*>(&h2);
-              o.w = *reinterpret_cast<uint32_t*>(&h3);
-              *reinterpret_cast<uint4*>(dst + j) = o;
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<uint4*>(dst + j) =
+                    make_uint4(v[h + j], v[h + j + 1], v[h + j + 2], v[h + j + 3]);
+            } else {
+              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + dbase + n0 + c + h;
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                uint4 o;
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[h + j]), __uint_as_float(v[h + j + 1]));
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 2]), __uint_as_float(v[h + j + 3]));
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 4]), __uint_as_float(v[h + j + 5]));
+                __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 6]), __uint_as_float(v[h + j + 7]));
+                o.x = *reinterpret_cast<uint32_t*>(&h0);
+                o.y = *reinterpret_cast<uint32_t*>(&h1);
+                o.z = *reinterpret_cast<uint32_t*>(&h2);
+                o.w = *reinterpret_cast<uint32_t*>(&h3);
+                *reinterpret_cast<uint4*>(dst + j) = o;
+              }
             }
           }
         }
@@ -432,26 +543,30 @@ bool make_map(CUtensorMap* map, const UmmaOperand& op, int box_rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, bool B_RES>
 cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                      const char* family, cudaStream_t s) {
-  auto kern = k_umma_gemm<BN, A_MN, B_MN>;
+  auto kern = k_umma_gemm<BN, A_MN, B_MN, B_RES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg<BN>::SMEM_BYTES);
+                                       Cfg<BN, B_RES>::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   begin_launch(family, s);
-  kern<<<grid, kThreads, Cfg<BN>::SMEM_BYTES, s>>>(ma, mb, p);
+  kern<<<grid, kThreads, Cfg<BN, B_RES>::SMEM_BYTES, s>>>(ma, mb, p);
   end_launch(family, s);
   return cudaGetLastError();
 }
 
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
-                      bool a_mn, bool b_mn, const char* family, cudaStream_t s) {
-  if (!a_mn && !b_mn) return launch_t<BN, false, false>(ma, mb, p, grid, family, s);
-  if (!a_mn && b_mn) return launch_t<BN, false, true>(ma, mb, p, grid, family, s);
-  if (a_mn && b_mn) return launch_t<BN, true, true>(ma, mb, p, grid, family, s);
-  return launch_t<BN, true, false>(ma, mb, p, grid, family, s);
+                      bool a_mn, bool b_mn, bool b_res, const char* family, cudaStream_t s) {
+  if (b_res) {  // A K-major only
+    if (!b_mn) return launch_t<BN, false, false, true>(ma, mb, p, grid, family, s);
+    return launch_t<BN, false, true, true>(ma, mb, p, grid, family, s);
+  }
+  if (!a_mn && !b_mn) return launch_t<BN, false, false, false>(ma, mb, p, grid, family, s);
+  if (!a_mn && b_mn) return launch_t<BN, false, true, false>(ma, mb, p, grid, family, s);
+  if (a_mn && b_mn) return launch_t<BN, true, true, false>(ma, mb, p, grid, family, s);
+  return launch_t<BN, true, false, false>(ma, mb, p, grid, family, s);
 }
 
 }  // namespace
@@ -463,7 +578,7 @@ int umma_choose_ksplit(int M, int N, int K, int batch) {
   if (total_kc <= 0) return 1;
   const int sms = num_sms();
   int want = 1;
-  if (tiles < sms) want = (2 * sms + tiles - 1) / tiles;
+  if (tiles < sms) want = sms / tiles;  // about one wave of items
   int max_split = total_kc / 4;  // at least 4 k-chunks (256 along K) per split
   if (max_split < 1) max_split = 1;
   if (want > max_split) want = max_split;
@@ -508,8 +623,12 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   p.err = device_error_flag();
   int grid = num_sms();
   if (grid > p.num_items) grid = p.num_items;
-  if (BN == 256) return launch_bn<256>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, family, s);
-  return launch_bn<128>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, family, s);
+  // keep B resident when one item's whole B (K <= 256) fits and the items share it
+  const bool b_res = !g.A.mn_major && p.kcps <= 4 && p.ksplit == 1 &&
+                     p.num_items >= 2 * grid && p.tiles_m >= 2;
+  if (BN == 256)
+    return launch_bn<256>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
+  return launch_bn<128>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
 }
 
 }  // namespace poetx

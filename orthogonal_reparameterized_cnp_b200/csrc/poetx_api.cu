@@ -130,8 +130,8 @@ CnpPoly cnp_poly(int k) {
 int cnp_mats(int k, bool backward) {
   const int d = (k + 1) / 2;
   // forward: Q, P_1..P_d, F'
-  // backward adds: D, N_1..N_d, Pm, R, R2, T, T2, A
-  return backward ? 2 * d + 9 : d + 2;
+  // backward adds: D, dG^T, N_1..N_d, Pm, R, R2, T, T2, A
+  return backward ? 2 * d + 10 : d + 2;
 }
 
 constexpr size_t kCnpChunkTarget = 256ull << 20;  // bytes per scratch matrix
@@ -356,6 +356,7 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     for (int j = 1; j <= d; ++j) Pw[j] = mat();
     float* Fp = mat();
     float* D = mat();
+    float* dGt = mat();
     for (int j = 1; j <= d; ++j) Nw[j] = mat();
     float* Pm = mat();
     float* R = mat();
@@ -384,7 +385,8 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
         coef[t * 2 + 0] = P.e[j0 + t];
         coef[t * 2 + 1] = -P.f[j0 + t];
       }
-      POETX_CUDA(launch_symcomb(X, 2, outs, cnt, coef, nb, b, s), "cnp N");
+      POETX_CUDA(launch_symcomb(X, 2, outs, cnt, coef, nb, b, s, j0 == 1 ? dGt : nullptr),
+                 "cnp N");
     }
     // Y = dS + dS^T = sum_j sum_a S^a N_j S^(j-1-a), by a Horner recursion from the top
     const float* Y = Nw[1];
@@ -431,7 +433,8 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
       Y = Tc;
     }
     // A = f_0 dG + dG F' - Y Q  (skew part of A gives dtheta)
-    SgemmArgs ga = sq_gemm(dg, 0, Fp, 0, A, nb, b, SG_FULL);
+    SgemmArgs ga = sq_gemm(dGt, 0, Fp, 0, A, nb, b, SG_FULL);
+    ga.a_sym = 2;  // dGt holds dG^T, so dG is read by rows
     ga.A2 = Y; ga.lda2 = b; ga.sA2 = bb;
     ga.B2 = Q; ga.ldb2 = b; ga.sB2 = bb;
     ga.K2 = b;

@@ -70,8 +70,8 @@ struct SgemmArgs {
   float skew_c = 0.f;
   float diag = 0.f;
   int mode = SG_FULL;
-  // structure of A and A2 when known: 0 general, +1 symmetric, -1 skew-symmetric (lets
-  // the square-block kernel read them already transposed)
+  // how A and A2 may be read by rows as their own transpose: 0 general, +1 symmetric,
+  // -1 skew-symmetric, 2 the pointer holds the operand's transpose
   int a_sym = 0, a2_sym = 0;
 };
 cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s);
@@ -80,9 +80,10 @@ cudaError_t launch_sgemm(const SgemmArgs& a, cudaStream_t s);
 // Q = skew(theta) for nblk blocks of size b.
 cudaError_t launch_theta_to_Q(const float* theta, float* Q, int nblk, int b, cudaStream_t s);
 // out_o = sum_s coef[o][s] * (X_s + X_s^T) for o < nout (symmetric outputs), s < nin.
+// When tout is given it also receives X[0]^T.
 cudaError_t launch_symcomb(const float* const* X, int nin, float* const* out, int nout,
                            const float* coef /* [nout][nin] row-major */, int nblk, int b,
-                           cudaStream_t s);
+                           cudaStream_t s, float* tout = nullptr);
 // dtheta_idx(i,j) = A_ij - A_ji for i < j.
 cudaError_t launch_pack_skew(const float* A, float* dtheta, int nblk, int b, cudaStream_t s);
 // dst[j] = (accumulate ? dst[j] : 0) + sum_s src[s * stride + j], s < nsplit (fixed order).
