@@ -1,0 +1,524 @@
+// The Cayley-Neumann parameterisation (POET-X technical summary, section 2.4) as one
+// persistent kernel per call: all of a call's steps -- expanding theta into Q, the
+// structured fp32 products, the symmetrising combinations, packing dtheta -- are jobs of
+// one launch.  Work items (one output tile of one job for one b x b block) are handed
+// out in job order through an atomic ticket; before computing, an item waits until the
+// jobs it reads have finished for its own block (per-(job, block) counters), so the
+// blocks flow through the chain independently and no launch boundary separates steps.
+//
+// Deadlock freedom: tickets are taken in increasing order by CTAs that are running, and
+// an item only waits on items with smaller tickets, so the lowest unfinished ticket can
+// always run (the grid is also sized to the CTAs that fit on the GPU at once).  Every wait is bounded anyway: after the
+// time limit the CTA records POETX_ERR_TIMEOUT in the device flag and stops.
+//
+// Data produced inside the launch is read through L2 only (cp.async.cg, ld.global.cg),
+// never through the non-coherent L1 / read-only paths.
+#include <cuda_bf16.h>
+
+#include "poetx_internal.h"
+
+namespace poetx {
+namespace {
+
+// kGroups groups of 128 threads per CTA; in a product tile every group accumulates the
+// whole 64 x 64 tile over its own share of K (own cp.async ring), then the partial tiles
+// are summed through shared memory in a fixed order.  kCtasPerSm CTAs share an SM so that
+// one tile's load latency overlaps another tile's arithmetic.
+constexpr int kGroups = 4;
+constexpr int kThreads = kGroups * 128;
+constexpr int kCtasPerSm = 4 / kGroups;
+constexpr int kGThreads = 128;
+constexpr int kBK = 16;
+constexpr int kLD = 64 + 4;
+constexpr int kStages = 4;
+constexpr int kStageFloats = 2 * kBK * kLD;
+constexpr int kRingFloats = kGroups * kStages * kStageFloats;  // 139 KB
+constexpr int kRedFloats = kGroups * 64 * 64;                   // 64 KB of partial tiles
+constexpr int kMirFloats = 2 * 64 * 65;                         // mirror staging
+constexpr int kPairFloats = 5 * 64 * 65;  // symmetrising job: 2 inputs + 3 outputs (d <= 3)
+constexpr int kSmemFloats0 =
+    kRingFloats > kRedFloats + kMirFloats ? kRingFloats : kRedFloats + kMirFloats;
+constexpr int kSmemFloats = kSmemFloats0 > kPairFloats ? kSmemFloats0 : kPairFloats;
+static_assert(kSmemFloats >= kPairFloats && kSmemFloats >= kRedFloats + kMirFloats &&
+                  kSmemFloats >= kRingFloats,
+              "shared memory must hold every job type's tiles");
+constexpr int kSmemBytes = kSmemFloats * 4;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ float4 ldcg4(const float* p) {
+  return __ldcg(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void tile_pair(int nt, int t, int& I, int& J) {
+  I = 0;
+  while (t >= nt - I) {
+    t -= nt - I;
+    ++I;
+  }
+  J = I + t;
+}
+
+__device__ __forceinline__ int64_t tri_idx(int i, int j, int b) {
+  return (int64_t)i * b - (int64_t)i * (i + 1) / 2 + (j - i - 1);
+}
+
+// ------------------------------------------------------------------ product tile
+// C-tile (64 x 64) of one block: acc = op(A1) B1 (+ alpha2 op(A2) B2), every A read by rows
+// (symmetric, skew, or given transposed), then the structured epilogue.
+__device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  const int tid = threadIdx.x;
+  const int grp = tid >> 7, gtid = tid & (kGThreads - 1);
+  const int tx = gtid & 15, ty = gtid >> 4;
+  const int nt = b / 64;
+  int I, Jt;
+  if (J.mode == SG_FULL) {
+    I = t / nt;
+    Jt = t - I * nt;
+  } else {
+    tile_pair(nt, t, I, Jt);
+  }
+  const int m0 = I * 64, n0 = Jt * 64;
+  const int64_t boff = (int64_t)z * b * b;
+  const float* A1 = J.A + boff;
+  const float* B1 = J.B + boff;
+  const float* A2 = J.A2 ? J.A2 + boff : nullptr;
+  const float* B2 = J.B2 ? J.B2 + boff : nullptr;
+  const int nk1 = b / kBK;
+  const int nk2 = A2 ? b / kBK : 0;
+  const int nkt = nk1 + nk2;
+  // this group's k tiles
+  const int kt_begin = (grp * nkt) / kGroups;
+  const int kt_end = ((grp + 1) * nkt) / kGroups;
+  const float s1 = J.a_sym < 0 ? -1.f : 1.f;
+  const float s2 = J.a2_sym < 0 ? -1.f : 1.f;
+  const float boundary = s1 * s2 * J.alpha2;
+  // the group's accumulators times g_scale are its share of op(A1)B1 + alpha2 op(A2)B2
+  const float g_scale = (nk2 > 0 && kt_end > nk1) ? s2 * J.alpha2 : s1;
+
+  float acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+
+  float* ring = smem + grp * kStages * kStageFloats;
+  auto As_ = [&](int st) { return reinterpret_cast<float (*)[kLD]>(ring + st * kStageFloats); };
+  auto Bs_ = [&](int st) {
+    return reinterpret_cast<float (*)[kLD]>(ring + st * kStageFloats + kBK * kLD);
+  };
+  auto issue = [&](int kt) {  // kt: absolute k tile index
+    if (kt < kt_end) {
+      const bool first = kt < nk1;
+      const float* A = first ? A1 : A2;
+      const float* B = first ? B1 : B2;
+      const int k0 = (first ? kt : kt - nk1) * kBK;
+      const int st = (kt - kt_begin) % kStages;
+      float (*As)[kLD] = As_(st);
+      float (*Bs)[kLD] = Bs_(st);
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        const int f = gtid + l * kGThreads;
+        const int r = f >> 4, c4 = (f & 15) * 4;
+        cp_async16(&As[r][c4], A + (int64_t)(k0 + r) * b + m0 + c4);
+        cp_async16(&Bs[r][c4], B + (int64_t)(k0 + r) * b + n0 + c4);
+      }
+    }
+    cp_commit();
+  };
+  // named barrier per group (ids 1..4; 0 is __syncthreads)
+  auto group_sync = [&]() {
+    asm volatile("bar.sync %0, %1;" ::"r"(grp + 1), "r"(kGThreads) : "memory");
+  };
+#pragma unroll
+  for (int st = 0; st < kStages - 1; ++st) issue(kt_begin + st);
+  for (int kt = kt_begin; kt < kt_end; ++kt) {
+    cp_wait<kStages - 2>();
+    group_sync();
+    issue(kt + kStages - 1);
+    if (nk2 > 0 && kt == nk1 && kt > kt_begin) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] *= boundary;
+    }
+    const int st = (kt - kt_begin) % kStages;
+    float (*As)[kLD] = As_(st);
+    float (*Bs)[kLD] = Bs_(st);
+#pragma unroll
+    for (int k = 0; k < kBK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[k][ty * 8 + 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[k][tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+    }
+  }
+  cp_wait<0>();
+  __syncthreads();  // every group is done with its ring: the space becomes red[]
+
+  // partial tiles -> red[grp][row][col]
+  float* red = smem;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    float* dst = red + (grp * 64 + ty * 8 + r) * 64 + tx * 4;
+    *reinterpret_cast<float4*>(dst) = make_float4(g_scale * acc[r][0], g_scale * acc[r][1],
+                                                  g_scale * acc[r][2], g_scale * acc[r][3]);
+  }
+  __syncthreads();
+  // epilogue: thread owns row il and 8 consecutive columns of the tile
+  // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
+  float* C = J.C + boff;
+  __nv_bfloat16* Cb = J.Cb ? J.Cb + boff : nullptr;
+  float* C2 = J.C2 ? J.C2 + boff : nullptr;
+  const bool structured = J.mode != SG_FULL;
+  float (*Ms)[65] = reinterpret_cast<float (*)[65]>(smem + kRedFloats);
+  float (*Ms2)[65] = reinterpret_cast<float (*)[65]>(smem + kRedFloats + 64 * 65);
+  for (int pass = 0; pass < 64 * 64 / (8 * kThreads); ++pass) {
+  const int il = pass * (kThreads / 8) + (tid >> 3), jl0 = (tid & 7) * 8;
+  const int i = m0 + il, j0 = n0 + jl0;
+  const int64_t row = (int64_t)i * b;
+  float a[8];
+  {
+    const float* r0 = red + il * 64 + jl0;
+    const float4 p0 = *reinterpret_cast<const float4*>(r0);
+    const float4 p1 = *reinterpret_cast<const float4*>(r0 + 4);
+    a[0] = p0.x; a[1] = p0.y; a[2] = p0.z; a[3] = p0.w;
+    a[4] = p1.x; a[5] = p1.y; a[6] = p1.z; a[7] = p1.w;
+#pragma unroll
+    for (int g2 = 1; g2 < kGroups; ++g2) {  // fixed summation order
+      const float* rg = r0 + g2 * 64 * 64;
+      const float4 q0 = *reinterpret_cast<const float4*>(rg);
+      const float4 q1 = *reinterpret_cast<const float4*>(rg + 4);
+      a[0] += q0.x; a[1] += q0.y; a[2] += q0.z; a[3] += q0.w;
+      a[4] += q1.x; a[5] += q1.y; a[6] += q1.z; a[7] += q1.w;
+    }
+  }
+  float sym[8], sym2[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const bool dg = (i == j0 + c);
+    sym[c] = dg ? J.diag : 0.f;
+    sym2[c] = dg ? J.diag2 : 0.f;
+  }
+  for (int q = 0; q < J.nadd; ++q) {
+    const float4 x0 = ldcg4(J.add[q] + boff + row + j0);
+    const float4 x1 = ldcg4(J.add[q] + boff + row + j0 + 4);
+    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      sym[c] += J.addc[q] * xs[c];
+      sym2[c] += J.addc2[q] * xs[c];
+    }
+  }
+  float skew[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) skew[c] = J.alpha * a[c];
+  if (J.skew_add) {
+    const float4 x0 = ldcg4(J.skew_add + boff + row + j0);
+    const float4 x1 = ldcg4(J.skew_add + boff + row + j0 + 4);
+    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) skew[c] += J.skew_c * xs[c];
+  }
+  float v[8], vm[8], v2[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const int j = j0 + c;
+    if (J.mode == SG_SYMSKEW) {
+      v[c] = (i == j) ? sym[c] : sym[c] + skew[c];
+      vm[c] = sym[c] - skew[c];
+    } else {
+      v[c] = skew[c] + sym[c];
+      vm[c] = v[c];
+    }
+    v2[c] = J.alpha_c2 * a[c] + sym2[c];
+  }
+  if (structured && I == Jt) {  // diagonal tile: this thread writes the upper triangle only
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int j = j0 + c;
+      if (i <= j) {
+        C[row + j] = v[c];
+        if (Cb) Cb[row + j] = __float2bfloat16_rn(v[c]);
+        if (C2) C2[row + j] = v2[c];
+      }
+    }
+  } else {
+    *reinterpret_cast<float4*>(C + row + j0) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(C + row + j0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    if (Cb) {
+      uint4 o;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
+      __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
+      o.x = *reinterpret_cast<uint32_t*>(&h0);
+      o.y = *reinterpret_cast<uint32_t*>(&h1);
+      o.z = *reinterpret_cast<uint32_t*>(&h2);
+      o.w = *reinterpret_cast<uint32_t*>(&h3);
+      *reinterpret_cast<uint4*>(Cb + row + j0) = o;
+    }
+    if (C2) {
+      *reinterpret_cast<float4*>(C2 + row + j0) = make_float4(v2[0], v2[1], v2[2], v2[3]);
+      *reinterpret_cast<float4*>(C2 + row + j0 + 4) = make_float4(v2[4], v2[5], v2[6], v2[7]);
+    }
+  }
+  if (structured) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      Ms[il][jl0 + c] = vm[c];
+      if (C2) Ms2[il][jl0 + c] = v2[c];
+    }
+  }
+  }  // passes
+  if (structured) {
+    __syncthreads();  // staged mirror values of every pass are visible
+    for (int e = tid; e < 64 * 64; e += kThreads) {
+      const int jl = e >> 6, il2 = e & 63;
+      if (I == Jt && il2 >= jl) continue;
+      const int64_t ji = (int64_t)(n0 + jl) * b + m0 + il2;
+      const float vmv = Ms[il2][jl];
+      C[ji] = vmv;
+      if (Cb) Cb[ji] = __float2bfloat16_rn(vmv);
+      if (C2) C2[ji] = Ms2[il2][jl];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ 64 x 64 tile-pair jobs
+// Tile pair (I, J), I <= J, of a block; thread (tx = tid & 63, ty = tid >> 6) walks rows
+// ty, ty + 8, ... of the 64 x 64 tile, so each row is one coalesced 256-byte access.
+constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;
+
+// theta -> Q: Q_ij = theta, Q_ji = -theta
+__device__ void expand_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  float (*tt)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
+  int I, Jt;
+  tile_pair(b / kPT, t, I, Jt);
+  const int64_t ntri = (int64_t)b * (b - 1) / 2;
+  const float* th = J.A + z * ntri;
+  float* q = J.C + (int64_t)z * b * b;
+  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
+  for (int r = ty; r < kPT; r += kPRows) {
+    const int i = I * kPT + r, j = Jt * kPT + tx;
+    tt[r][tx] = (i < j) ? __ldcg(th + tri_idx(i, j, b)) : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < kPT; r += kPRows) {
+    const int i = I * kPT + r, j = Jt * kPT + tx;
+    q[(int64_t)i * b + j] = (I == Jt && r > tx) ? -tt[tx][r] : tt[r][tx];
+  }
+  if (I != Jt) {
+    for (int r = ty; r < kPT; r += kPRows) {
+      const int i = Jt * kPT + r, j = I * kPT + tx;
+      q[(int64_t)i * b + j] = -tt[tx][r];
+    }
+  }
+}
+
+// out_o = sum_s coef[o][s] (X_s + X_s^T) (symmetric outputs), optional Cb_f = X_0^T
+__device__ void symcomb_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  float (*ta)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
+  float (*tb)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kPT * kPLD);
+  float (*acc)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem + 2 * kPT * kPLD);
+  int I, Jt;
+  tile_pair(b / kPT, t, I, Jt);
+  const int64_t base = (int64_t)z * b * b;
+  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
+  const float* X[2] = {J.A, J.B};
+  float* out[4] = {J.C, J.C2, J.add_out[0], J.add_out[1]};
+  for (int o = 0; o < J.nout; ++o)
+    for (int r = ty; r < kPT; r += kPRows) acc[o][r][tx] = 0.f;
+  for (int s = 0; s < J.nin; ++s) {
+    const float* x = X[s] + base;
+    __syncthreads();
+    for (int r = ty; r < kPT; r += kPRows) {
+      ta[r][tx] = __ldcg(x + (int64_t)(I * kPT + r) * b + Jt * kPT + tx);
+      tb[r][tx] = __ldcg(x + (int64_t)(Jt * kPT + r) * b + I * kPT + tx);
+    }
+    __syncthreads();
+    for (int r = ty; r < kPT; r += kPRows) {
+      const float v = ta[r][tx] + tb[tx][r];  // (X + X^T)[I*64 + r, J*64 + tx]
+      for (int o = 0; o < J.nout; ++o) acc[o][r][tx] += J.coef[o][s] * v;
+    }
+    if (s == 0 && J.Cb_f) {  // transposed copy: (I,J) <- X(J,I)^T, (J,I) <- X(I,J)^T
+      float* y = J.Cb_f + base;
+      for (int r = ty; r < kPT; r += kPRows) {
+        y[(int64_t)(I * kPT + r) * b + Jt * kPT + tx] = tb[tx][r];
+        if (I != Jt) y[(int64_t)(Jt * kPT + r) * b + I * kPT + tx] = ta[tx][r];
+      }
+    }
+  }
+  __syncthreads();
+  for (int o = 0; o < J.nout; ++o) {
+    float* y = out[o] + base;
+    for (int r = ty; r < kPT; r += kPRows)
+      y[(int64_t)(I * kPT + r) * b + Jt * kPT + tx] =
+          (I == Jt && r > tx) ? acc[o][tx][r] : acc[o][r][tx];
+    if (I != Jt)
+      for (int r = ty; r < kPT; r += kPRows)
+        y[(int64_t)(Jt * kPT + r) * b + I * kPT + tx] = acc[o][tx][r];
+  }
+}
+
+// dtheta_idx(i, j) = A_ij - A_ji
+__device__ void pack_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  float (*ta)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
+  float (*tb)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kPT * kPLD);
+  int I, Jt;
+  tile_pair(b / kPT, t, I, Jt);
+  const float* a = J.A + (int64_t)z * b * b;
+  float* th = J.C + z * ((int64_t)b * (b - 1) / 2);
+  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
+  for (int r = ty; r < kPT; r += kPRows) {
+    ta[r][tx] = __ldcg(a + (int64_t)(I * kPT + r) * b + Jt * kPT + tx);
+    tb[r][tx] = __ldcg(a + (int64_t)(Jt * kPT + r) * b + I * kPT + tx);
+  }
+  __syncthreads();
+  for (int r = ty; r < kPT; r += kPRows) {
+    const int i = I * kPT + r, j = Jt * kPT + tx;
+    if (i < j) th[tri_idx(i, j, b)] = ta[r][tx] - tb[tx][r];
+  }
+}
+
+// ------------------------------------------------------------------ the graph kernel
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid_constant__ CnpGraph g) {
+  extern __shared__ __align__(16) float smem[];
+  __shared__ int s_item, s_next;
+  __shared__ int s_ok;
+  int* ticket = g.counters + g.njobs * g.nblk;
+  const int total = g.item_start[g.njobs];
+  if (threadIdx.x == 0) s_next = atomicAdd(ticket, 1);
+  for (;;) {
+    __syncthreads();  // smem of the previous item is free; s_next is visible
+    if (threadIdx.x == 0) {
+      s_item = s_next;
+      s_ok = 1;
+    }
+    __syncthreads();
+    const int item = s_item;
+    if (item >= total) break;
+    int j = 0;
+    while (item >= g.item_start[j + 1]) ++j;
+    const CnpJob& J = g.job[j];
+    const int local = item - g.item_start[j];
+    const int z = local / J.tiles;
+    const int t = local - z * J.tiles;
+    if (threadIdx.x == 0) {
+      // next ticket in flight while this item runs
+      s_next = atomicAdd(ticket, 1);
+      // wait until every job this one reads has finished for block z
+      const unsigned long long t0 = gtimer();
+      for (int d = 0; d < j && s_ok; ++d) {
+        if (!((J.deps >> d) & 1u)) continue;
+        const int* cnt = g.counters + d * g.nblk + z;
+        const int need = g.job[d].tiles;
+        unsigned spins = 0;
+        while (ld_acquire(cnt) < need) {
+          if ((++spins & 31u) == 0) {
+            if (*reinterpret_cast<volatile int*>(g.err) != 0 ||
+                gtimer() - t0 > kWaitLimitNs) {
+              atomicCAS(g.err, 0, (int)POETX_ERR_TIMEOUT);
+              s_ok = 0;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (!s_ok) break;
+    switch (J.type) {
+      case JOB_EXPAND: expand_tile(J, z, t, g.b, smem); break;
+      case JOB_PRODUCT: product_tile(J, z, t, g.b, smem); break;
+      case JOB_SYMCOMB: symcomb_tile(J, z, t, g.b, smem); break;
+      default: pack_tile(J, z, t, g.b, smem); break;
+    }
+    // publish: the barrier orders every thread's stores before thread 0's release
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_add(g.counters + j * g.nblk + z, 1);
+  }
+}
+
+__global__ void k_zero_ints(int* p, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
+}
+
+}  // namespace
+
+int cnp_graph_tiles(int type, int mode, int b) {
+  if (type == JOB_PRODUCT) {
+    const int nt = b / 64;
+    return mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
+  }
+  const int nt = b / 64;  // 64 x 64 tile pairs
+  return nt * (nt + 1) / 2;
+}
+
+cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
+  if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;
+  g.item_start[0] = 0;
+  for (int j = 0; j < g.njobs; ++j) {
+    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.b);
+    g.item_start[j + 1] = g.item_start[j] + g.job[j].tiles * g.nblk;
+  }
+  g.err = device_error_flag();
+  const int ncount = g.njobs * g.nblk + 1;
+  begin_launch("cnp_elementwise", s);
+  k_zero_ints<<<(ncount + 255) / 256, 256, 0, s>>>(g.counters, ncount);
+  end_launch("cnp_elementwise", s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // persistent grid: never more CTAs than can be resident at once
+  static int per_sm_dev[64] = {0};  // once per device, outside any stream capture
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  int& per_sm = per_sm_dev[dev];
+  if (per_sm == 0) {
+    int v = 0;
+    e = cudaFuncSetAttribute(k_cnp_graph, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k_cnp_graph, kThreads, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    per_sm = v > 0 ? v : 1;
+  }
+  int grid = num_sms() * per_sm;
+  const int total = g.item_start[g.njobs];
+  if (grid > total) grid = total;
+  begin_launch("cnp_sgemm", s);
+  k_cnp_graph<<<grid, kThreads, kSmemBytes, s>>>(g);
+  end_launch("cnp_sgemm", s);
+  return cudaGetLastError();
+}
+
+}  // namespace poetx

@@ -195,9 +195,16 @@ cudaError_t pipe_launch(const void* in, void* out, const int32_t* row_idx, const
   int R = (int)((32 * 1024) / row_bytes);
   R = R < 1 ? 1 : (R > 16 ? 16 : R);
   const size_t smem = 2 * (size_t)R * row_bytes;
-  cudaError_t e = cudaFuncSetAttribute(k_gather_rows_pipe<E, MAXV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-  if (e != cudaSuccess) return e;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_gather_rows_pipe<E, MAXV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
   const int nbatch = (rows + R - 1) / R;
   int per_sm = (int)((200 * 1024) / (smem + 1024));
   per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
@@ -231,7 +238,7 @@ cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
     return pipe_launch<E, 8>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
   }
   if (row_bytes <= (size_t)kMaxSmemRowBytes) {
-    static bool attr_set = false;
+    static bool attr_set = false;  // single-device use; the pipelined path covers the rest
     if (!attr_set) {
       cudaError_t e = cudaFuncSetAttribute(k_gather_rows_smem<E>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,

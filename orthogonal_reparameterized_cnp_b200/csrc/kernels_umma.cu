@@ -547,9 +547,16 @@ template <int BN, bool A_MN, bool B_MN, bool B_RES>
 cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
                      const char* family, cudaStream_t s) {
   auto kern = k_umma_gemm<BN, A_MN, B_MN, B_RES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg<BN, B_RES>::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  static bool attr_done[64] = {false};  // once per device, outside any stream capture
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<BN, B_RES>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
   begin_launch(family, s);
   kern<<<grid, kThreads, Cfg<BN, B_RES>::SMEM_BYTES, s>>>(ma, mb, p);
   end_launch(family, s);

@@ -136,9 +136,16 @@ int cnp_mats(int k, bool backward) {
 
 constexpr size_t kCnpChunkTarget = 256ull << 20;  // bytes per scratch matrix
 
+// per block: the matrices plus the task graph's done-counters (<= 16 jobs)
+constexpr size_t kCnpCounterBytesPerBlock = 64;
+constexpr size_t kCnpFixedBytes = 256;
+
 size_t cnp_per_block(int b, int k, bool backward) {
-  return (size_t)cnp_mats(k, backward) * align_up((size_t)b * b * 4);
+  return (size_t)cnp_mats(k, backward) * align_up((size_t)b * b * 4) + kCnpCounterBytesPerBlock;
 }
+
+// The one-launch task graph covers square blocks with b % 64 == 0 and k <= 6.
+bool cnp_graph_ok(int b, int k) { return b >= 64 && b % 64 == 0 && (k + 1) / 2 <= 3; }
 
 int cnp_validate(const void* theta, const void* out, int nblk, int b, int k) {
   if (nblk < 0) return fail(POETX_ERR_INVALID_ARG, "nblk must be >= 0");
@@ -152,7 +159,7 @@ int cnp_validate(const void* theta, const void* out, int nblk, int b, int k) {
 template <typename Fn>
 int cnp_chunks(int nblk, int b, int k, bool backward, void* ws, size_t ws_bytes, Fn fn) {
   const size_t per = cnp_per_block(b, k, backward);
-  size_t cap = ws_bytes / per;
+  size_t cap = ws_bytes > kCnpFixedBytes ? (ws_bytes - kCnpFixedBytes) / per : 0;
   if (cap < 1) return fail(POETX_ERR_WORKSPACE, "CNP scratch smaller than one block needs");
   if (!ws) return fail(POETX_ERR_INVALID_ARG, "null scratch");
   if (!aligned16(ws)) return fail(POETX_ERR_ALIGN, "scratch must be 16-byte aligned");
@@ -263,7 +270,7 @@ size_t poetx_cnp_workspace(int32_t nblk, int32_t b, int32_t k) {
   const size_t per_mat_cap = kCnpChunkTarget / ((size_t)b * b * 4);
   size_t chunk = (size_t)nblk;
   if (per_mat_cap >= 1 && chunk > per_mat_cap) chunk = per_mat_cap;
-  return chunk * cnp_per_block(b, k, true);
+  return chunk * cnp_per_block(b, k, true) + kCnpFixedBytes;
 }
 
 }  // extern "C"
@@ -294,6 +301,188 @@ int cnp_powers(const float* Q, std::vector<float*>& Pw, float* Fp, const CnpPoly
   return POETX_OK;
 }
 
+// ---- the task-graph form of the CNP (one persistent launch per chunk) -------------
+CnpJob prod_job(const float* A, int a_sym, const float* B, float* C, int mode, unsigned deps) {
+  CnpJob j;
+  j.type = JOB_PRODUCT;
+  j.mode = mode;
+  j.A = A;
+  j.a_sym = a_sym;
+  j.B = B;
+  j.C = C;
+  j.deps = deps;
+  return j;
+}
+
+// powers P_1 = Q Q, P_p = S P_{p-1}; the last also emits F' = sum_{j>=1} f_j P_j (C2).
+// Returns the job index of P_j in idx[j].
+void graph_powers(CnpGraph& g, int jQ, const float* Q, float* const* Pw, float* Fp,
+                  const CnpPoly& P, int* idx) {
+  const int d = P.d;
+  for (int j = 1; j <= d; ++j) {
+    CnpJob jb = (j == 1) ? prod_job(Q, -1, Q, Pw[1], SG_SYM, 1u << jQ)
+                         : prod_job(Pw[1], 1, Pw[j - 1], Pw[j], SG_SYM,
+                                    (1u << idx[1]) | (1u << idx[j - 1]));
+    if (j == d) {
+      jb.C2 = Fp;
+      jb.alpha_c2 = P.f[d];
+      for (int t = 1; t < d; ++t) {
+        jb.add[jb.nadd] = Pw[t];
+        jb.addc[jb.nadd] = 0.f;
+        jb.addc2[jb.nadd] = P.f[t];
+        ++jb.nadd;
+        jb.deps |= 1u << idx[t];
+      }
+    }
+    idx[j] = g.njobs;
+    g.job[g.njobs++] = jb;
+  }
+}
+
+int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* Fp, float* G,
+                  __nv_bfloat16* Gb, int* counters, const CnpPoly& P, int nb, int b,
+                  cudaStream_t s) {
+  const int d = P.d;
+  CnpGraph g;
+  g.nblk = nb;
+  g.b = b;
+  g.counters = counters;
+  CnpJob ex;
+  ex.type = JOB_EXPAND;
+  ex.A = theta;
+  ex.C = const_cast<float*>(Q);
+  g.job[g.njobs++] = ex;
+  int idx[4] = {0, 0, 0, 0};
+  graph_powers(g, 0, Q, Pw, Fp, P, idx);
+  // G = E + f_0 Q + Q F' (upper tiles; E symmetric, QF skew)
+  CnpJob jg = prod_job(Q, -1, Fp, G, SG_SYMSKEW, 1u);
+  jg.Cb = Gb;
+  jg.diag = P.e[0];
+  for (int j = 1; j <= d; ++j) {
+    jg.add[jg.nadd] = Pw[j];
+    jg.addc[jg.nadd] = P.e[j];
+    ++jg.nadd;
+    jg.deps |= 1u << idx[j];
+  }
+  jg.skew_add = Q;
+  jg.skew_c = P.f[0];
+  g.job[g.njobs++] = jg;
+  POETX_CUDA(launch_cnp_graph(g, s), "cnp graph (forward)");
+  return POETX_OK;
+}
+
+struct BwdMats {
+  float *Q, *P[4], *Fp, *D, *dGt, *N[4], *Pm, *R, *R2, *T, *T2, *A;
+};
+
+int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdMats& M,
+                  int* counters, const CnpPoly& P, int nb, int b, cudaStream_t s) {
+  const int d = P.d;
+  CnpGraph g;
+  g.nblk = nb;
+  g.b = b;
+  g.counters = counters;
+  CnpJob ex;
+  ex.type = JOB_EXPAND;
+  ex.A = theta;
+  ex.C = M.Q;
+  g.job[g.njobs++] = ex;
+  int idx[4] = {0, 0, 0, 0};
+  graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx);
+  // D = Q dG (the adjoint reaching F is Q^T dG = -D)
+  const int jD = g.njobs;
+  g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
+  // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, and dG^T
+  const int jN = g.njobs;
+  {
+    CnpJob jn;
+    jn.type = JOB_SYMCOMB;
+    jn.A = dg;
+    jn.B = M.D;
+    jn.nin = 2;
+    jn.nout = d;
+    float* outs[4] = {M.N[1], d >= 2 ? M.N[2] : nullptr, d >= 3 ? M.N[3] : nullptr, nullptr};
+    jn.C = outs[0];
+    jn.C2 = outs[1];
+    jn.add_out[0] = outs[2];
+    for (int o = 0; o < d; ++o) {
+      jn.coef[o][0] = P.e[o + 1];
+      jn.coef[o][1] = -P.f[o + 1];
+    }
+    jn.Cb_f = M.dGt;
+    jn.deps = 1u << jD;
+    g.job[g.njobs++] = jn;
+  }
+  // Y = sum_j sum_a S^a N_j S^(j-1-a)
+  const float* Y = M.N[1];
+  int jY = jN;
+  const int jS = idx[1];
+  const float* S = M.P[1];
+  if (d >= 2) {
+    const int jPm = g.njobs;
+    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
+    // T_{d-2} = N_{d-1} + Pm + Pm^T
+    const int jT = g.njobs;
+    CnpJob jt;
+    jt.type = JOB_SYMCOMB;
+    jt.A = M.N[d - 1];
+    jt.B = M.Pm;
+    jt.nin = 2;
+    jt.nout = 1;
+    jt.coef[0][0] = 0.5f;
+    jt.coef[0][1] = 1.f;
+    jt.C = M.T;
+    jt.deps = (1u << jN) | (1u << jPm);
+    g.job[g.njobs++] = jt;
+    Y = M.T;
+    jY = jT;
+    if (d == 3) {
+      // transposed Horner terms keep every A operand symmetric:
+      //   Rt_1 = N_2 + S N_3,  Rt_0 = N_1 + S Rt_1,  T_0 = Rt_0 + T_1 S
+      const int jR1 = g.njobs;
+      CnpJob r1 = prod_job(S, 1, M.N[3], M.R, SG_FULL, (1u << jS) | (1u << jN));
+      r1.add[0] = M.N[2];
+      r1.addc[0] = 1.f;
+      r1.nadd = 1;
+      g.job[g.njobs++] = r1;
+      const int jR0 = g.njobs;
+      CnpJob r0 = prod_job(S, 1, M.R, M.R2, SG_FULL, (1u << jS) | (1u << jN) | (1u << jR1));
+      r0.add[0] = M.N[1];
+      r0.addc[0] = 1.f;
+      r0.nadd = 1;
+      g.job[g.njobs++] = r0;
+      const int jT0 = g.njobs;
+      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jT) | (1u << jS) | (1u << jR0));
+      t0.add[0] = M.R2;
+      t0.addc[0] = 1.f;
+      t0.nadd = 1;
+      g.job[g.njobs++] = t0;
+      Y = M.T2;
+      jY = jT0;
+    }
+  }
+  // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji
+  const int jA = g.njobs;
+  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL,
+                       1u | (1u << jN) | (1u << idx[d]) | (1u << jY));
+  ja.A2 = Y;
+  ja.a2_sym = 1;
+  ja.B2 = M.Q;
+  ja.alpha2 = -1.f;
+  ja.add[0] = dg;
+  ja.addc[0] = P.f[0];
+  ja.nadd = 1;
+  g.job[g.njobs++] = ja;
+  CnpJob pk;
+  pk.type = JOB_PACK;
+  pk.A = M.A;
+  pk.C = dtheta;
+  pk.deps = 1u << jA;
+  g.job[g.njobs++] = pk;
+  POETX_CUDA(launch_cnp_graph(g, s), "cnp graph (backward)");
+  return POETX_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -315,6 +504,13 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
     std::vector<float*> Pw(d + 1, nullptr);
     for (int j = 1; j <= d; ++j) Pw[j] = static_cast<float*>(cv.take(bb * 4 * nb));
     float* Fp = static_cast<float*>(cv.take(bb * 4 * nb));
+    if (cnp_graph_ok(b, k)) {
+      int* counters = static_cast<int*>(cv.take(kCnpCounterBytesPerBlock * nb + 4));
+      __nv_bfloat16* Gb =
+          G_bf16 ? static_cast<__nv_bfloat16*>(G_bf16) + b0 * bb : nullptr;
+      return run_fwd_graph(theta + b0 * ntri, Q, Pw.data(), Fp, G + b0 * bb, Gb, counters, P,
+                           nb, b, s);
+    }
     POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
     int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
     if (st2 != POETX_OK) return st2;
@@ -365,6 +561,18 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     float* T2 = mat();
     float* A = mat();
     const float* dg = dG + b0 * bb;
+    if (cnp_graph_ok(b, k)) {
+      int* counters = static_cast<int*>(cv.take(kCnpCounterBytesPerBlock * nb + 4));
+      BwdMats M;
+      M.Q = Q;
+      for (int j = 0; j < 4; ++j) {
+        M.P[j] = j <= d ? Pw[j] : nullptr;
+        M.N[j] = j <= d ? Nw[j] : nullptr;
+      }
+      M.Fp = Fp; M.D = D; M.dGt = dGt; M.Pm = Pm; M.R = R; M.R2 = R2; M.T = T; M.T2 = T2;
+      M.A = A;
+      return run_bwd_graph(theta + b0 * ntri, dg, dtheta + b0 * ntri, M, counters, P, nb, b, s);
+    }
     POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
     int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
     if (st2 != POETX_OK) return st2;

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libpoetx translation units (host side).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -91,6 +92,54 @@ cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, fl
                                 int64_t count, int accumulate, cudaStream_t s);
 // fp32 -> bf16 (round to nearest even)
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s);
+
+// ---- CNP as one persistent task-graph launch (kernels_cnp_graph.cu) -----------------
+// Each job is one step applied to every block of a chunk; an item is one output tile of
+// one job for one block.  Square blocks with b % 64 == 0; products read every A operand
+// by rows (a_sym: -1 skew, +1 symmetric, 2 given as its transpose).
+enum CnpJobType { JOB_EXPAND = 0, JOB_PRODUCT = 1, JOB_SYMCOMB = 2, JOB_PACK = 3 };
+constexpr int kCnpMaxJobs = 14;
+
+struct CnpJob {
+  int type = JOB_PRODUCT;
+  int mode = SG_FULL;       // products: SG_FULL / SG_SYM / SG_SYMSKEW
+  int tiles = 0;            // items per block (filled in by the launcher)
+  unsigned deps = 0;        // bit d: reads job d's output for the same block
+  // products: C = epilogue(op(A) op(B) [+ alpha2 op(A2) op(B2)]), as SgemmArgs
+  // expand: A = theta, C = Q;  pack: A = matrix, C = dtheta
+  // symcomb: X = {A, B} (nin), outputs {C, C2, add_out[0], add_out[1]} (nout),
+  //          Cb_f = transposed copy of A (optional)
+  const float* A = nullptr;
+  const float* B = nullptr;
+  const float* A2 = nullptr;
+  const float* B2 = nullptr;
+  int a_sym = 0, a2_sym = 0;
+  float alpha = 1.f, alpha2 = 1.f;
+  float* C = nullptr;
+  __nv_bfloat16* Cb = nullptr;
+  float* C2 = nullptr;
+  float alpha_c2 = 0.f, diag = 0.f, diag2 = 0.f;
+  int nadd = 0;
+  const float* add[4] = {nullptr, nullptr, nullptr, nullptr};
+  float addc[4] = {0, 0, 0, 0};
+  float addc2[4] = {0, 0, 0, 0};
+  const float* skew_add = nullptr;
+  float skew_c = 0.f;
+  int nin = 0, nout = 0;
+  float coef[4][2] = {{0, 0}, {0, 0}, {0, 0}, {0, 0}};
+  float* add_out[2] = {nullptr, nullptr};
+  float* Cb_f = nullptr;
+};
+
+struct CnpGraph {
+  CnpJob job[kCnpMaxJobs];
+  int njobs = 0, nblk = 0, b = 0;
+  int item_start[kCnpMaxJobs + 1] = {0};
+  int* counters = nullptr;  // scratch: njobs * nblk done-counters + 1 ticket
+  int* err = nullptr;
+};
+// Zeroes the counters and runs the graph (two launches).
+cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s);
 
 // ---- tcgen05 GEMM (kernels_umma.cu) ----------------------------------------------
 // D[M x N] = A[M x K] . B[N x K]^T per batch entry, bf16 operands, fp32 accumulation.
