@@ -51,8 +51,9 @@ struct Cfg {
   static constexpr int RING_BYTES = B_RES ? STAGES * A_BYTES : STAGES * (A_BYTES + B_BYTES);
   static constexpr int BRES_BYTES = B_RES ? KCH_RES * B_BYTES : 0;
   static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int EPI_BYTES = 8 * 4096;  // one 4 KB TMA-store staging tile per epilogue warp
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BRES_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BRES_BYTES + EPI_BYTES + BAR_BYTES;
 };
 
 struct Params {
@@ -63,6 +64,7 @@ struct Params {
   int out_f32;
   long long ldd, d_boff_col, d_boff, d_split;
   int* err;
+  int y_per_bz, y_per_split;  // output tensor rows per batch entry / per split
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -126,6 +128,31 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -265,14 +292,15 @@ __device__ __forceinline__ int b_key(const Params& p, int item) {
 template <int BN, bool A_MN, bool B_MN, bool B_RES>
 __global__ void __launch_bounds__(kThreads, 1)
     k_umma_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tmD, const Params p) {
   using C = Cfg<BN, B_RES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t sA = base;                                   // STAGES x A_BYTES
   const uint32_t sB = base + C::STAGES * C::A_BYTES;          // ring B (or resident B)
-  const uint32_t sBar = base + C::RING_BYTES + C::BRES_BYTES;
+  const uint32_t sEpi = base + C::RING_BYTES + C::BRES_BYTES;  // 1024-aligned staging tiles
+  const uint32_t sBar = sEpi + C::EPI_BYTES;
   // barrier block: full[S], empty[S], tfull[2], tempty[2], drain, bfull, bempty, tmem slot
   auto full_bar = [&](int s) { return sBar + 8u * s; };
   auto empty_bar = [&](int s) { return sBar + 8u * (C::STAGES + s); };
@@ -309,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -452,10 +481,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // warp w drains TMEM lane quadrant (w % 4) and column half (w - 2) / 4 of each tile,
-    // 64 columns per tcgen05.ld
+    // 64 columns per tcgen05.ld.  Each 32-row piece is converted into this warp's 4 KB
+    // staging tile in the 128-byte-swizzled layout (16-byte chunk k of row r sits at chunk
+    // k ^ (r % 8)) and written by one TMA tensor store; TMA clips rows beyond the matrix.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     constexpr int HALF = BN / 2;
+    const uint32_t stage = sEpi + (uint32_t)(warp - 2) * 4096u;
+    const uint32_t my_row = stage + (uint32_t)lane * 128u;
+    const uint32_t sw = (uint32_t)(lane & 7);
     int tcount = 0;
     for (int item = rng.first; item < rng.last; item += rng.step, ++tcount) {
       const Item w = decode(p, item);
@@ -466,40 +500,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (!ready) break;
       tc_fence_after();
-      const int row = w.tm * kBM + q * 32 + lane;
+      const int row0 = w.tm * kBM + q * 32;
       const int n0 = w.tn * BN;
-      const long long dbase = (long long)w.split * p.d_split + (long long)w.bz * p.d_boff +
-                              (long long)row * p.ldd + (long long)w.bz * p.d_boff_col;
+      const int ybase = w.split * p.y_per_split + w.bz * p.y_per_bz + row0;
+      const int xbase = w.bz * (int)p.d_boff_col + n0;
 #pragma unroll 1
       for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
         uint32_t v[64];
         tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), v);
         tmem_wait_ld();
+        if (n0 + c >= p.N) continue;  // (uniform across the warp)
+        if (p.out_f32) {
 #pragma unroll
-        for (int h = 0; h < 64; h += 32) {
-          if (row < p.M && n0 + c + h < p.N) {
-            if (p.out_f32) {
-              float* dst = static_cast<float*>(p.D) + dbase + n0 + c + h;
+          for (int h = 0; h < 64; h += 32) {  // two 32-column fp32 pieces
+            if (lane == 0) bulk_wait_read0();  // the previous store has read the staging tile
+            __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<uint4*>(dst + j) =
-                    make_uint4(v[h + j], v[h + j + 1], v[h + j + 2], v[h + j + 3]);
-            } else {
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + dbase + n0 + c + h;
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                uint4 o;
-                __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v[h + j]), __uint_as_float(v[h + j + 1]));
-                __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 2]), __uint_as_float(v[h + j + 3]));
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 4]), __uint_as_float(v[h + j + 5]));
-                __nv_bfloat162 h3 = __floats2bfloat162_rn(__uint_as_float(v[h + j + 6]), __uint_as_float(v[h + j + 7]));
-                o.x = *reinterpret_cast<uint32_t*>(&h0);
-                o.y = *reinterpret_cast<uint32_t*>(&h1);
-                o.z = *reinterpret_cast<uint32_t*>(&h2);
-                o.w = *reinterpret_cast<uint32_t*>(&h3);
-                *reinterpret_cast<uint4*>(dst + j) = o;
-              }
+            for (int k = 0; k < 8; ++k)
+              sts128(my_row + (((uint32_t)k ^ sw) << 4), v[h + 4 * k], v[h + 4 * k + 1],
+                     v[h + 4 * k + 2], v[h + 4 * k + 3]);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmD, xbase + c + h, ybase, stage);
+              bulk_commit();
             }
+          }
+        } else {
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(v[8 * k + 2 * e]),
+                                                        __uint_as_float(v[8 * k + 2 * e + 1]));
+              o[e] = *reinterpret_cast<uint32_t*>(&hh);
+            }
+            sts128(my_row + (((uint32_t)k ^ sw) << 4), o[0], o[1], o[2], o[3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmD, xbase + c, ybase, stage);
+            bulk_commit();
           }
         }
       }
@@ -507,6 +552,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
     }
+    if (lane == 0) bulk_wait0();  // every store of this warp has landed before exit
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -544,8 +591,8 @@ bool make_map(CUtensorMap* map, const UmmaOperand& op, int box_rows) {
 }
 
 template <int BN, bool A_MN, bool B_MN, bool B_RES>
-cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
-                     const char* family, cudaStream_t s) {
+cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
+                     const Params& p, int grid, const char* family, cudaStream_t s) {
   auto kern = k_umma_gemm<BN, A_MN, B_MN, B_RES>;
   static bool attr_done[64] = {false};  // once per device, outside any stream capture
   int dev = 0;
@@ -558,22 +605,39 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const Params&
     attr_done[dev] = true;
   }
   begin_launch(family, s);
-  kern<<<grid, kThreads, Cfg<BN, B_RES>::SMEM_BYTES, s>>>(ma, mb, p);
+  kern<<<grid, kThreads, Cfg<BN, B_RES>::SMEM_BYTES, s>>>(ma, mb, md, p);
   end_launch(family, s);
   return cudaGetLastError();
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, int grid,
-                      bool a_mn, bool b_mn, bool b_res, const char* family, cudaStream_t s) {
+cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
+                      const Params& p, int grid, bool a_mn, bool b_mn, bool b_res,
+                      const char* family, cudaStream_t s) {
   if (b_res) {  // A K-major only
-    if (!b_mn) return launch_t<BN, false, false, true>(ma, mb, p, grid, family, s);
-    return launch_t<BN, false, true, true>(ma, mb, p, grid, family, s);
+    if (!b_mn) return launch_t<BN, false, false, true>(ma, mb, md, p, grid, family, s);
+    return launch_t<BN, false, true, true>(ma, mb, md, p, grid, family, s);
   }
-  if (!a_mn && !b_mn) return launch_t<BN, false, false, false>(ma, mb, p, grid, family, s);
-  if (!a_mn && b_mn) return launch_t<BN, false, true, false>(ma, mb, p, grid, family, s);
-  if (a_mn && b_mn) return launch_t<BN, true, true, false>(ma, mb, p, grid, family, s);
-  return launch_t<BN, true, false, false>(ma, mb, p, grid, family, s);
+  if (!a_mn && !b_mn) return launch_t<BN, false, false, false>(ma, mb, md, p, grid, family, s);
+  if (!a_mn && b_mn) return launch_t<BN, false, true, false>(ma, mb, md, p, grid, family, s);
+  if (a_mn && b_mn) return launch_t<BN, true, true, false>(ma, mb, md, p, grid, family, s);
+  return launch_t<BN, true, false, false>(ma, mb, md, p, grid, family, s);
+}
+
+// Store map of the output: 32-row boxes of 128 bytes (64 bf16 or 32 fp32), 128-byte swizzle.
+bool make_out_map(CUtensorMap* map, void* ptr, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -628,14 +692,23 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   p.d_boff = g.d_boff;
   p.d_split = g.d_split;
   p.err = device_error_flag();
+  // output as a 2-D row-major tensor: batch entries / splits are row offsets (d_boff,
+  // d_split multiples of ldd) or column offsets (d_boff_col)
+  if (g.ldd <= 0 || g.d_boff % g.ldd != 0 || g.d_split % g.ldd != 0) return cudaErrorInvalidValue;
+  p.y_per_bz = (int)(g.d_boff / g.ldd);
+  p.y_per_split = (int)(g.d_split / g.ldd);
+  const int64_t out_rows = g.d_split ? (int64_t)p.ksplit * (g.d_split / g.ldd)
+                                     : (g.d_boff ? (int64_t)g.batch * (g.d_boff / g.ldd) : g.M);
+  CUtensorMap md;
+  if (!make_out_map(&md, g.D, out_rows, g.ldd, g.ldd, g.out_f32 != 0)) return cudaErrorInvalidValue;
   int grid = num_sms();
   if (grid > p.num_items) grid = p.num_items;
   // keep B resident when one item's whole B (K <= 256) fits and the items share it
   const bool b_res = !g.A.mn_major && p.kcps <= 4 && p.ksplit == 1 &&
                      p.num_items >= 2 * grid && p.tiles_m >= 2;
   if (BN == 256)
-    return launch_bn<256>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
-  return launch_bn<128>(ma, mb, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
+    return launch_bn<256>(ma, mb, md, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
+  return launch_bn<128>(ma, mb, md, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
 }
 
 }  // namespace poetx
