@@ -35,15 +35,21 @@ constexpr int kStageFloats = 2 * kBK * kLD;
 constexpr int kRingFloats = kGroups * kStages * kStageFloats;  // 139 KB
 constexpr int kRedFloats = kGroups * 64 * 64;                   // 64 KB of partial tiles
 constexpr int kMirFloats = 2 * 64 * 65;                         // mirror staging
-constexpr int kPairFloats = 5 * 64 * 65;  // symmetrising job: 2 inputs + 3 outputs (d <= 3)
-constexpr int kSmemFloats0 =
-    kRingFloats > kRedFloats + kMirFloats ? kRingFloats : kRedFloats + kMirFloats;
-constexpr int kSmemFloats = kSmemFloats0 > kPairFloats ? kSmemFloats0 : kPairFloats;
-static_assert(kSmemFloats >= kPairFloats && kSmemFloats >= kRedFloats + kMirFloats &&
-                  kSmemFloats >= kRingFloats,
-              "shared memory must hold every job type's tiles");
+constexpr int kPairFloats = 4 * 64 * 65;  // symmetrising job: 2 inputs x tiles (I,J), (J,I)
+// Epilogue operand tiles (the adds of a product, or the pair epilogue's (I,J) and (J,I)
+// tiles) are fetched with the first k tiles into their own region after the ring, so
+// the epilogue never waits on L2.  Row stride 68 keeps 16-byte cp.async destinations.
+constexpr int kEpiTiles = 4;
+constexpr int kELD = 68;
+constexpr int kEpiFloats = kEpiTiles * 64 * kELD;
+constexpr int kSmemFloats = kRingFloats + kEpiFloats;
+static_assert(kPairFloats <= kRingFloats && kRedFloats + kMirFloats <= kRingFloats &&
+                  kRedFloats + 2 * 64 * 65 <= kRingFloats,
+              "every job type's staging must fit in the ring region");
 constexpr int kSmemBytes = kSmemFloats * 4;
+static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory per CTA");
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;  // 64 x 64 tile-pair jobs
 
 __device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
@@ -56,6 +62,9 @@ __device__ __forceinline__ void cp_wait() {
 }
 __device__ __forceinline__ float4 ldcg4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ void st4(float* p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
 }
 __device__ __forceinline__ unsigned long long gtimer() {
   unsigned long long t;
@@ -81,6 +90,93 @@ __device__ __forceinline__ int64_t tri_idx(int i, int j, int b) {
   return (int64_t)i * b - (int64_t)i * (i + 1) / 2 + (j - i - 1);
 }
 
+// ------------------------------------------------------------------ pair epilogue
+// After a pair item's reduction: red[0..1] hold tile (I,J) of X, red[2..3] tile (J,I)
+// (for I == J all four hold partials of the one tile).  X and X^T are combined here; the
+// other operand's (I,J) and (J,I) tiles were prefetched into the epilogue region, so
+// every global access is a coalesced row and every transposed read comes from smem.
+__device__ void pair_epilogue(const CnpJob& J, int z, int I, int Jt, int b, float* smem) {
+  const int tid = threadIdx.x;
+  const bool diag = (I == Jt);
+  const float* red = smem;
+  float (*X1)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kRedFloats);
+  float (*X2)[kPLD] = diag ? X1 : reinterpret_cast<float (*)[kPLD]>(smem + kRedFloats + 64 * kPLD);
+  const float (*GA)[kELD] = reinterpret_cast<const float (*)[kELD]>(smem + kRingFloats);
+  const float (*GB)[kELD] = (diag || J.pair == PAIR_T)
+                                ? GA
+                                : reinterpret_cast<const float (*)[kELD]>(smem + kRingFloats + 64 * kELD);
+  const int64_t boff = (int64_t)z * b * b;
+  const int i0 = I * 64, j0 = Jt * 64;
+  // combine the partial tiles (fixed order)
+  for (int e = tid; e < 64 * 64; e += kThreads) {
+    const int r = e >> 6, c = e & 63;
+    if (diag) {
+      X1[r][c] = J.alpha * (red[e] + red[4096 + e] + red[2 * 4096 + e] + red[3 * 4096 + e]);
+    } else {
+      X1[r][c] = J.alpha * (red[e] + red[4096 + e]);
+      X2[r][c] = J.alpha * (red[2 * 4096 + e] + red[3 * 4096 + e]);
+    }
+  }
+  __syncthreads();
+  // pass 0: positions (i, j) of tile (I, J); pass 1: the mirrored tile (J, I).  For
+  // PAIR_T, G = add[0] is symmetric, so its (j, i) element is read as (i, j).  A thread
+  // forms 4 consecutive elements of a row (one 16-byte store per output).
+  const int passes = (!diag && J.pair != PAIR_PACK) ? 2 : 1;
+  for (int pass = 0; pass < passes; ++pass) {
+    for (int e = tid; e < 64 * 16; e += kThreads) {
+      const int r = e >> 4, c4 = (e & 15) * 4;
+      float xs[4], xd[4], gs[4], gd[4];  // X_ij + X_ji, X_ij - X_ji, same for G
+      float gt[4];                       // G_ji (the dG^T copy)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int c = c4 + w;
+        float xij, xji, gij, gji;
+        if (pass == 0) {
+          xij = X1[r][c];
+          xji = X2[c][r];
+          gij = GA[r][c];
+          gji = (J.pair == PAIR_T) ? gij : GB[c][r];
+        } else {
+          xij = X1[c][r];
+          xji = X2[r][c];
+          gij = GA[c][r];
+          gji = (J.pair == PAIR_T) ? gij : GB[r][c];
+        }
+        xs[w] = xij + xji;
+        xd[w] = xij - xji;
+        gs[w] = gij + gji;
+        gd[w] = gij - gji;
+        gt[w] = (pass == 0) ? gji : gij;
+      }
+      // pass 0 writes row i0 + r from column j0 + c4; pass 1 row j0 + r from column i0 + c4
+      const int64_t dst = (pass == 0) ? (int64_t)(i0 + r) * b + j0 + c4
+                                      : (int64_t)(j0 + r) * b + i0 + c4;
+      if (J.pair == PAIR_N) {
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+          if (o >= J.nout) break;
+          float* out = (o == 0) ? J.C : (o == 1) ? J.C2 : J.add_out[0];
+          const float a0 = J.coef[o][0], a1 = J.coef[o][1];
+          st4(out + boff + dst, a0 * gs[0] + a1 * xs[0], a0 * gs[1] + a1 * xs[1],
+              a0 * gs[2] + a1 * xs[2], a0 * gs[3] + a1 * xs[3]);
+        }
+        if (J.Cb_f) st4(J.Cb_f + boff + dst, gt[0], gt[1], gt[2], gt[3]);  // dG^T
+      } else if (J.pair == PAIR_T) {
+        // G symmetric: gs = 2 G_ij
+        st4(J.C + boff + dst, 0.5f * gs[0] + xs[0], 0.5f * gs[1] + xs[1], 0.5f * gs[2] + xs[2],
+            0.5f * gs[3] + xs[3]);
+      } else {  // PAIR_PACK, pass 0 only: i < j
+        float* th = J.C + z * ((int64_t)b * (b - 1) / 2);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int i = i0 + r, j = j0 + c4 + w;
+          if (i < j) th[tri_idx(i, j, b)] = J.addc[0] * gd[w] + xd[w];
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ product tile
 // C-tile (64 x 64) of one block: acc = op(A1) B1 (+ alpha2 op(A2) B2), every A read by rows
 // (symmetric, skew, or given transposed), then the structured epilogue.
@@ -90,13 +186,19 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   const int tx = gtid & 15, ty = gtid >> 4;
   const int nt = b / 64;
   int I, Jt;
-  if (J.mode == SG_FULL) {
+  if (J.mode == SG_FULL && !J.pair) {
     I = t / nt;
     Jt = t - I * nt;
   } else {
     tile_pair(nt, t, I, Jt);
   }
-  const int m0 = I * 64, n0 = Jt * 64;
+  // pair items with I != J: groups 0-1 compute tile (I, J), groups 2-3 tile (J, I), each
+  // splitting K in two; otherwise all groups split K of the one tile four ways
+  const bool two_tiles = J.pair && I != Jt;
+  const int tile_id = two_tiles ? (grp >> 1) : 0;
+  const int gsplit = two_tiles ? (grp & 1) : grp;
+  const int nsplit = two_tiles ? 2 : kGroups;
+  const int m0 = (tile_id ? Jt : I) * 64, n0 = (tile_id ? I : Jt) * 64;
   const int64_t boff = (int64_t)z * b * b;
   const float* A1 = J.A + boff;
   const float* B1 = J.B + boff;
@@ -106,8 +208,8 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   const int nk2 = A2 ? b / kBK : 0;
   const int nkt = nk1 + nk2;
   // this group's k tiles
-  const int kt_begin = (grp * nkt) / kGroups;
-  const int kt_end = ((grp + 1) * nkt) / kGroups;
+  const int kt_begin = (gsplit * nkt) / nsplit;
+  const int kt_end = ((gsplit + 1) * nkt) / nsplit;
   const float s1 = J.a_sym < 0 ? -1.f : 1.f;
   const float s2 = J.a2_sym < 0 ? -1.f : 1.f;
   const float boundary = s1 * s2 * J.alpha2;
@@ -150,8 +252,33 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   };
 #pragma unroll
   for (int st = 0; st < kStages - 1; ++st) issue(kt_begin + st);
+  // epilogue operand tiles: one cp.async group of their own, committed after the first
+  // kStages - 1 k tiles, so they queue behind the operands the mainloop needs first
+  {
+    float* E = smem + kRingFloats;
+    auto fetch = [&](int e, const float* src, int row0, int col0) {
+      const float* g0 = src + boff + (int64_t)row0 * b + col0;
+#pragma unroll
+      for (int l = 0; l < 64 * 16 / kThreads; ++l) {
+        const int f = tid + l * kThreads;
+        const int r = f >> 4, c4 = (f & 15) * 4;
+        cp_async16(E + e * 64 * kELD + r * kELD + c4, g0 + (int64_t)r * b + c4);
+      }
+    };
+    if (J.pair) {
+      const float* G = (J.pair == PAIR_N) ? J.B : J.add[0];
+      fetch(0, G, I * 64, Jt * 64);
+      if (I != Jt && J.pair != PAIR_T) fetch(1, G, Jt * 64, I * 64);
+    } else {
+      for (int q = 0; q < J.nadd; ++q) fetch(q, J.add[q], m0, n0);
+      if (J.skew_add) fetch(J.nadd, J.skew_add, m0, n0);
+    }
+    cp_commit();
+  }
   for (int kt = kt_begin; kt < kt_end; ++kt) {
-    cp_wait<kStages - 2>();
+    // k tile kt is complete once at most kStages - 2 later groups are pending (plus the
+    // epilogue group while it is still younger than kt)
+    if (kt - kt_begin < kStages - 1) cp_wait<kStages - 1>(); else cp_wait<kStages - 2>();
     group_sync();
     issue(kt + kStages - 1);
     if (nk2 > 0 && kt == nk1 && kt > kt_begin) {
@@ -179,7 +306,7 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   cp_wait<0>();
   __syncthreads();  // every group is done with its ring: the space becomes red[]
 
-  // partial tiles -> red[grp][row][col]
+  // partial tiles -> red[grp][row][col]  (pair items: red[0..1] tile (I,J), red[2..3] (J,I))
   float* red = smem;
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
@@ -188,6 +315,10 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
                                                   g_scale * acc[r][2], g_scale * acc[r][3]);
   }
   __syncthreads();
+  if (J.pair) {
+    pair_epilogue(J, z, I, Jt, b, smem);
+    return;
+  }
   // epilogue: thread owns row il and 8 consecutive columns of the tile
   // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
   float* C = J.C + boff;
@@ -223,9 +354,10 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
     sym[c] = dg ? J.diag : 0.f;
     sym2[c] = dg ? J.diag2 : 0.f;
   }
+  const float* E = smem + kRingFloats + il * kELD + jl0;
   for (int q = 0; q < J.nadd; ++q) {
-    const float4 x0 = ldcg4(J.add[q] + boff + row + j0);
-    const float4 x1 = ldcg4(J.add[q] + boff + row + j0 + 4);
+    const float4 x0 = *reinterpret_cast<const float4*>(E + q * 64 * kELD);
+    const float4 x1 = *reinterpret_cast<const float4*>(E + q * 64 * kELD + 4);
     const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -237,8 +369,8 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
 #pragma unroll
   for (int c = 0; c < 8; ++c) skew[c] = J.alpha * a[c];
   if (J.skew_add) {
-    const float4 x0 = ldcg4(J.skew_add + boff + row + j0);
-    const float4 x1 = ldcg4(J.skew_add + boff + row + j0 + 4);
+    const float4 x0 = *reinterpret_cast<const float4*>(E + J.nadd * 64 * kELD);
+    const float4 x1 = *reinterpret_cast<const float4*>(E + J.nadd * 64 * kELD + 4);
     const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
     for (int c = 0; c < 8; ++c) skew[c] += J.skew_c * xs[c];
@@ -296,14 +428,35 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   }  // passes
   if (structured) {
     __syncthreads();  // staged mirror values of every pass are visible
-    for (int e = tid; e < 64 * 64; e += kThreads) {
-      const int jl = e >> 6, il2 = e & 63;
-      if (I == Jt && il2 >= jl) continue;
-      const int64_t ji = (int64_t)(n0 + jl) * b + m0 + il2;
-      const float vmv = Ms[il2][jl];
-      C[ji] = vmv;
-      if (Cb) Cb[ji] = __float2bfloat16_rn(vmv);
-      if (C2) C2[ji] = Ms2[il2][jl];
+    // row jl of the mirrored tile is column jl of this one; a thread writes 4 consecutive
+    // elements (wide stores: the store count, not the bytes, sets the cost here)
+    for (int e = tid; e < 64 * 16; e += kThreads) {
+      const int jl = e >> 4, il4 = (e & 15) * 4;
+      const int64_t ji = (int64_t)(n0 + jl) * b + m0 + il4;
+      const float4 v = make_float4(Ms[il4][jl], Ms[il4 + 1][jl], Ms[il4 + 2][jl], Ms[il4 + 3][jl]);
+      if (I != Jt) {
+        *reinterpret_cast<float4*>(C + ji) = v;
+        if (Cb) {
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(v.z, v.w);
+          uint2 o;
+          o.x = *reinterpret_cast<uint32_t*>(&h0);
+          o.y = *reinterpret_cast<uint32_t*>(&h1);
+          *reinterpret_cast<uint2*>(Cb + ji) = o;
+        }
+        if (C2)
+          *reinterpret_cast<float4*>(C2 + ji) =
+              make_float4(Ms2[il4][jl], Ms2[il4 + 1][jl], Ms2[il4 + 2][jl], Ms2[il4 + 3][jl]);
+      } else {  // diagonal tile: the strictly lower triangle only
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (il4 + u >= jl) continue;
+          C[ji + u] = vv[u];
+          if (Cb) Cb[ji + u] = __float2bfloat16_rn(vv[u]);
+          if (C2) C2[ji + u] = Ms2[il4 + u][jl];
+        }
+      }
     }
   }
 }
@@ -311,7 +464,15 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
 // ------------------------------------------------------------------ 64 x 64 tile-pair jobs
 // Tile pair (I, J), I <= J, of a block; thread (tx = tid & 63, ty = tid >> 6) walks rows
 // ty, ty + 8, ... of the 64 x 64 tile, so each row is one coalesced 256-byte access.
-constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;
+
+// A thread handles 4 consecutive columns c4.. of rows r = (tid >> 4) + 32 u (u < 2) of a
+// tile: every global access is a 16-byte vector of a coalesced row (the number of
+// requests, not the bytes, bounds these small jobs), and all of a thread's loads are
+// issued before any of them is used, so a tile costs one L2 round trip.
+constexpr int kQuadRows = kThreads / 16;           // rows covered per sweep
+constexpr int kQuadSweeps = kPT / kQuadRows;        // sweeps per 64-row tile
+static_assert(kQuadRows * kQuadSweeps == kPT, "tile sweep");
+
 
 // theta -> Q: Q_ij = theta, Q_ji = -theta
 __device__ void expand_tile(const CnpJob& J, int z, int t, int b, float* smem) {
@@ -321,66 +482,111 @@ __device__ void expand_tile(const CnpJob& J, int z, int t, int b, float* smem) {
   const int64_t ntri = (int64_t)b * (b - 1) / 2;
   const float* th = J.A + z * ntri;
   float* q = J.C + (int64_t)z * b * b;
-  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
-  for (int r = ty; r < kPT; r += kPRows) {
-    const int i = I * kPT + r, j = Jt * kPT + tx;
-    tt[r][tx] = (i < j) ? __ldcg(th + tri_idx(i, j, b)) : 0.f;
-  }
-  __syncthreads();
-  for (int r = ty; r < kPT; r += kPRows) {
-    const int i = I * kPT + r, j = Jt * kPT + tx;
-    q[(int64_t)i * b + j] = (I == Jt && r > tx) ? -tt[tx][r] : tt[r][tx];
-  }
-  if (I != Jt) {
-    for (int r = ty; r < kPT; r += kPRows) {
-      const int i = Jt * kPT + r, j = I * kPT + tx;
-      q[(int64_t)i * b + j] = -tt[tx][r];
+  const int c4 = (threadIdx.x & 15) * 4, r0 = threadIdx.x >> 4;
+  float v[kQuadSweeps][4];
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u) {
+    const int i = I * kPT + r0 + u * kQuadRows;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = Jt * kPT + c4 + w;
+      v[u][w] = (i < j) ? __ldcg(th + tri_idx(i, j, b)) : 0.f;
     }
+  }
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) tt[r0 + u * kQuadRows][c4 + w] = v[u][w];
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u) {
+    const int r = r0 + u * kQuadRows;
+    float o[4], m[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int c = c4 + w;
+      o[w] = (I == Jt && r > c) ? -tt[c][r] : tt[r][c];
+      m[w] = -tt[c][r];
+    }
+    st4(q + (int64_t)(I * kPT + r) * b + Jt * kPT + c4, o[0], o[1], o[2], o[3]);
+    if (I != Jt) st4(q + (int64_t)(Jt * kPT + r) * b + I * kPT + c4, m[0], m[1], m[2], m[3]);
   }
 }
 
-// out_o = sum_s coef[o][s] (X_s + X_s^T) (symmetric outputs), optional Cb_f = X_0^T
+// out_o = sum_s coef[o][s] (X_s + X_s^T) (symmetric outputs), optional Cb_f = X_0^T.
+// Both tiles (I,J) and (J,I) of every input are staged first; each output element is then
+// formed directly (the sum is commutative, so diagonal tiles come out exactly symmetric).
 __device__ void symcomb_tile(const CnpJob& J, int z, int t, int b, float* smem) {
-  float (*ta)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
-  float (*tb)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kPT * kPLD);
-  float (*acc)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem + 2 * kPT * kPLD);
+  float (*ta)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem);            // X_s(I,J)
+  float (*tb)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem + 2 * kPT * kPLD);  // X_s(J,I)
   int I, Jt;
   tile_pair(b / kPT, t, I, Jt);
   const int64_t base = (int64_t)z * b * b;
-  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
-  const float* X[2] = {J.A, J.B};
-  float* out[4] = {J.C, J.C2, J.add_out[0], J.add_out[1]};
-  for (int o = 0; o < J.nout; ++o)
-    for (int r = ty; r < kPT; r += kPRows) acc[o][r][tx] = 0.f;
-  for (int s = 0; s < J.nin; ++s) {
-    const float* x = X[s] + base;
-    __syncthreads();
-    for (int r = ty; r < kPT; r += kPRows) {
-      ta[r][tx] = __ldcg(x + (int64_t)(I * kPT + r) * b + Jt * kPT + tx);
-      tb[r][tx] = __ldcg(x + (int64_t)(Jt * kPT + r) * b + I * kPT + tx);
+  const int c4 = (threadIdx.x & 15) * 4, r0 = threadIdx.x >> 4;
+  const int nin = J.nin, nout = J.nout;
+  float4 va[2][kQuadSweeps], vb[2][kQuadSweeps];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    if (s >= nin) break;
+    const float* x = (s == 0 ? J.A : J.B) + base;
+#pragma unroll
+    for (int u = 0; u < kQuadSweeps; ++u) {
+      const int r = r0 + u * kQuadRows;
+      va[s][u] = ldcg4(x + (int64_t)(I * kPT + r) * b + Jt * kPT + c4);
+      vb[s][u] = ldcg4(x + (int64_t)(Jt * kPT + r) * b + I * kPT + c4);
     }
-    __syncthreads();
-    for (int r = ty; r < kPT; r += kPRows) {
-      const float v = ta[r][tx] + tb[tx][r];  // (X + X^T)[I*64 + r, J*64 + tx]
-      for (int o = 0; o < J.nout; ++o) acc[o][r][tx] += J.coef[o][s] * v;
-    }
-    if (s == 0 && J.Cb_f) {  // transposed copy: (I,J) <- X(J,I)^T, (J,I) <- X(I,J)^T
-      float* y = J.Cb_f + base;
-      for (int r = ty; r < kPT; r += kPRows) {
-        y[(int64_t)(I * kPT + r) * b + Jt * kPT + tx] = tb[tx][r];
-        if (I != Jt) y[(int64_t)(Jt * kPT + r) * b + I * kPT + tx] = ta[tx][r];
-      }
+  }
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    if (s >= nin) break;
+#pragma unroll
+    for (int u = 0; u < kQuadSweeps; ++u) {
+      const int r = r0 + u * kQuadRows;
+      ta[s][r][c4] = va[s][u].x; ta[s][r][c4 + 1] = va[s][u].y;
+      ta[s][r][c4 + 2] = va[s][u].z; ta[s][r][c4 + 3] = va[s][u].w;
+      tb[s][r][c4] = vb[s][u].x; tb[s][r][c4 + 1] = vb[s][u].y;
+      tb[s][r][c4 + 2] = vb[s][u].z; tb[s][r][c4 + 3] = vb[s][u].w;
     }
   }
   __syncthreads();
-  for (int o = 0; o < J.nout; ++o) {
-    float* y = out[o] + base;
-    for (int r = ty; r < kPT; r += kPRows)
-      y[(int64_t)(I * kPT + r) * b + Jt * kPT + tx] =
-          (I == Jt && r > tx) ? acc[o][tx][r] : acc[o][r][tx];
-    if (I != Jt)
-      for (int r = ty; r < kPT; r += kPRows)
-        y[(int64_t)(Jt * kPT + r) * b + I * kPT + tx] = acc[o][tx][r];
+  const bool two = (I != Jt);
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u) {
+    const int r = r0 + u * kQuadRows;
+    // (X + X^T) at (I*64 + r, J*64 + c) and, for the mirrored tile, (J*64 + r, I*64 + c)
+    float v1[2][4], v2[2][4];
+#pragma unroll
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        v1[s][w] = (s < nin) ? ta[s][r][c4 + w] + tb[s][c4 + w][r] : 0.f;
+        v2[s][w] = (s < nin) ? tb[s][r][c4 + w] + ta[s][c4 + w][r] : 0.f;
+      }
+#pragma unroll
+    for (int o = 0; o < 4; ++o) {
+      if (o >= nout) break;
+      float a1[4] = {0.f, 0.f, 0.f, 0.f}, a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (s >= nin) break;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          a1[w] += J.coef[o][s] * v1[s][w];
+          a2[w] += J.coef[o][s] * v2[s][w];
+        }
+      }
+      float* y = (o == 0 ? J.C : o == 1 ? J.C2 : J.add_out[o - 2]) + base;
+      st4(y + (int64_t)(I * kPT + r) * b + Jt * kPT + c4, a1[0], a1[1], a1[2], a1[3]);
+      if (two) st4(y + (int64_t)(Jt * kPT + r) * b + I * kPT + c4, a2[0], a2[1], a2[2], a2[3]);
+    }
+    if (J.Cb_f) {  // transposed copy: (I,J) <- X_0(J,I)^T, (J,I) <- X_0(I,J)^T
+      float* y = J.Cb_f + base;
+      st4(y + (int64_t)(I * kPT + r) * b + Jt * kPT + c4, tb[0][c4][r], tb[0][c4 + 1][r],
+          tb[0][c4 + 2][r], tb[0][c4 + 3][r]);
+      if (two)
+        st4(y + (int64_t)(Jt * kPT + r) * b + I * kPT + c4, ta[0][c4][r], ta[0][c4 + 1][r],
+            ta[0][c4 + 2][r], ta[0][c4 + 3][r]);
+    }
   }
 }
 
@@ -392,13 +598,26 @@ __device__ void pack_tile(const CnpJob& J, int z, int t, int b, float* smem) {
   tile_pair(b / kPT, t, I, Jt);
   const float* a = J.A + (int64_t)z * b * b;
   float* th = J.C + z * ((int64_t)b * (b - 1) / 2);
-  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
-  for (int r = ty; r < kPT; r += kPRows) {
-    ta[r][tx] = __ldcg(a + (int64_t)(I * kPT + r) * b + Jt * kPT + tx);
-    tb[r][tx] = __ldcg(a + (int64_t)(Jt * kPT + r) * b + I * kPT + tx);
+  const int c4 = (threadIdx.x & 15) * 4, r0 = threadIdx.x >> 4;
+  float4 va[kQuadSweeps], vb[kQuadSweeps];
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u) {
+    const int r = r0 + u * kQuadRows;
+    va[u] = ldcg4(a + (int64_t)(I * kPT + r) * b + Jt * kPT + c4);
+    vb[u] = ldcg4(a + (int64_t)(Jt * kPT + r) * b + I * kPT + c4);
+  }
+#pragma unroll
+  for (int u = 0; u < kQuadSweeps; ++u) {
+    const int r = r0 + u * kQuadRows;
+    ta[r][c4] = va[u].x; ta[r][c4 + 1] = va[u].y; ta[r][c4 + 2] = va[u].z; ta[r][c4 + 3] = va[u].w;
+    tb[r][c4] = vb[u].x; tb[r][c4 + 1] = vb[u].y; tb[r][c4 + 2] = vb[u].z; tb[r][c4 + 3] = vb[u].w;
   }
   __syncthreads();
-  for (int r = ty; r < kPT; r += kPRows) {
+  // packed rows are contiguous in j but not 16-byte aligned: scalar stores, tx-major
+  const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
+#pragma unroll
+  for (int u = 0; u < kPT / kPRows; ++u) {
+    const int r = ty + u * kPRows;
     const int i = I * kPT + r, j = Jt * kPT + tx;
     if (i < j) th[tri_idx(i, j, b)] = ta[r][tx] - tb[tx][r];
   }
@@ -413,6 +632,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_item, s_next;
   __shared__ int s_ok;
+  // the current item's job descriptor, copied from the parameter space once per item so
+  // that the tile code reads its fields as shared-memory broadcasts
+  __shared__ __align__(16) int s_job[(sizeof(CnpJob) + 3) / 4];
   int* ticket = g.counters + g.njobs * g.nblk;
   const int total = g.item_start[g.njobs];
   if (threadIdx.x == 0) s_next = atomicAdd(ticket, 1);
@@ -427,17 +649,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
     if (item >= total) break;
     int j = 0;
     while (item >= g.item_start[j + 1]) ++j;
-    const CnpJob& J = g.job[j];
+    {
+      const int* src = reinterpret_cast<const int*>(&g.job[j]);
+      for (int w = threadIdx.x; w < (int)(sizeof(CnpJob) / 4); w += blockDim.x) s_job[w] = src[w];
+    }
+    const int tiles = g.job[j].tiles;
     const int local = item - g.item_start[j];
-    const int z = local / J.tiles;
-    const int t = local - z * J.tiles;
+    const int z = local / tiles;
+    const int t = local - z * tiles;
+    const unsigned deps = g.job[j].deps;
     if (threadIdx.x == 0) {
       // next ticket in flight while this item runs
       s_next = atomicAdd(ticket, 1);
       // wait until every job this one reads has finished for block z
       const unsigned long long t0 = gtimer();
       for (int d = 0; d < j && s_ok; ++d) {
-        if (!((J.deps >> d) & 1u)) continue;
+        if (!((deps >> d) & 1u)) continue;
         const int* cnt = g.counters + d * g.nblk + z;
         const int need = g.job[d].tiles;
         unsigned spins = 0;
@@ -454,8 +681,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
         }
       }
     }
-    __syncthreads();
+    __syncthreads();  // also publishes s_job
     if (!s_ok) break;
+    const CnpJob& J = *reinterpret_cast<const CnpJob*>(s_job);
     switch (J.type) {
       case JOB_EXPAND: expand_tile(J, z, t, g.b, smem); break;
       case JOB_PRODUCT: product_tile(J, z, t, g.b, smem); break;
@@ -474,10 +702,10 @@ __global__ void k_zero_ints(int* p, int n) {
 
 }  // namespace
 
-int cnp_graph_tiles(int type, int mode, int b) {
+int cnp_graph_tiles(int type, int mode, int pair, int b) {
   if (type == JOB_PRODUCT) {
     const int nt = b / 64;
-    return mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
+    return (mode == SG_FULL && !pair) ? nt * nt : nt * (nt + 1) / 2;
   }
   const int nt = b / 64;  // 64 x 64 tile pairs
   return nt * (nt + 1) / 2;
@@ -487,8 +715,17 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;
   g.item_start[0] = 0;
   for (int j = 0; j < g.njobs; ++j) {
-    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.b);
+    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.job[j].pair, g.b);
     g.item_start[j + 1] = g.item_start[j] + g.job[j].tiles * g.nblk;
+  }
+  for (int j = 0; j < g.njobs; ++j) {  // shapes the tile code relies on
+    const CnpJob& J = g.job[j];
+    if (J.type == JOB_PRODUCT && !J.pair && J.nadd + (J.skew_add ? 1 : 0) > kEpiTiles)
+      return cudaErrorInvalidValue;
+    if (J.type == JOB_PRODUCT && J.pair == PAIR_N && (J.nout < 1 || J.nout > 3))
+      return cudaErrorInvalidValue;
+    if (J.type == JOB_SYMCOMB && (J.nin < 1 || J.nin > 2 || J.nout < 1 || J.nout > 4))
+      return cudaErrorInvalidValue;
   }
   g.err = device_error_flag();
   const int ncount = g.njobs * g.nblk + 1;

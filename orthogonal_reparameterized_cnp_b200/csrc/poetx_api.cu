@@ -317,9 +317,10 @@ CnpJob prod_job(const float* A, int a_sym, const float* B, float* C, int mode, u
 // powers P_1 = Q Q, P_p = S P_{p-1}; the last also emits F' = sum_{j>=1} f_j P_j (C2).
 // Returns the job index of P_j in idx[j].
 void graph_powers(CnpGraph& g, int jQ, const float* Q, float* const* Pw, float* Fp,
-                  const CnpPoly& P, int* idx) {
+                  const CnpPoly& P, int* idx, int j_first = 1, int j_last = -1) {
   const int d = P.d;
-  for (int j = 1; j <= d; ++j) {
+  if (j_last < 0) j_last = d;
+  for (int j = j_first; j <= j_last; ++j) {
     CnpJob jb = (j == 1) ? prod_job(Q, -1, Q, Pw[1], SG_SYM, 1u << jQ)
                          : prod_job(Pw[1], 1, Pw[j - 1], Pw[j], SG_SYM,
                                     (1u << idx[1]) | (1u << idx[j - 1]));
@@ -371,6 +372,10 @@ int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* F
   return POETX_OK;
 }
 
+// Backward products as tile pairs whose epilogue forms the symmetrised / packed results
+// (fewer dependent steps), or as plain tiles followed by elementwise jobs.
+constexpr bool kBwdPairItems = false;
+
 struct BwdMats {
   float *Q, *P[4], *Fp, *D, *dGt, *N[4], *Pm, *R, *R2, *T, *T2, *A;
 };
@@ -388,28 +393,44 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   ex.C = M.Q;
   g.job[g.njobs++] = ex;
   int idx[4] = {0, 0, 0, 0};
-  graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx);
-  // D = Q dG (the adjoint reaching F is Q^T dG = -D)
-  const int jD = g.njobs;
-  g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
-  // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, and dG^T
-  const int jN = g.njobs;
-  {
-    CnpJob jn;
-    jn.type = JOB_SYMCOMB;
-    jn.A = dg;
-    jn.B = M.D;
-    jn.nin = 2;
+  // jobs are queued level by level so independent work is not stuck behind tiles that
+  // wait: S and the D / N step (both need only Q), then the higher powers, then the
+  // Horner terms
+  const bool pair = kBwdPairItems;
+  graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 1, 1);
+  // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, with D = Q dG (the adjoint reaching
+  // F is Q^T dG = -D), plus dG^T.  Pair items form D tile pair by tile pair and write the
+  // N_j directly; otherwise D is a product and a symmetrising job forms the N_j.
+  auto n_coefs = [&](CnpJob& jn) {
     jn.nout = d;
-    float* outs[4] = {M.N[1], d >= 2 ? M.N[2] : nullptr, d >= 3 ? M.N[3] : nullptr, nullptr};
-    jn.C = outs[0];
-    jn.C2 = outs[1];
-    jn.add_out[0] = outs[2];
+    jn.C = M.N[1];
+    jn.C2 = d >= 2 ? M.N[2] : nullptr;
+    jn.add_out[0] = d >= 3 ? M.N[3] : nullptr;
     for (int o = 0; o < d; ++o) {
       jn.coef[o][0] = P.e[o + 1];
       jn.coef[o][1] = -P.f[o + 1];
     }
     jn.Cb_f = M.dGt;
+  };
+  int jN = 0;
+  if (pair) {
+    jN = g.njobs;
+    CnpJob jn = prod_job(M.Q, -1, dg, M.N[1], SG_FULL, 1u);
+    jn.pair = PAIR_N;
+    n_coefs(jn);
+    g.job[g.njobs++] = jn;
+    if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
+  } else {
+    const int jD = g.njobs;
+    g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
+    if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
+    jN = g.njobs;
+    CnpJob jn;
+    jn.type = JOB_SYMCOMB;
+    jn.A = dg;
+    jn.B = M.D;
+    jn.nin = 2;
+    n_coefs(jn);
     jn.deps = 1u << jD;
     g.job[g.njobs++] = jn;
   }
@@ -419,23 +440,31 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   const int jS = idx[1];
   const float* S = M.P[1];
   if (d >= 2) {
-    const int jPm = g.njobs;
-    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
-    // T_{d-2} = N_{d-1} + Pm + Pm^T
+    // T_{d-2} = N_{d-1} + Pm + Pm^T with Pm = N_d S
     const int jT = g.njobs;
-    CnpJob jt;
-    jt.type = JOB_SYMCOMB;
-    jt.A = M.N[d - 1];
-    jt.B = M.Pm;
-    jt.nin = 2;
-    jt.nout = 1;
-    jt.coef[0][0] = 0.5f;
-    jt.coef[0][1] = 1.f;
-    jt.C = M.T;
-    jt.deps = (1u << jN) | (1u << jPm);
-    g.job[g.njobs++] = jt;
+    if (pair) {
+      CnpJob jt = prod_job(M.N[d], 1, S, M.T, SG_FULL, (1u << jN) | (1u << jS));
+      jt.pair = PAIR_T;
+      jt.add[0] = M.N[d - 1];
+      g.job[g.njobs++] = jt;
+    } else {
+      const int jPm = g.njobs;
+      g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
+      CnpJob jt;
+      jt.type = JOB_SYMCOMB;
+      jt.A = M.N[d - 1];
+      jt.B = M.Pm;
+      jt.nin = 2;
+      jt.nout = 1;
+      jt.coef[0][0] = 0.5f;  // N_{d-1} is symmetric: 0.5 (N + N^T) = N
+      jt.coef[0][1] = 1.f;
+      jt.C = M.T;
+      jt.deps = (1u << jN) | (1u << jPm);
+      g.job[g.njobs++] = jt;
+    }
+    const int jTT = pair ? jT : g.njobs - 1;
     Y = M.T;
-    jY = jT;
+    jY = jTT;
     if (d == 3) {
       // transposed Horner terms keep every A operand symmetric:
       //   Rt_1 = N_2 + S N_3,  Rt_0 = N_1 + S Rt_1,  T_0 = Rt_0 + T_1 S
@@ -452,7 +481,7 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       r0.nadd = 1;
       g.job[g.njobs++] = r0;
       const int jT0 = g.njobs;
-      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jT) | (1u << jS) | (1u << jR0));
+      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jTT) | (1u << jS) | (1u << jR0));
       t0.add[0] = M.R2;
       t0.addc[0] = 1.f;
       t0.nadd = 1;
@@ -461,9 +490,9 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       jY = jT0;
     }
   }
-  // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji
-  const int jA = g.njobs;
-  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL,
+  // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji (packed by the pair epilogue, or
+  // by a packing job)
+  CnpJob ja = prod_job(M.dGt, 2, M.Fp, pair ? dtheta : M.A, SG_FULL,
                        1u | (1u << jN) | (1u << idx[d]) | (1u << jY));
   ja.A2 = Y;
   ja.a2_sym = 1;
@@ -471,14 +500,20 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   ja.alpha2 = -1.f;
   ja.add[0] = dg;
   ja.addc[0] = P.f[0];
-  ja.nadd = 1;
-  g.job[g.njobs++] = ja;
-  CnpJob pk;
-  pk.type = JOB_PACK;
-  pk.A = M.A;
-  pk.C = dtheta;
-  pk.deps = 1u << jA;
-  g.job[g.njobs++] = pk;
+  if (pair) {
+    ja.pair = PAIR_PACK;
+    g.job[g.njobs++] = ja;
+  } else {
+    ja.nadd = 1;
+    const int jA = g.njobs;
+    g.job[g.njobs++] = ja;
+    CnpJob pk;
+    pk.type = JOB_PACK;
+    pk.A = M.A;
+    pk.C = dtheta;
+    pk.deps = 1u << jA;
+    g.job[g.njobs++] = pk;
+  }
   POETX_CUDA(launch_cnp_graph(g, s), "cnp graph (backward)");
   return POETX_OK;
 }
