@@ -23,7 +23,7 @@ namespace {
 // kGroups groups of 128 threads per CTA; in a product tile every group accumulates the
 // whole 64 x 64 tile over its own share of K (own cp.async ring), then the partial tiles
 // are summed through shared memory in a fixed order.  kCtasPerSm CTAs share an SM so that
-// one tile's load latency overlaps another tile's arithmetic.
+// one item's load / epilogue latency overlaps another item's arithmetic.
 constexpr int kGroups = 4;
 constexpr int kThreads = kGroups * 128;
 constexpr int kCtasPerSm = 4 / kGroups;
@@ -33,21 +33,21 @@ constexpr int kLD = 64 + 4;
 constexpr int kStages = 4;
 constexpr int kStageFloats = 2 * kBK * kLD;
 constexpr int kRingFloats = kGroups * kStages * kStageFloats;  // 139 KB
-constexpr int kRedFloats = kGroups * 64 * 64;                   // 64 KB of partial tiles
+constexpr int kRedFloats = kGroups * 64 * 64;                   // partial tiles
 constexpr int kMirFloats = 2 * 64 * 65;                         // mirror staging
 constexpr int kPairFloats = 4 * 64 * 65;  // symmetrising job: 2 inputs x tiles (I,J), (J,I)
-// Epilogue operand tiles (the adds of a product, or the pair epilogue's (I,J) and (J,I)
-// tiles) are fetched with the first k tiles into their own region after the ring, so
-// the epilogue never waits on L2.  Row stride 68 keeps 16-byte cp.async destinations.
-constexpr int kEpiTiles = 4;
+// Epilogue operand tiles (the adds and the skew term of a product) are fetched with the
+// first k tiles into their own region after the ring, so the epilogue never waits on
+// L2.  Row stride 68 keeps 16-byte cp.async destinations.
+constexpr int kEpiTiles = 2;
 constexpr int kELD = 68;
 constexpr int kEpiFloats = kEpiTiles * 64 * kELD;
 constexpr int kSmemFloats = kRingFloats + kEpiFloats;
-static_assert(kPairFloats <= kRingFloats && kRedFloats + kMirFloats <= kRingFloats &&
-                  kRedFloats + 2 * 64 * 65 <= kRingFloats,
-              "every job type's staging must fit in the ring region");
+static_assert(kRedFloats + kMirFloats <= kRingFloats,
+              "partial tiles and mirror staging must fit in the ring region");
+static_assert(kPairFloats <= kSmemFloats, "symmetrising job staging must fit");
 constexpr int kSmemBytes = kSmemFloats * 4;
-static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory per CTA");
+static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 227 * 1024, "shared memory per SM");
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;  // 64 x 64 tile-pair jobs
 
@@ -90,93 +90,6 @@ __device__ __forceinline__ int64_t tri_idx(int i, int j, int b) {
   return (int64_t)i * b - (int64_t)i * (i + 1) / 2 + (j - i - 1);
 }
 
-// ------------------------------------------------------------------ pair epilogue
-// After a pair item's reduction: red[0..1] hold tile (I,J) of X, red[2..3] tile (J,I)
-// (for I == J all four hold partials of the one tile).  X and X^T are combined here; the
-// other operand's (I,J) and (J,I) tiles were prefetched into the epilogue region, so
-// every global access is a coalesced row and every transposed read comes from smem.
-__device__ void pair_epilogue(const CnpJob& J, int z, int I, int Jt, int b, float* smem) {
-  const int tid = threadIdx.x;
-  const bool diag = (I == Jt);
-  const float* red = smem;
-  float (*X1)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kRedFloats);
-  float (*X2)[kPLD] = diag ? X1 : reinterpret_cast<float (*)[kPLD]>(smem + kRedFloats + 64 * kPLD);
-  const float (*GA)[kELD] = reinterpret_cast<const float (*)[kELD]>(smem + kRingFloats);
-  const float (*GB)[kELD] = (diag || J.pair == PAIR_T)
-                                ? GA
-                                : reinterpret_cast<const float (*)[kELD]>(smem + kRingFloats + 64 * kELD);
-  const int64_t boff = (int64_t)z * b * b;
-  const int i0 = I * 64, j0 = Jt * 64;
-  // combine the partial tiles (fixed order)
-  for (int e = tid; e < 64 * 64; e += kThreads) {
-    const int r = e >> 6, c = e & 63;
-    if (diag) {
-      X1[r][c] = J.alpha * (red[e] + red[4096 + e] + red[2 * 4096 + e] + red[3 * 4096 + e]);
-    } else {
-      X1[r][c] = J.alpha * (red[e] + red[4096 + e]);
-      X2[r][c] = J.alpha * (red[2 * 4096 + e] + red[3 * 4096 + e]);
-    }
-  }
-  __syncthreads();
-  // pass 0: positions (i, j) of tile (I, J); pass 1: the mirrored tile (J, I).  For
-  // PAIR_T, G = add[0] is symmetric, so its (j, i) element is read as (i, j).  A thread
-  // forms 4 consecutive elements of a row (one 16-byte store per output).
-  const int passes = (!diag && J.pair != PAIR_PACK) ? 2 : 1;
-  for (int pass = 0; pass < passes; ++pass) {
-    for (int e = tid; e < 64 * 16; e += kThreads) {
-      const int r = e >> 4, c4 = (e & 15) * 4;
-      float xs[4], xd[4], gs[4], gd[4];  // X_ij + X_ji, X_ij - X_ji, same for G
-      float gt[4];                       // G_ji (the dG^T copy)
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const int c = c4 + w;
-        float xij, xji, gij, gji;
-        if (pass == 0) {
-          xij = X1[r][c];
-          xji = X2[c][r];
-          gij = GA[r][c];
-          gji = (J.pair == PAIR_T) ? gij : GB[c][r];
-        } else {
-          xij = X1[c][r];
-          xji = X2[r][c];
-          gij = GA[c][r];
-          gji = (J.pair == PAIR_T) ? gij : GB[r][c];
-        }
-        xs[w] = xij + xji;
-        xd[w] = xij - xji;
-        gs[w] = gij + gji;
-        gd[w] = gij - gji;
-        gt[w] = (pass == 0) ? gji : gij;
-      }
-      // pass 0 writes row i0 + r from column j0 + c4; pass 1 row j0 + r from column i0 + c4
-      const int64_t dst = (pass == 0) ? (int64_t)(i0 + r) * b + j0 + c4
-                                      : (int64_t)(j0 + r) * b + i0 + c4;
-      if (J.pair == PAIR_N) {
-#pragma unroll
-        for (int o = 0; o < 3; ++o) {
-          if (o >= J.nout) break;
-          float* out = (o == 0) ? J.C : (o == 1) ? J.C2 : J.add_out[0];
-          const float a0 = J.coef[o][0], a1 = J.coef[o][1];
-          st4(out + boff + dst, a0 * gs[0] + a1 * xs[0], a0 * gs[1] + a1 * xs[1],
-              a0 * gs[2] + a1 * xs[2], a0 * gs[3] + a1 * xs[3]);
-        }
-        if (J.Cb_f) st4(J.Cb_f + boff + dst, gt[0], gt[1], gt[2], gt[3]);  // dG^T
-      } else if (J.pair == PAIR_T) {
-        // G symmetric: gs = 2 G_ij
-        st4(J.C + boff + dst, 0.5f * gs[0] + xs[0], 0.5f * gs[1] + xs[1], 0.5f * gs[2] + xs[2],
-            0.5f * gs[3] + xs[3]);
-      } else {  // PAIR_PACK, pass 0 only: i < j
-        float* th = J.C + z * ((int64_t)b * (b - 1) / 2);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int i = i0 + r, j = j0 + c4 + w;
-          if (i < j) th[tri_idx(i, j, b)] = J.addc[0] * gd[w] + xd[w];
-        }
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------ product tile
 // C-tile (64 x 64) of one block: acc = op(A1) B1 (+ alpha2 op(A2) B2), every A read by rows
 // (symmetric, skew, or given transposed), then the structured epilogue.
@@ -186,19 +99,13 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   const int tx = gtid & 15, ty = gtid >> 4;
   const int nt = b / 64;
   int I, Jt;
-  if (J.mode == SG_FULL && !J.pair) {
+  if (J.mode == SG_FULL) {
     I = t / nt;
     Jt = t - I * nt;
   } else {
     tile_pair(nt, t, I, Jt);
   }
-  // pair items with I != J: groups 0-1 compute tile (I, J), groups 2-3 tile (J, I), each
-  // splitting K in two; otherwise all groups split K of the one tile four ways
-  const bool two_tiles = J.pair && I != Jt;
-  const int tile_id = two_tiles ? (grp >> 1) : 0;
-  const int gsplit = two_tiles ? (grp & 1) : grp;
-  const int nsplit = two_tiles ? 2 : kGroups;
-  const int m0 = (tile_id ? Jt : I) * 64, n0 = (tile_id ? I : Jt) * 64;
+  const int m0 = I * 64, n0 = Jt * 64;
   const int64_t boff = (int64_t)z * b * b;
   const float* A1 = J.A + boff;
   const float* B1 = J.B + boff;
@@ -208,8 +115,8 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   const int nk2 = A2 ? b / kBK : 0;
   const int nkt = nk1 + nk2;
   // this group's k tiles
-  const int kt_begin = (gsplit * nkt) / nsplit;
-  const int kt_end = ((gsplit + 1) * nkt) / nsplit;
+  const int kt_begin = (grp * nkt) / kGroups;
+  const int kt_end = ((grp + 1) * nkt) / kGroups;
   const float s1 = J.a_sym < 0 ? -1.f : 1.f;
   const float s2 = J.a2_sym < 0 ? -1.f : 1.f;
   const float boundary = s1 * s2 * J.alpha2;
@@ -265,14 +172,8 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
         cp_async16(E + e * 64 * kELD + r * kELD + c4, g0 + (int64_t)r * b + c4);
       }
     };
-    if (J.pair) {
-      const float* G = (J.pair == PAIR_N) ? J.B : J.add[0];
-      fetch(0, G, I * 64, Jt * 64);
-      if (I != Jt && J.pair != PAIR_T) fetch(1, G, Jt * 64, I * 64);
-    } else {
-      for (int q = 0; q < J.nadd; ++q) fetch(q, J.add[q], m0, n0);
-      if (J.skew_add) fetch(J.nadd, J.skew_add, m0, n0);
-    }
+    for (int q = 0; q < J.nadd; ++q) fetch(q, J.add[q], m0, n0);
+    if (J.skew_add) fetch(J.nadd, J.skew_add, m0, n0);
     cp_commit();
   }
   for (int kt = kt_begin; kt < kt_end; ++kt) {
@@ -306,7 +207,7 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   cp_wait<0>();
   __syncthreads();  // every group is done with its ring: the space becomes red[]
 
-  // partial tiles -> red[grp][row][col]  (pair items: red[0..1] tile (I,J), red[2..3] (J,I))
+  // partial tiles -> red[grp][row][col]
   float* red = smem;
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
@@ -315,10 +216,6 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
                                                   g_scale * acc[r][2], g_scale * acc[r][3]);
   }
   __syncthreads();
-  if (J.pair) {
-    pair_epilogue(J, z, I, Jt, b, smem);
-    return;
-  }
   // epilogue: thread owns row il and 8 consecutive columns of the tile
   // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
   float* C = J.C + boff;
@@ -702,10 +599,10 @@ __global__ void k_zero_ints(int* p, int n) {
 
 }  // namespace
 
-int cnp_graph_tiles(int type, int mode, int pair, int b) {
+int cnp_graph_tiles(int type, int mode, int b) {
   if (type == JOB_PRODUCT) {
     const int nt = b / 64;
-    return (mode == SG_FULL && !pair) ? nt * nt : nt * (nt + 1) / 2;
+    return mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
   }
   const int nt = b / 64;  // 64 x 64 tile pairs
   return nt * (nt + 1) / 2;
@@ -715,14 +612,12 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;
   g.item_start[0] = 0;
   for (int j = 0; j < g.njobs; ++j) {
-    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.job[j].pair, g.b);
+    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.b);
     g.item_start[j + 1] = g.item_start[j] + g.job[j].tiles * g.nblk;
   }
   for (int j = 0; j < g.njobs; ++j) {  // shapes the tile code relies on
     const CnpJob& J = g.job[j];
-    if (J.type == JOB_PRODUCT && !J.pair && J.nadd + (J.skew_add ? 1 : 0) > kEpiTiles)
-      return cudaErrorInvalidValue;
-    if (J.type == JOB_PRODUCT && J.pair == PAIR_N && (J.nout < 1 || J.nout > 3))
+    if (J.type == JOB_PRODUCT && J.nadd + (J.skew_add ? 1 : 0) > kEpiTiles)
       return cudaErrorInvalidValue;
     if (J.type == JOB_SYMCOMB && (J.nin < 1 || J.nin > 2 || J.nout < 1 || J.nout > 4))
       return cudaErrorInvalidValue;

@@ -314,7 +314,10 @@ CnpJob prod_job(const float* A, int a_sym, const float* B, float* C, int mode, u
   return j;
 }
 
-// powers P_1 = Q Q, P_p = S P_{p-1}; the last also emits F' = sum_{j>=1} f_j P_j (C2).
+// powers P_1 = Q Q, P_p = S P_{p-1}.  The last product emits, instead of P_d itself,
+//   C  = E(S) = e_0 I + sum_{j>=1} e_j P_j     and     C2 = F' = sum_{j>=1} f_j P_j,
+// so later steps read one tile for each polynomial (for d = 1 the single product keeps
+// C = S, which the backward reads, and E is formed where it is used).
 // Returns the job index of P_j in idx[j].
 void graph_powers(CnpGraph& g, int jQ, const float* Q, float* const* Pw, float* Fp,
                   const CnpPoly& P, int* idx, int j_first = 1, int j_last = -1) {
@@ -327,9 +330,13 @@ void graph_powers(CnpGraph& g, int jQ, const float* Q, float* const* Pw, float* 
     if (j == d) {
       jb.C2 = Fp;
       jb.alpha_c2 = P.f[d];
+      if (d >= 2) {
+        jb.alpha = P.e[d];
+        jb.diag = P.e[0];
+      }
       for (int t = 1; t < d; ++t) {
         jb.add[jb.nadd] = Pw[t];
-        jb.addc[jb.nadd] = 0.f;
+        jb.addc[jb.nadd] = P.e[t];
         jb.addc2[jb.nadd] = P.f[t];
         ++jb.nadd;
         jb.deps |= 1u << idx[t];
@@ -355,26 +362,20 @@ int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* F
   g.job[g.njobs++] = ex;
   int idx[4] = {0, 0, 0, 0};
   graph_powers(g, 0, Q, Pw, Fp, P, idx);
-  // G = E + f_0 Q + Q F' (upper tiles; E symmetric, QF skew)
-  CnpJob jg = prod_job(Q, -1, Fp, G, SG_SYMSKEW, 1u);
+  // G = E + f_0 Q + Q F' (upper tiles; E symmetric, QF skew); E is the last power job's
+  // output for d >= 2, else e_0 I + e_1 S
+  CnpJob jg = prod_job(Q, -1, Fp, G, SG_SYMSKEW, 1u | (1u << idx[d]));
   jg.Cb = Gb;
-  jg.diag = P.e[0];
-  for (int j = 1; j <= d; ++j) {
-    jg.add[jg.nadd] = Pw[j];
-    jg.addc[jg.nadd] = P.e[j];
-    ++jg.nadd;
-    jg.deps |= 1u << idx[j];
-  }
+  jg.add[0] = Pw[d];
+  jg.addc[0] = d >= 2 ? 1.f : P.e[1];
+  jg.diag = d >= 2 ? 0.f : P.e[0];
+  jg.nadd = 1;
   jg.skew_add = Q;
   jg.skew_c = P.f[0];
   g.job[g.njobs++] = jg;
   POETX_CUDA(launch_cnp_graph(g, s), "cnp graph (forward)");
   return POETX_OK;
 }
-
-// Backward products as tile pairs whose epilogue forms the symmetrised / packed results
-// (fewer dependent steps), or as plain tiles followed by elementwise jobs.
-constexpr bool kBwdPairItems = false;
 
 struct BwdMats {
   float *Q, *P[4], *Fp, *D, *dGt, *N[4], *Pm, *R, *R2, *T, *T2, *A;
@@ -394,14 +395,20 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   g.job[g.njobs++] = ex;
   int idx[4] = {0, 0, 0, 0};
   // jobs are queued level by level so independent work is not stuck behind tiles that
-  // wait: S and the D / N step (both need only Q), then the higher powers, then the
-  // Horner terms
-  const bool pair = kBwdPairItems;
+  // wait: S and D (both need only Q), then the higher powers, then the Horner terms
   graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 1, 1);
-  // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, with D = Q dG (the adjoint reaching
-  // F is Q^T dG = -D), plus dG^T.  Pair items form D tile pair by tile pair and write the
-  // N_j directly; otherwise D is a product and a symmetrising job forms the N_j.
-  auto n_coefs = [&](CnpJob& jn) {
+  // D = Q dG (the adjoint reaching F is Q^T dG = -D)
+  const int jD = g.njobs;
+  g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
+  if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
+  // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, and dG^T
+  const int jN = g.njobs;
+  {
+    CnpJob jn;
+    jn.type = JOB_SYMCOMB;
+    jn.A = dg;
+    jn.B = M.D;
+    jn.nin = 2;
     jn.nout = d;
     jn.C = M.N[1];
     jn.C2 = d >= 2 ? M.N[2] : nullptr;
@@ -411,26 +418,6 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       jn.coef[o][1] = -P.f[o + 1];
     }
     jn.Cb_f = M.dGt;
-  };
-  int jN = 0;
-  if (pair) {
-    jN = g.njobs;
-    CnpJob jn = prod_job(M.Q, -1, dg, M.N[1], SG_FULL, 1u);
-    jn.pair = PAIR_N;
-    n_coefs(jn);
-    g.job[g.njobs++] = jn;
-    if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
-  } else {
-    const int jD = g.njobs;
-    g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
-    if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
-    jN = g.njobs;
-    CnpJob jn;
-    jn.type = JOB_SYMCOMB;
-    jn.A = dg;
-    jn.B = M.D;
-    jn.nin = 2;
-    n_coefs(jn);
     jn.deps = 1u << jD;
     g.job[g.njobs++] = jn;
   }
@@ -441,30 +428,22 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   const float* S = M.P[1];
   if (d >= 2) {
     // T_{d-2} = N_{d-1} + Pm + Pm^T with Pm = N_d S
+    const int jPm = g.njobs;
+    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
     const int jT = g.njobs;
-    if (pair) {
-      CnpJob jt = prod_job(M.N[d], 1, S, M.T, SG_FULL, (1u << jN) | (1u << jS));
-      jt.pair = PAIR_T;
-      jt.add[0] = M.N[d - 1];
-      g.job[g.njobs++] = jt;
-    } else {
-      const int jPm = g.njobs;
-      g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
-      CnpJob jt;
-      jt.type = JOB_SYMCOMB;
-      jt.A = M.N[d - 1];
-      jt.B = M.Pm;
-      jt.nin = 2;
-      jt.nout = 1;
-      jt.coef[0][0] = 0.5f;  // N_{d-1} is symmetric: 0.5 (N + N^T) = N
-      jt.coef[0][1] = 1.f;
-      jt.C = M.T;
-      jt.deps = (1u << jN) | (1u << jPm);
-      g.job[g.njobs++] = jt;
-    }
-    const int jTT = pair ? jT : g.njobs - 1;
+    CnpJob jt;
+    jt.type = JOB_SYMCOMB;
+    jt.A = M.N[d - 1];
+    jt.B = M.Pm;
+    jt.nin = 2;
+    jt.nout = 1;
+    jt.coef[0][0] = 0.5f;  // N_{d-1} is symmetric: 0.5 (N + N^T) = N
+    jt.coef[0][1] = 1.f;
+    jt.C = M.T;
+    jt.deps = (1u << jN) | (1u << jPm);
+    g.job[g.njobs++] = jt;
     Y = M.T;
-    jY = jTT;
+    jY = jT;
     if (d == 3) {
       // transposed Horner terms keep every A operand symmetric:
       //   Rt_1 = N_2 + S N_3,  Rt_0 = N_1 + S Rt_1,  T_0 = Rt_0 + T_1 S
@@ -481,7 +460,7 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       r0.nadd = 1;
       g.job[g.njobs++] = r0;
       const int jT0 = g.njobs;
-      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jTT) | (1u << jS) | (1u << jR0));
+      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jT) | (1u << jS) | (1u << jR0));
       t0.add[0] = M.R2;
       t0.addc[0] = 1.f;
       t0.nadd = 1;
@@ -490,9 +469,9 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       jY = jT0;
     }
   }
-  // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji (packed by the pair epilogue, or
-  // by a packing job)
-  CnpJob ja = prod_job(M.dGt, 2, M.Fp, pair ? dtheta : M.A, SG_FULL,
+  // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji
+  const int jA = g.njobs;
+  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL,
                        1u | (1u << jN) | (1u << idx[d]) | (1u << jY));
   ja.A2 = Y;
   ja.a2_sym = 1;
@@ -500,20 +479,14 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   ja.alpha2 = -1.f;
   ja.add[0] = dg;
   ja.addc[0] = P.f[0];
-  if (pair) {
-    ja.pair = PAIR_PACK;
-    g.job[g.njobs++] = ja;
-  } else {
-    ja.nadd = 1;
-    const int jA = g.njobs;
-    g.job[g.njobs++] = ja;
-    CnpJob pk;
-    pk.type = JOB_PACK;
-    pk.A = M.A;
-    pk.C = dtheta;
-    pk.deps = 1u << jA;
-    g.job[g.njobs++] = pk;
-  }
+  ja.nadd = 1;
+  g.job[g.njobs++] = ja;
+  CnpJob pk;
+  pk.type = JOB_PACK;
+  pk.A = M.A;
+  pk.C = dtheta;
+  pk.deps = 1u << jA;
+  g.job[g.njobs++] = pk;
   POETX_CUDA(launch_cnp_graph(g, s), "cnp graph (backward)");
   return POETX_OK;
 }

@@ -98,18 +98,11 @@ cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaS
 // one job for one block.  Square blocks with b % 64 == 0; products read every A operand
 // by rows (a_sym: -1 skew, +1 symmetric, 2 given as its transpose).
 enum CnpJobType { JOB_EXPAND = 0, JOB_PRODUCT = 1, JOB_SYMCOMB = 2, JOB_PACK = 3 };
-enum CnpPairKind { PAIR_NONE = 0, PAIR_N = 1, PAIR_T = 2, PAIR_PACK = 3 };
 constexpr int kCnpMaxJobs = 14;
 
 struct CnpJob {
   int type = JOB_PRODUCT;
   int mode = SG_FULL;       // products: SG_FULL / SG_SYM / SG_SYMSKEW
-  // products computed as tile pairs (I,J)+(J,I) whose epilogue combines X and X^T:
-  //   PAIR_N:    out_o = coef[o][0] (dG + dG^T) + coef[o][1] (X + X^T), o < nout, and
-  //              Cb_f = dG^T; dG = B        (outputs C, C2, add_out[0])
-  //   PAIR_T:    C = add[0] + X + X^T
-  //   PAIR_PACK: C[idx(i,j)] = addc[0] (add[0]_ij - add[0]_ji) + X_ij - X_ji   (i < j)
-  int pair = 0;
   int tiles = 0;            // items per block (filled in by the launcher)
   unsigned deps = 0;        // bit d: reads job d's output for the same block
   // products: C = epilogue(op(A) op(B) [+ alpha2 op(A2) op(B2)]), as SgemmArgs
