@@ -207,6 +207,19 @@ def poet_weight(W0, G_P, G_R, perm_P, perm_R) -> np.ndarray:
     return R @ np.asarray(W0, dtype=np.float64) @ P
 
 
+def outer_merge(W0, G_P, G_R, perm_P, perm_R, perm_P_new, perm_R_new):
+    """Outer-loop merge and re-initialisation.  The original POET step folds the rotations
+    into the weight, W <- R_i W P_i ([POET-X] technical summary 2.1, where it is the
+    weight-centric update the input-centric form replaces; [POET] abstract: W = R W0 P).
+    At the end of an inner loop the learnt R, P are absorbed this way, W0_new = R W0 P
+    (dense R, P built as in poet_weight), and the next inner loop starts from theta = 0
+    with fresh permutations, whose merged weight is W0'_new = Pi_R' W0_new Pi_P'^T.
+
+    Returns (W0_new, W0'_new)."""
+    W0_new = poet_weight(W0, G_P, G_R, perm_P, perm_R)
+    return W0_new, merge_perm(W0_new, perm_R_new, perm_P_new)
+
+
 def layer_dense(x, W0, G_P, G_R, perm_P, perm_R) -> np.ndarray:
     """Rows of Y = (R W0 P x_t)^T with the four permutations as matrices and the unmerged
     W0 (the weight-centric reading; small sizes only)."""

@@ -247,6 +247,56 @@ def test_spectrum_preserved_with_exact_cayley():
     assert np.allclose(s0, s1, rtol=1e-12, atol=1e-12)
 
 
+# ----------------------------------------------------------------- outer-loop merge
+def test_outer_merge_at_zero_theta_is_a_pure_remerge():
+    # theta = 0 => G = I: W0_new = W0 exactly and W0'_new is W0 gathered by the new maps.
+    n, m, b = 32, 48, 8
+    x, W0, tP, tR, dy, pP, pR = _small_layer(n, m, b, 4, 2, 21)
+    GP = ref.cnp_forward(np.zeros_like(tP), b, 4)
+    GR = ref.cnp_forward(np.zeros_like(tR), b, 4)
+    pP2, _ = ref.make_perm(101, n)
+    pR2, _ = ref.make_perm(102, m)
+    W0_new, W0p_new = ref.outer_merge(W0, GP, GR, pP, pR, pP2, pR2)
+    assert np.array_equal(W0_new, W0)
+    assert np.array_equal(W0p_new, W0[np.ix_(pR2, pP2)])
+
+
+def test_outer_merge_keeps_the_spectrum_with_exact_cayley():
+    # [POET] abstract: the transform preserves the singular values of W0, so the merge
+    # with exactly orthogonal factors must too.
+    n, m, b = 32, 24, 8
+    x, W0, tP, tR, dy, pP, pR = _small_layer(n, m, b, 4, 2, 23, scale=0.3)
+    CP = np.stack([ref.cayley_exact(ref.theta_to_Q(t, b)) for t in tP])
+    CR = np.stack([ref.cayley_exact(ref.theta_to_Q(t, b)) for t in tR])
+    pP2, _ = ref.make_perm(7, n)
+    pR2, _ = ref.make_perm(8, m)
+    W0_new, W0p_new = ref.outer_merge(W0, CP, CR, pP, pR, pP2, pR2)
+    s0 = np.linalg.svd(W0, compute_uv=False)
+    assert np.allclose(np.linalg.svd(W0_new, compute_uv=False), s0, rtol=1e-12, atol=1e-12)
+    assert np.allclose(np.linalg.svd(W0p_new, compute_uv=False), s0, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,m,b,k", [(16, 24, 4, 4), (64, 32, 16, 3)])
+def test_outer_merge_preserves_the_layer(n, m, b, k):
+    # The layer with rotations G and permutations p equals the layer after the merge with
+    # theta = 0 and new permutations p' (input-centric forward with index maps on both
+    # sides, so the merge is checked against a different code path than its own).
+    x, W0, tP, tR, dy, pP, pR = _small_layer(n, m, b, k, 5, n * m)
+    GP, GR = ref.cnp_forward(tP, b, k), ref.cnp_forward(tR, b, k)
+    pP2, _ = ref.make_perm(n + 5, n)
+    pR2, _ = ref.make_perm(m + 6, m)
+    y0 = ref.layer_forward(x, ref.merge_perm(W0, pR, pP), GP, GR, pP, pR)[0]
+    _, W0p_new = ref.outer_merge(W0, GP, GR, pP, pR, pP2, pR2)
+    I_P = ref.cnp_forward(np.zeros_like(tP), b, k)
+    I_R = ref.cnp_forward(np.zeros_like(tR), b, k)
+    y1 = ref.layer_forward(x, W0p_new, I_P, I_R, pP2, pR2)[0]
+    assert np.allclose(y1, y0, rtol=1e-12, atol=1e-12 * np.abs(y0).max())
+    # a planted mistake (the rotations applied transposed) breaks the equivalence
+    _, bad = ref.outer_merge(W0, GP.transpose(0, 2, 1), GR, pP, pR, pP2, pR2)
+    y2 = ref.layer_forward(x, bad, I_P, I_R, pP2, pR2)[0]
+    assert not np.allclose(y2, y0, rtol=1e-6, atol=1e-6 * np.abs(y0).max())
+
+
 @pytest.mark.parametrize("k", [2, 4])
 def test_spectrum_bounds_with_cnp(k):
     # P6 with the truncated G: each factor has singular values in [1-eps, 1+eps],
