@@ -12,9 +12,11 @@ Workload: the Llama-1B-shaped attention projection, n = m = 2048, b = 256, k = 4
 T = 8192 tokens (4 x 2048), bf16 activations, fp32 theta / CNP.  Inputs rotate over three
 seeded sets (192 MB of x and dy, larger than the 126 MB L2) between steps.
 
-Under torchrun (N > 1) every rank runs its own replica (weak scaling); the step time is
-the maximum over ranks.  ``--impl reference`` times the float64 CPU oracle instead
-(rank 0 only) on a bounded token sample per step.
+Under torchrun (N > 1) the step is data parallel (weak scaling): every rank takes its own
+T tokens with theta, G and W0' replicated, and the step ends with one NCCL sum all-reduce
+of dtheta; the step time is the maximum over ranks.  The outer-loop merge (once per inner
+loop, outside the step) is timed separately after the timed region.  ``--impl reference``
+times the float64 CPU oracle instead (rank 0 only) on a bounded token sample per step.
 """
 from __future__ import annotations
 
@@ -330,8 +332,15 @@ def run_poetx(args):
     dx = torch.empty((s.T, s.n), dtype=act, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    from orthogonal_reparameterized_cnp_b200 import dp
+
+    def exchange():  # the data-parallel step's one collective (a no-op on one rank)
+        if world > 1:
+            dp.allreduce_dtheta(layer.dtheta)
+
     def step(i):
         layer.step(xs[i % nsets], dys[i % nsets], y, dx, stream)
+        exchange()
 
     def barrier():
         if world > 1:
@@ -377,6 +386,7 @@ def run_poetx(args):
             graphs.append(gr)
         for i in range(3):
             graphs[i % nsets].replay()
+            exchange()
         torch.cuda.synchronize(dev)
         if P.device_status(stream) != P.POETX_OK:
             raise RuntimeError("device status not OK after graph warm-up")
@@ -392,7 +402,8 @@ def run_poetx(args):
     ev0.record(stream)
     for i in range(args.steps):
         if graphs:
-            graphs[i % nsets].replay()
+            graphs[i % nsets].replay()  # the layer's kernels; the collective stays outside
+            exchange()
         else:
             step(i)
     ev1.record(stream)
@@ -472,6 +483,7 @@ def run_poetx(args):
             ddyin.copy_(hdy[i % nsets], non_blocking=True)
             layer.theta.copy_(hth, non_blocking=True)
             layer.step(dxin, ddyin, y, dx, stream)
+            exchange()
             hy.copy_(y, non_blocking=True)
             hdx.copy_(dx, non_blocking=True)
             hdth.copy_(layer.dtheta, non_blocking=True)
@@ -495,6 +507,41 @@ def run_poetx(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps}
 
+    # outer-loop merge (once per inner loop, not part of the step): device time per call
+    outer = None
+    if s.dtype == "bf16":
+        pP2, _ = P.make_perm(inp.seed_P + 1000003, s.n)
+        pR2, _ = P.make_perm(inp.seed_R + 1000003, s.m)
+        i32 = lambda a: torch.as_tensor(np.asarray(a, dtype=np.int32), device=dev)  # noqa: E731
+        pP2d, pR2d = i32(pP2), i32(pR2)
+        W0p_new = torch.empty_like(layer.W0p)
+        mws = torch.empty(P.outer_merge_workspace(s.m, s.n, P.POETX_BF16), dtype=torch.uint8,
+                          device=dev)
+        GP, GR = layer.G_ops()
+
+        def merge_call():
+            P.outer_merge(layer.W0p, GP, GR, s.b, layer.inv_P, layer.inv_R, pP2d, pR2d,
+                          W0p_new, mws, stream)
+
+        for _ in range(3):
+            merge_call()
+        reps = 20
+        m0 = torch.cuda.Event(enable_timing=True)
+        m1 = torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for _ in range(reps):
+            merge_call()
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        mms = m0.elapsed_time(m1) / reps
+        # algorithmic: read W0' and write W0'_new (bf16), read both G; 2 b-wide products
+        mbytes = 2 * s.m * s.n * 2 + (s.n + s.m) * s.b * 2
+        outer = {"ms": mms, "achieved_gbs": mbytes / (mms / 1e3) / 1e9,
+                 "achieved_tflops": 4.0 * s.m * s.n * s.b / (mms / 1e3) / 1e12,
+                 "launches": 5}
+        if P.device_status(stream) != P.POETX_OK:
+            raise RuntimeError("device status not OK after the outer merge")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_throughput(s, args.oracle_budget)
@@ -510,7 +557,7 @@ def run_poetx(args):
                    "l2": f"inputs rotate over {nsets} sets of x and dy "
                          f"({nsets * (s.T * (s.n + s.m) * (2 if s.dtype == 'bf16' else 4)) >> 20} MB"
                          f" > 126 MB L2)",
-                   "parallelism": "replicas" if world > 1 else "single",
+                   "parallelism": f"dp{world}" if world > 1 else "single",
                    "launch": "cuda_graph" if graphs else "eager",
                    "roofline_timing": ("eager steps after the timed region" if graphs
                                        else "inside the timed region")},
@@ -520,6 +567,7 @@ def run_poetx(args):
         "roofline": roof,
         "cpu_baseline": cpu,
         "kernels": breakdown,
+        "outer_merge": outer,
         "cnp_blocks_per_s": world * nblk * args.steps / (max_ms / 1e3),
     }
     if rank == 0:

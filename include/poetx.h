@@ -103,6 +103,34 @@ int poetx_merge_perm(const void* W0, void* W0p, int32_t m, int32_t n, const int3
                      const int32_t* perm_P, int dtype, void* stream);
 
 /*
+ * Outer-loop merge and re-initialisation.  The original POET step W <- R_i W P_i (POET-X
+ * technical summary section 2.1, the weight-centric update that the input-centric layer
+ * replaces inside an inner loop) folds the rotations of a finished inner loop into the
+ * frozen weight; the next inner loop starts from theta = 0 under fresh permutations:
+ *   M = G_R W0' G_P                 two batched block-diagonal products (block i of G_R
+ *                                   acts on rows [ib, (i+1)b), block j of G_P on columns)
+ *   W0p_new[i, j] = M[inv_R[perm_R_new[i]], inv_P[perm_P_new[j]]]
+ * i.e. W0p_new = Pi_R' (R W0 P) Pi_P'^T with R = Pi_R^T G_R Pi_R, P = Pi_P^T G_P Pi_P.
+ * The caller sets theta to zero afterwards (G = I); this call does not touch theta.
+ *   W0p        device [m, n] (dtype): merged weight of the current permutations, read.
+ *   G_P, G_R   device [n/b, b, b], [m/b, b, b] (dtype: the bf16 copies for POETX_BF16,
+ *              fp32 for POETX_F32), read.
+ *   inv_P, inv_R           device int32 [n], [m]: inverses of the current permutations.
+ *   perm_P_new, perm_R_new device int32 [n], [m]: the next permutations.
+ *   W0p_new    device [m, n] (dtype), written; must not alias W0p.
+ *   ws         device scratch of poetx_outer_merge_workspace(m, n, dtype) bytes.
+ * bf16: tcgen05 products with fp32 accumulation; G_R W0' and M are rounded to bf16 (as
+ * the layer's activations are).  fp32: SIMT fp32 products.
+ * Shapes: m % b == 0, n % b == 0; bf16 also needs b % 128 == 0.  All pointers 16-byte
+ * aligned.  Errors: INVALID_ARG, SHAPE, DTYPE, ALIGN, WORKSPACE, CUDA.
+ */
+size_t poetx_outer_merge_workspace(int32_t m, int32_t n, int dtype);
+int poetx_outer_merge(const void* W0p, const void* G_P, const void* G_R, int32_t m, int32_t n,
+                      int32_t b, const int32_t* inv_P, const int32_t* inv_R,
+                      const int32_t* perm_P_new, const int32_t* perm_R_new, void* W0p_new,
+                      int dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Index-map permutation of the columns of a row-major matrix (POET-X section 2.2,
  * permutation acceleration): out[t, i] = in[t, idx[i]] for t < rows, i < cols.
  * With idx = perm this applies Pi to every row; with idx = inv it applies Pi^T.

@@ -430,7 +430,25 @@ cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
   return cudaGetLastError();
 }
 
+__global__ void k_compose_perm(const int32_t* __restrict__ outer, const int32_t* __restrict__ inner,
+                               int32_t* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const int j = min(max(inner[i], 0), n - 1);
+    out[i] = outer[j];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_compose_perm(const int32_t* outer, const int32_t* inner, int32_t* out, int n,
+                                cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  begin_launch("permute", s);
+  k_compose_perm<<<(n + 255) / 256, 256, 0, s>>>(outer, inner, out, n);
+  end_launch("permute", s);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gather(const void* in, void* out, const int32_t* row_idx,
                           const int32_t* col_idx, int rows, int cols, int64_t ld_in,

@@ -979,6 +979,69 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
   return POETX_OK;
 }
 
+size_t poetx_outer_merge_workspace(int32_t m, int32_t n, int dtype) {
+  if (m <= 0 || n <= 0 || (dtype != POETX_F32 && dtype != POETX_BF16)) return 0;
+  const size_t es = dtype == POETX_BF16 ? 2 : 4;
+  return 2 * align_up((size_t)m * n * es) + align_up((size_t)m * 4) + align_up((size_t)n * 4);
+}
+
+int poetx_outer_merge(const void* W0p, const void* G_P, const void* G_R, int32_t m, int32_t n,
+                      int32_t b, const int32_t* inv_P, const int32_t* inv_R,
+                      const int32_t* perm_P_new, const int32_t* perm_R_new, void* W0p_new,
+                      int dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m <= 0 || n <= 0 || b <= 0) return fail(POETX_ERR_INVALID_ARG, "sizes must be positive");
+  if (m % b != 0 || n % b != 0) return fail(POETX_ERR_SHAPE, "m and n must be multiples of b");
+  if (dtype == POETX_BF16 && b % 128 != 0)
+    return fail(POETX_ERR_SHAPE, "bf16 outer merge needs b % 128 == 0");
+  if (!W0p || !G_P || !G_R || !inv_P || !inv_R || !perm_P_new || !perm_R_new || !W0p_new || !ws)
+    return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (W0p == W0p_new) return fail(POETX_ERR_INVALID_ARG, "W0p and W0p_new must be distinct");
+  for (const void* q : {W0p, G_P, G_R, (const void*)inv_P, (const void*)inv_R,
+                        (const void*)perm_P_new, (const void*)perm_R_new, (const void*)W0p_new,
+                        (const void*)ws})
+    if (!aligned16(q)) return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  if (ws_bytes < poetx_outer_merge_workspace(m, n, dtype))
+    return fail(POETX_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t es = dtype == POETX_BF16 ? 2 : 4;
+  Carve cv(ws);
+  void* M1 = cv.take((size_t)m * n * es);
+  void* M = cv.take((size_t)m * n * es);
+  int32_t* rmap = static_cast<int32_t*>(cv.take((size_t)m * 4));
+  int32_t* cmap = static_cast<int32_t*>(cv.take((size_t)n * 4));
+  // index maps of the re-merge: W0p_new[i, j] = M[inv_R[perm_R_new[i]], inv_P[perm_P_new[j]]]
+  POETX_CUDA(launch_compose_perm(inv_R, perm_R_new, rmap, m, s), "outer merge row map");
+  POETX_CUDA(launch_compose_perm(inv_P, perm_P_new, cmap, n, s), "outer merge column map");
+  const int nR = m / b;
+  if (dtype == POETX_BF16) {
+    // M1 rows of block i = G_R,i W0'[rows of block i]: D = A B^T with A[r][k] = G_R,i[r][k]
+    // (K-major) and B[c][k] = W0'[ib + k][c] (MN-major)
+    UmmaGemm g;
+    g.A.ptr = G_R; g.A.rows = (int64_t)nR * b; g.A.cols = b; g.A.ld = b;
+    g.A.mn_major = 0; g.A.boff_mn = b;
+    g.B.ptr = W0p; g.B.rows = m; g.B.cols = n; g.B.ld = n;
+    g.B.mn_major = 1; g.B.boff_k = b;
+    g.M = b; g.N = n; g.K = b; g.batch = nR;
+    g.D = M1; g.out_f32 = 0; g.ldd = n; g.d_boff = (int64_t)b * n;
+    POETX_CUDA(launch_umma_gemm(g, "gemm_blockdiag", s), "outer merge G_R W0'");
+    // M[:, block j] = M1[:, block j] G_P,j
+    POETX_CUDA(bf16_blockdiag(M1, G_P, M, m, n, b, true, s), "outer merge M1 G_P");
+  } else {
+    SgemmArgs g;
+    g.A = static_cast<const float*>(G_R); g.lda = b; g.sA = (int64_t)b * b;
+    g.B = static_cast<const float*>(W0p); g.ldb = n; g.sB = (int64_t)b * n;
+    g.C = static_cast<float*>(M1); g.ldc = n; g.sC = (int64_t)b * n;
+    g.M = b; g.N = n; g.K = b; g.batch = nR;
+    POETX_CUDA(launch_sgemm(g, s), "outer merge G_R W0'");
+    POETX_CUDA(f32_blockdiag(static_cast<const float*>(M1), static_cast<const float*>(G_P),
+                             static_cast<float*>(M), m, n, b, false, s),
+               "outer merge M1 G_P");
+  }
+  POETX_CUDA(launch_gather(M, W0p_new, rmap, cmap, m, n, n, n, (int)es, s), "outer merge gather");
+  return POETX_OK;
+}
+
 int poetx_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");

@@ -33,6 +33,9 @@ int num_sms();
 cudaError_t launch_gather(const void* in, void* out, const int32_t* row_idx,
                           const int32_t* col_idx, int rows, int cols, int64_t ld_in,
                           int64_t ld_out, int elem_bytes, cudaStream_t s);
+// out[i] = outer[inner[i]] for i < n (composition of two index maps; indices clamped)
+cudaError_t launch_compose_perm(const int32_t* outer, const int32_t* inner, int32_t* out, int n,
+                                cudaStream_t s);
 
 // ---- fp32 SIMT batched GEMM (kernels_sgemm.cu) -----------------------------------
 enum SgemmMode { SG_FULL = 0, SG_SYM = 1, SG_SYMSKEW = 2 };

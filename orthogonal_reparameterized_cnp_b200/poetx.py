@@ -48,6 +48,9 @@ SIGNATURES = {
     "poetx_make_perm": (_c_int, [_c_u64, _c_i32, _i32p, _i32p]),
     "poetx_merge_perm": (_c_int, [_vp, _vp, _c_i32, _c_i32, _vp, _vp, _c_int, _vp]),
     "poetx_permute_cols": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
+    "poetx_outer_merge_workspace": (_c_size, [_c_i32, _c_i32, _c_int]),
+    "poetx_outer_merge": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _vp, _vp, _vp,
+                                   _vp, _c_int, _vp, _c_size, _vp]),
     "poetx_cnp_workspace": (_c_size, [_c_i32, _c_i32, _c_i32]),
     "poetx_cnp_fwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
     "poetx_cnp_bwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
@@ -185,6 +188,22 @@ def merge_perm(W0, W0p, perm_R, perm_P, stream=None):
     m, n = W0.shape
     _check(_load().poetx_merge_perm(_ptr(W0), _ptr(W0p), m, n, _ptr(perm_R), _ptr(perm_P),
                                     _dtype_code(W0), _stream(stream)), "poetx_merge_perm")
+
+
+def outer_merge_workspace(m: int, n: int, dtype_code: int) -> int:
+    return int(_load().poetx_outer_merge_workspace(m, n, dtype_code))
+
+
+def outer_merge(W0p, G_P, G_R, b: int, inv_P, inv_R, perm_P_new, perm_R_new, W0p_new, ws,
+                stream=None):
+    """W0p_new = merged weight, under the new permutations, of R W0 P (see the header)."""
+    _require_cuda()
+    m, n = W0p.shape
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_outer_merge(_ptr(W0p), _ptr(G_P), _ptr(G_R), m, n, b, _ptr(inv_P),
+                                     _ptr(inv_R), _ptr(perm_P_new), _ptr(perm_R_new),
+                                     _ptr(W0p_new), _dtype_code(W0p), _ptr(ws), ws_bytes,
+                                     _stream(stream)), "poetx_outer_merge")
 
 
 def permute_cols(x, out, idx, stream=None):

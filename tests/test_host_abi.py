@@ -122,6 +122,27 @@ def test_linear_workspace_queries():
     assert P.linear_bwd_workspace(d, False, False) > P.linear_bwd_workspace(d, True, True)
 
 
+def test_outer_merge_validation_before_launch():
+    lib = P.lib()
+    f = ctypes.c_void_p(0x50000)
+    big = 1 << 40
+
+    def call(m=512, n=256, b=128, dtype=P.POETX_BF16, w=f, out=ctypes.c_void_p(0x60000),
+             ws_bytes=big):
+        return lib.poetx_outer_merge(w, f, f, m, n, b, f, f, f, f, out, dtype, f, ws_bytes, None)
+
+    assert call(m=500) == P.POETX_ERR_SHAPE                 # m % b
+    assert call(b=64) == P.POETX_ERR_SHAPE                  # bf16 needs b % 128 == 0
+    assert call(b=0) == P.POETX_ERR_INVALID_ARG
+    assert call(dtype=9) == P.POETX_ERR_DTYPE
+    assert call(w=None) == P.POETX_ERR_INVALID_ARG
+    assert call(out=f) == P.POETX_ERR_INVALID_ARG           # output aliases the input
+    assert call(w=ctypes.c_void_p(0x50008)) == P.POETX_ERR_ALIGN
+    assert call(ws_bytes=1024) == P.POETX_ERR_WORKSPACE
+    assert P.outer_merge_workspace(2048, 2048, P.POETX_BF16) >= 2 * 2048 * 2048 * 2
+    assert P.outer_merge_workspace(0, 2048, P.POETX_BF16) == 0
+
+
 def test_profile_and_launch_counter_without_launches():
     n0 = P.launch_count()
     assert P.launch_count() == n0
