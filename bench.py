@@ -144,7 +144,8 @@ def family_work(s, ksplit_R=1, ksplit_P=1):
     d = (k + 1) // 2
     cnp_fwd = (d + 1) * b ** 3                        # d symmetric powers + G (half products)
     y_terms = 0 if d == 1 else (2 * b ** 3 + (d - 2) * 3 * b ** 3)
-    cnp_bwd = d * b ** 3 + 2 * b ** 3 + y_terms + 4 * b ** 3
+    # the backward reads S and F' kept by the forward: D, the Horner terms, A
+    cnp_bwd = 2 * b ** 3 + y_terms + 4 * b ** 3
     return {
         "gemm_w0": {"bound": "tensor", "flops": 2 * (2.0 * T * n * m), "launches": 2},
         "gemm_blockdiag": {"bound": "hbm", "launches": 4,

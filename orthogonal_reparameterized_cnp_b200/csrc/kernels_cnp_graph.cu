@@ -64,7 +64,15 @@ __device__ __forceinline__ float4 ldcg4(const float* p) {
   return __ldcg(reinterpret_cast<const float4*>(p));
 }
 __device__ __forceinline__ void st4(float* p, float a, float b, float c, float d) {
-  *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+  __stcg(reinterpret_cast<float4*>(p), make_float4(a, b, c, d));
+}
+__device__ __forceinline__ unsigned short bf16_bits(float x) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const unsigned short*>(&h);
+}
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 __device__ __forceinline__ unsigned long long gtimer() {
   unsigned long long t;
@@ -218,140 +226,147 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   __syncthreads();
   // epilogue: thread owns row il and 8 consecutive columns of the tile
   // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
-  float* C = J.C + boff;
-  __nv_bfloat16* Cb = J.Cb ? J.Cb + boff : nullptr;
-  float* C2 = J.C2 ? J.C2 + boff : nullptr;
-  const bool structured = J.mode != SG_FULL;
+  // The job's scalars are read into registers before the first store, and every store is
+  // an explicit global-space store, so no store can be taken to overwrite shared memory.
+  float* const C = J.C + boff;
+  __nv_bfloat16* const Cb = J.Cb ? J.Cb + boff : nullptr;
+  float* const C2 = J.C2 ? J.C2 + boff : nullptr;
+  const int mode = J.mode;
+  const bool structured = mode != SG_FULL;
+  const float alpha = J.alpha, diag = J.diag, diag2 = J.diag2, alpha_c2 = J.alpha_c2;
+  const float skew_c = J.skew_c;
+  const int nadd = J.nadd;
+  const bool has_skew = J.skew_add != nullptr;
+  float addc[kEpiTiles], addc2[kEpiTiles];
+#pragma unroll
+  for (int q = 0; q < kEpiTiles; ++q) {
+    addc[q] = q < nadd ? J.addc[q] : 0.f;
+    addc2[q] = q < nadd ? J.addc2[q] : 0.f;
+  }
   float (*Ms)[65] = reinterpret_cast<float (*)[65]>(smem + kRedFloats);
   float (*Ms2)[65] = reinterpret_cast<float (*)[65]>(smem + kRedFloats + 64 * 65);
+#pragma unroll 1
   for (int pass = 0; pass < 64 * 64 / (8 * kThreads); ++pass) {
-  const int il = pass * (kThreads / 8) + (tid >> 3), jl0 = (tid & 7) * 8;
-  const int i = m0 + il, j0 = n0 + jl0;
-  const int64_t row = (int64_t)i * b;
-  float a[8];
-  {
-    const float* r0 = red + il * 64 + jl0;
-    const float4 p0 = *reinterpret_cast<const float4*>(r0);
-    const float4 p1 = *reinterpret_cast<const float4*>(r0 + 4);
-    a[0] = p0.x; a[1] = p0.y; a[2] = p0.z; a[3] = p0.w;
-    a[4] = p1.x; a[5] = p1.y; a[6] = p1.z; a[7] = p1.w;
+    const int il = pass * (kThreads / 8) + (tid >> 3), jl0 = (tid & 7) * 8;
+    const int i = m0 + il, j0 = n0 + jl0;
+    const int64_t row = (int64_t)i * b;
+    float a[8];
+    {
+      const float* r0 = red + il * 64 + jl0;
+      const float4 p0 = *reinterpret_cast<const float4*>(r0);
+      const float4 p1 = *reinterpret_cast<const float4*>(r0 + 4);
+      a[0] = p0.x; a[1] = p0.y; a[2] = p0.z; a[3] = p0.w;
+      a[4] = p1.x; a[5] = p1.y; a[6] = p1.z; a[7] = p1.w;
 #pragma unroll
-    for (int g2 = 1; g2 < kGroups; ++g2) {  // fixed summation order
-      const float* rg = r0 + g2 * 64 * 64;
-      const float4 q0 = *reinterpret_cast<const float4*>(rg);
-      const float4 q1 = *reinterpret_cast<const float4*>(rg + 4);
-      a[0] += q0.x; a[1] += q0.y; a[2] += q0.z; a[3] += q0.w;
-      a[4] += q1.x; a[5] += q1.y; a[6] += q1.z; a[7] += q1.w;
+      for (int g2 = 1; g2 < kGroups; ++g2) {  // fixed summation order
+        const float* rg = r0 + g2 * 64 * 64;
+        const float4 q0 = *reinterpret_cast<const float4*>(rg);
+        const float4 q1 = *reinterpret_cast<const float4*>(rg + 4);
+        a[0] += q0.x; a[1] += q0.y; a[2] += q0.z; a[3] += q0.w;
+        a[4] += q1.x; a[5] += q1.y; a[6] += q1.z; a[7] += q1.w;
+      }
     }
-  }
-  float sym[8], sym2[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const bool dg = (i == j0 + c);
-    sym[c] = dg ? J.diag : 0.f;
-    sym2[c] = dg ? J.diag2 : 0.f;
-  }
-  const float* E = smem + kRingFloats + il * kELD + jl0;
-  for (int q = 0; q < J.nadd; ++q) {
-    const float4 x0 = *reinterpret_cast<const float4*>(E + q * 64 * kELD);
-    const float4 x1 = *reinterpret_cast<const float4*>(E + q * 64 * kELD + 4);
-    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float sym[8], sym2[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      sym[c] += J.addc[q] * xs[c];
-      sym2[c] += J.addc2[q] * xs[c];
+      const bool dg = (i == j0 + c);
+      sym[c] = dg ? diag : 0.f;
+      sym2[c] = dg ? diag2 : 0.f;
     }
-  }
-  float skew[8];
+    const float* E = smem + kRingFloats + il * kELD + jl0;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) skew[c] = J.alpha * a[c];
-  if (J.skew_add) {
-    const float4 x0 = *reinterpret_cast<const float4*>(E + J.nadd * 64 * kELD);
-    const float4 x1 = *reinterpret_cast<const float4*>(E + J.nadd * 64 * kELD + 4);
-    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    for (int q = 0; q < kEpiTiles; ++q) {
+      if (q >= nadd) break;
+      const float4 x0 = *reinterpret_cast<const float4*>(E + q * 64 * kELD);
+      const float4 x1 = *reinterpret_cast<const float4*>(E + q * 64 * kELD + 4);
+      const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) skew[c] += J.skew_c * xs[c];
-  }
-  float v[8], vm[8], v2[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const int j = j0 + c;
-    if (J.mode == SG_SYMSKEW) {
-      v[c] = (i == j) ? sym[c] : sym[c] + skew[c];
-      vm[c] = sym[c] - skew[c];
-    } else {
-      v[c] = skew[c] + sym[c];
-      vm[c] = v[c];
+      for (int c = 0; c < 8; ++c) {
+        sym[c] += addc[q] * xs[c];
+        sym2[c] += addc2[q] * xs[c];
+      }
     }
-    v2[c] = J.alpha_c2 * a[c] + sym2[c];
-  }
-  if (structured && I == Jt) {  // diagonal tile: this thread writes the upper triangle only
+    float skew[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) skew[c] = alpha * a[c];
+    if (has_skew) {
+      const float4 x0 = *reinterpret_cast<const float4*>(E + nadd * 64 * kELD);
+      const float4 x1 = *reinterpret_cast<const float4*>(E + nadd * 64 * kELD + 4);
+      const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) skew[c] += skew_c * xs[c];
+    }
+    float v[8], vm[8], v2[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const int j = j0 + c;
-      if (i <= j) {
-        C[row + j] = v[c];
-        if (Cb) Cb[row + j] = __float2bfloat16_rn(v[c]);
-        if (C2) C2[row + j] = v2[c];
+      if (mode == SG_SYMSKEW) {
+        v[c] = (i == j) ? sym[c] : sym[c] + skew[c];
+        vm[c] = sym[c] - skew[c];
+      } else {
+        v[c] = skew[c] + sym[c];
+        vm[c] = v[c];
+      }
+      v2[c] = alpha_c2 * a[c] + sym2[c];
+    }
+    if (structured) {  // mirror staging first: shared-memory work before the stores
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        Ms[il][jl0 + c] = vm[c];
+        if (C2) Ms2[il][jl0 + c] = v2[c];
       }
     }
-  } else {
-    *reinterpret_cast<float4*>(C + row + j0) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(C + row + j0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    if (Cb) {
-      uint4 o;
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
-      __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
-      o.x = *reinterpret_cast<uint32_t*>(&h0);
-      o.y = *reinterpret_cast<uint32_t*>(&h1);
-      o.z = *reinterpret_cast<uint32_t*>(&h2);
-      o.w = *reinterpret_cast<uint32_t*>(&h3);
-      *reinterpret_cast<uint4*>(Cb + row + j0) = o;
-    }
-    if (C2) {
-      *reinterpret_cast<float4*>(C2 + row + j0) = make_float4(v2[0], v2[1], v2[2], v2[3]);
-      *reinterpret_cast<float4*>(C2 + row + j0 + 4) = make_float4(v2[4], v2[5], v2[6], v2[7]);
-    }
-  }
-  if (structured) {
+    if (structured && I == Jt) {  // diagonal tile: this thread writes the upper triangle only
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      Ms[il][jl0 + c] = vm[c];
-      if (C2) Ms2[il][jl0 + c] = v2[c];
+      for (int c = 0; c < 8; ++c) {
+        const int j = j0 + c;
+        if (i <= j) {
+          __stcg(C + row + j, v[c]);
+          if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + j), bf16_bits(v[c]));
+          if (C2) __stcg(C2 + row + j, v2[c]);
+        }
+      }
+    } else {
+      __stcg(reinterpret_cast<float4*>(C + row + j0), make_float4(v[0], v[1], v[2], v[3]));
+      __stcg(reinterpret_cast<float4*>(C + row + j0 + 4), make_float4(v[4], v[5], v[6], v[7]));
+      if (Cb) {
+        const uint4 o = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
+                                   bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
+        __stcg(reinterpret_cast<uint4*>(Cb + row + j0), o);
+      }
+      if (C2) {
+        __stcg(reinterpret_cast<float4*>(C2 + row + j0), make_float4(v2[0], v2[1], v2[2], v2[3]));
+        __stcg(reinterpret_cast<float4*>(C2 + row + j0 + 4),
+               make_float4(v2[4], v2[5], v2[6], v2[7]));
+      }
     }
-  }
   }  // passes
   if (structured) {
     __syncthreads();  // staged mirror values of every pass are visible
     // row jl of the mirrored tile is column jl of this one; a thread writes 4 consecutive
     // elements (wide stores: the store count, not the bytes, sets the cost here)
+#pragma unroll 1
     for (int e = tid; e < 64 * 16; e += kThreads) {
       const int jl = e >> 4, il4 = (e & 15) * 4;
       const int64_t ji = (int64_t)(n0 + jl) * b + m0 + il4;
       const float4 v = make_float4(Ms[il4][jl], Ms[il4 + 1][jl], Ms[il4 + 2][jl], Ms[il4 + 3][jl]);
+      float4 v2 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (C2) v2 = make_float4(Ms2[il4][jl], Ms2[il4 + 1][jl], Ms2[il4 + 2][jl], Ms2[il4 + 3][jl]);
       if (I != Jt) {
-        *reinterpret_cast<float4*>(C + ji) = v;
-        if (Cb) {
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(v.z, v.w);
-          uint2 o;
-          o.x = *reinterpret_cast<uint32_t*>(&h0);
-          o.y = *reinterpret_cast<uint32_t*>(&h1);
-          *reinterpret_cast<uint2*>(Cb + ji) = o;
-        }
-        if (C2)
-          *reinterpret_cast<float4*>(C2 + ji) =
-              make_float4(Ms2[il4][jl], Ms2[il4 + 1][jl], Ms2[il4 + 2][jl], Ms2[il4 + 3][jl]);
+        __stcg(reinterpret_cast<float4*>(C + ji), v);
+        if (Cb)
+          __stcg(reinterpret_cast<uint2*>(Cb + ji),
+                 make_uint2(bf16x2_bits(v.x, v.y), bf16x2_bits(v.z, v.w)));
+        if (C2) __stcg(reinterpret_cast<float4*>(C2 + ji), v2);
       } else {  // diagonal tile: the strictly lower triangle only
         const float vv[4] = {v.x, v.y, v.z, v.w};
+        const float ww[4] = {v2.x, v2.y, v2.z, v2.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (il4 + u >= jl) continue;
-          C[ji + u] = vv[u];
-          if (Cb) Cb[ji + u] = __float2bfloat16_rn(vv[u]);
-          if (C2) C2[ji + u] = Ms2[il4 + u][jl];
+          __stcg(C + ji + u, vv[u]);
+          if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + ji + u), bf16_bits(vv[u]));
+          if (C2) __stcg(C2 + ji + u, ww[u]);
         }
       }
     }
@@ -516,7 +531,7 @@ __device__ void pack_tile(const CnpJob& J, int z, int t, int b, float* smem) {
   for (int u = 0; u < kPT / kPRows; ++u) {
     const int r = ty + u * kPRows;
     const int i = I * kPT + r, j = Jt * kPT + tx;
-    if (i < j) th[tri_idx(i, j, b)] = ta[r][tx] - tb[tx][r];
+    if (i < j) __stcg(th + tri_idx(i, j, b), ta[r][tx] - tb[tx][r]);
   }
 }
 

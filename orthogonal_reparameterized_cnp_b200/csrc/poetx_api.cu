@@ -379,6 +379,7 @@ int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* F
 
 struct BwdMats {
   float *Q, *P[4], *Fp, *D, *dGt, *N[4], *Pm, *R, *R2, *T, *T2, *A;
+  bool saved = false;  // P[1] = S and Fp = F' are given (from the forward): no power jobs
 };
 
 int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdMats& M,
@@ -395,12 +396,16 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   g.job[g.njobs++] = ex;
   int idx[4] = {0, 0, 0, 0};
   // jobs are queued level by level so independent work is not stuck behind tiles that
-  // wait: S and D (both need only Q), then the higher powers, then the Horner terms
-  graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 1, 1);
+  // wait: S and D (both need only Q), then the higher powers, then the Horner terms.
+  // With S and F' saved by the forward there are no power jobs at all.
+  if (!M.saved) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 1, 1);
   // D = Q dG (the adjoint reaching F is Q^T dG = -D)
   const int jD = g.njobs;
   g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
-  if (d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
+  if (!M.saved && d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
+  // dependency bits on S and on F' (none when they are inputs)
+  const unsigned dS = M.saved ? 0u : 1u << idx[1];
+  const unsigned dF = M.saved ? 0u : 1u << idx[d];
   // N_j = e_j (dG + dG^T) - f_j (D + D^T), j = 1..d, and dG^T
   const int jN = g.njobs;
   {
@@ -424,12 +429,11 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   // Y = sum_j sum_a S^a N_j S^(j-1-a)
   const float* Y = M.N[1];
   int jY = jN;
-  const int jS = idx[1];
   const float* S = M.P[1];
   if (d >= 2) {
     // T_{d-2} = N_{d-1} + Pm + Pm^T with Pm = N_d S
     const int jPm = g.njobs;
-    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | (1u << jS));
+    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | dS);
     const int jT = g.njobs;
     CnpJob jt;
     jt.type = JOB_SYMCOMB;
@@ -448,19 +452,19 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
       // transposed Horner terms keep every A operand symmetric:
       //   Rt_1 = N_2 + S N_3,  Rt_0 = N_1 + S Rt_1,  T_0 = Rt_0 + T_1 S
       const int jR1 = g.njobs;
-      CnpJob r1 = prod_job(S, 1, M.N[3], M.R, SG_FULL, (1u << jS) | (1u << jN));
+      CnpJob r1 = prod_job(S, 1, M.N[3], M.R, SG_FULL, dS | (1u << jN));
       r1.add[0] = M.N[2];
       r1.addc[0] = 1.f;
       r1.nadd = 1;
       g.job[g.njobs++] = r1;
       const int jR0 = g.njobs;
-      CnpJob r0 = prod_job(S, 1, M.R, M.R2, SG_FULL, (1u << jS) | (1u << jN) | (1u << jR1));
+      CnpJob r0 = prod_job(S, 1, M.R, M.R2, SG_FULL, dS | (1u << jN) | (1u << jR1));
       r0.add[0] = M.N[1];
       r0.addc[0] = 1.f;
       r0.nadd = 1;
       g.job[g.njobs++] = r0;
       const int jT0 = g.njobs;
-      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jT) | (1u << jS) | (1u << jR0));
+      CnpJob t0 = prod_job(M.T, 1, S, M.T2, SG_SYM, (1u << jT) | dS | (1u << jR0));
       t0.add[0] = M.R2;
       t0.addc[0] = 1.f;
       t0.nadd = 1;
@@ -471,8 +475,7 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   }
   // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji
   const int jA = g.njobs;
-  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL,
-                       1u | (1u << jN) | (1u << idx[d]) | (1u << jY));
+  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL, 1u | (1u << jN) | dF | (1u << jY));
   ja.A2 = Y;
   ja.a2_sym = 1;
   ja.B2 = M.Q;
@@ -495,12 +498,15 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
 
 extern "C" {
 
-int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b, int32_t k,
-                  void* ws, size_t ws_bytes, void* stream) {
+// S_save / F_save (optional, both or neither): receive S = Q^2 and F' per block.
+static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* S_save, float* F_save,
+                        int32_t nblk, int32_t b, int32_t k, void* ws, size_t ws_bytes,
+                        void* stream) {
   int st = cnp_validate(theta, G, nblk, b, k);
   if (st != POETX_OK) return st;
   if (nblk == 0) return POETX_OK;
-  if (!aligned16(theta) || !aligned16(G) || (G_bf16 && !aligned16(G_bf16)))
+  if (!aligned16(theta) || !aligned16(G) || (G_bf16 && !aligned16(G_bf16)) ||
+      !aligned16(S_save) || !aligned16(F_save))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CnpPoly P = cnp_poly(k);
@@ -512,6 +518,10 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
     std::vector<float*> Pw(d + 1, nullptr);
     for (int j = 1; j <= d; ++j) Pw[j] = static_cast<float*>(cv.take(bb * 4 * nb));
     float* Fp = static_cast<float*>(cv.take(bb * 4 * nb));
+    if (S_save) {  // the saved matrices are written in place of the scratch copies
+      Pw[1] = S_save + b0 * bb;
+      Fp = F_save + b0 * bb;
+    }
     if (cnp_graph_ok(b, k)) {
       int* counters = static_cast<int*>(cv.take(kCnpCounterBytesPerBlock * nb + 4));
       __nv_bfloat16* Gb =
@@ -540,13 +550,28 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
   });
 }
 
-int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nblk, int32_t b,
-                  int32_t k, void* ws, size_t ws_bytes, void* stream) {
+int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b, int32_t k,
+                  void* ws, size_t ws_bytes, void* stream) {
+  return cnp_fwd_impl(theta, G, G_bf16, nullptr, nullptr, nblk, b, k, ws, ws_bytes, stream);
+}
+
+int poetx_cnp_fwd_save(const float* theta, float* G, void* G_bf16, float* S_save, float* F_save,
+                       int32_t nblk, int32_t b, int32_t k, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (nblk > 0 && (!S_save || !F_save)) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  return cnp_fwd_impl(theta, G, G_bf16, S_save, F_save, nblk, b, k, ws, ws_bytes, stream);
+}
+
+// S_saved / F_saved (optional, both or neither): S and F' of the forward on the same theta.
+static int cnp_bwd_impl(const float* theta, const float* dG, const float* S_saved,
+                        const float* F_saved, float* dtheta, int32_t nblk, int32_t b, int32_t k,
+                        void* ws, size_t ws_bytes, void* stream) {
   int st = cnp_validate(theta, dtheta, nblk, b, k);
   if (st != POETX_OK) return st;
   if (nblk == 0) return POETX_OK;
   if (!dG) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(theta) || !aligned16(dG) || !aligned16(dtheta))
+  if (!aligned16(theta) || !aligned16(dG) || !aligned16(dtheta) || !aligned16(S_saved) ||
+      !aligned16(F_saved))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CnpPoly P = cnp_poly(k);
@@ -569,6 +594,11 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     float* T2 = mat();
     float* A = mat();
     const float* dg = dG + b0 * bb;
+    const bool saved = S_saved != nullptr;
+    if (saved) {  // S and F' come from the forward; the backward reads nothing else of them
+      Pw[1] = const_cast<float*>(S_saved) + b0 * bb;
+      Fp = const_cast<float*>(F_saved) + b0 * bb;
+    }
     if (cnp_graph_ok(b, k)) {
       int* counters = static_cast<int*>(cv.take(kCnpCounterBytesPerBlock * nb + 4));
       BwdMats M;
@@ -579,11 +609,14 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
       }
       M.Fp = Fp; M.D = D; M.dGt = dGt; M.Pm = Pm; M.R = R; M.R2 = R2; M.T = T; M.T2 = T2;
       M.A = A;
+      M.saved = saved;
       return run_bwd_graph(theta + b0 * ntri, dg, dtheta + b0 * ntri, M, counters, P, nb, b, s);
     }
     POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
-    int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
-    if (st2 != POETX_OK) return st2;
+    if (!saved) {
+      int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
+      if (st2 != POETX_OK) return st2;
+    }
     // D = Q dG; the adjoint reaching F is Q^T dG = -D.
     {
       SgemmArgs gd = sq_gemm(Q, 0, dg, 0, D, nb, b, SG_FULL);
@@ -663,6 +696,18 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
     POETX_CUDA(launch_pack_skew(A, dtheta + b0 * ntri, nb, b, s), "cnp pack");
     return POETX_OK;
   });
+}
+
+int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nblk, int32_t b,
+                  int32_t k, void* ws, size_t ws_bytes, void* stream) {
+  return cnp_bwd_impl(theta, dG, nullptr, nullptr, dtheta, nblk, b, k, ws, ws_bytes, stream);
+}
+
+int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* S_saved,
+                        const float* F_saved, float* dtheta, int32_t nblk, int32_t b, int32_t k,
+                        void* ws, size_t ws_bytes, void* stream) {
+  if (nblk > 0 && (!S_saved || !F_saved)) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  return cnp_bwd_impl(theta, dG, S_saved, F_saved, dtheta, nblk, b, k, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
