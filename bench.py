@@ -41,9 +41,10 @@ SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 SM_MAX_MHZ = 1965.0
 
-# DRAM bytes per launch of the dominant kernel from the committed ncu capture
-# (profiles/gemm_w0_llama1b.md); None until a capture of the current kernel exists.
-MEASURED_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of a family's kernel from one ncu capture of the
+# current kernel (cold caches; mean over the family's launches in one step); families
+# without a capture of their current kernel report null.
+MEASURED_TRAFFIC = {"cnp_sgemm": (2.148e6 + 0.008e6 + 14.723e6 + 0.596e6) / 2}
 
 
 def parse_args(argv=None):
