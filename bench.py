@@ -468,38 +468,36 @@ def run_poetx(args):
             if "bytes" in ww:
                 bd["achieved_gbs"] = ww["bytes"] / (bd["ms_per_step"] / 1e3) / 1e9
 
-    # end to end through the public API with host buffers (pinned), copies timed
+    # end to end through the public API with host buffers (pinned), copies timed: every
+    # step uploads its x, dy, theta and downloads y, dx, dtheta; the host pipeline runs
+    # the uploads of the next step and the downloads of the previous one on the two copy
+    # engines while a step computes
     e2e = None
     if args.e2e_steps > 0:
+        from orthogonal_reparameterized_cnp_b200.host_pipeline import HostPipeline
         hx = [xs[i].cpu().pin_memory() for i in range(nsets)]
         hdy = [dys[i].cpu().pin_memory() for i in range(nsets)]
         hth = layer.theta.cpu().pin_memory()
         hy = torch.empty(y.shape, dtype=act).pin_memory()
         hdx = torch.empty(dx.shape, dtype=act).pin_memory()
         hdth = torch.empty(layer.dtheta.shape, dtype=torch.float32).pin_memory()
-        dxin = torch.empty_like(xs[0])
-        ddyin = torch.empty_like(dys[0])
+        pipe = HostPipeline(layer, nbuf=2, exchange=exchange if world > 1 else None)
 
         def e2e_step(i):
-            dxin.copy_(hx[i % nsets], non_blocking=True)
-            ddyin.copy_(hdy[i % nsets], non_blocking=True)
-            layer.theta.copy_(hth, non_blocking=True)
-            layer.step(dxin, ddyin, y, dx, stream)
-            exchange()
-            hy.copy_(y, non_blocking=True)
-            hdx.copy_(dx, non_blocking=True)
-            hdth.copy_(layer.dtheta, non_blocking=True)
+            pipe.submit(i, hx[i % nsets], hdy[i % nsets], hth, hy, hdx, hdth)
 
         for i in range(3):
             e2e_step(i)
+        pipe.synchronize()
         barrier()
         torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(pipe.h2d)  # every step's first operation (its upload) follows this
         for i in range(args.e2e_steps):
             e2e_step(i)
-        e1.record(stream)
+        e1.record(pipe.d2h)  # the last download is the last operation of the last step
+        pipe.synchronize()
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
         h2d = hx[0].numel() * hx[0].element_size() + hdy[0].numel() * hdy[0].element_size() + \
@@ -507,7 +505,9 @@ def run_poetx(args):
         d2h = hy.numel() * hy.element_size() + hdx.numel() * hdx.element_size() + hdth.numel() * 4
         e2e = {"value": job_tokens_per_s(world, s.T, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps}
+               "steps": args.e2e_steps, "copies": "overlapped with compute (2 buffer sets)"}
+        if P.device_status(stream) != P.POETX_OK:
+            raise RuntimeError("device status not OK after the end-to-end steps")
 
     # outer-loop merge (once per inner loop, not part of the step): device time per call
     outer = None
