@@ -220,6 +220,28 @@ def outer_merge(W0, G_P, G_R, perm_P, perm_R, perm_P_new, perm_R_new):
     return W0_new, merge_perm(W0_new, perm_R_new, perm_P_new)
 
 
+def quantize_rows_int8(W):
+    """Per-row symmetric int8 base weight (POET-XQ: training on a low-bit base model whose
+    weight is dequantised on the fly, [POET-X] technical summary 2.6).  The pages give no
+    scheme; the reading here: one fp32 scale per output channel (row), s = max|w| / 127,
+    q = round-to-nearest-even(w / s) clamped to [-127, 127]; an all-zero row has s = 0
+    and q = 0.  The rounding decides integers, so it is taken in fp32 (IEEE division,
+    as the GPU takes it).  Returns (q int8 [m, n], s float32 [m])."""
+    W32 = np.asarray(W, dtype=np.float32)
+    amax = np.max(np.abs(W32), axis=1) if W32.shape[1] else np.zeros(W32.shape[0], np.float32)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint(W32 / safe[:, None]).astype(np.float32)
+    q = np.clip(q, -127, 127)
+    q[s == 0] = 0
+    return q.astype(np.int8), s
+
+
+def dequantize_rows(q, s) -> np.ndarray:
+    """W = s[i] q[i, j] (float64)."""
+    return np.asarray(s, dtype=np.float64)[:, None] * np.asarray(q, dtype=np.float64)
+
+
 def layer_dense(x, W0, G_P, G_R, perm_P, perm_R) -> np.ndarray:
     """Rows of Y = (R W0 P x_t)^T with the four permutations as matrices and the unmerged
     W0 (the weight-centric reading; small sizes only)."""

@@ -297,6 +297,41 @@ def test_outer_merge_preserves_the_layer(n, m, b, k):
     assert not np.allclose(y2, y0, rtol=1e-6, atol=1e-6 * np.abs(y0).max())
 
 
+# ------------------------------------------------------------------ int8 base weight
+def test_int8_rows_round_trip_within_half_a_step():
+    # every element is within s/2 of its dequantised value (plus fp32 rounding of w / s),
+    # each nonzero row reaches the full code range, and codes stay in [-127, 127]
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((37, 53)) * rng.uniform(0.01, 3, (37, 1))).astype(np.float32)
+    W[5] = 0.0
+    q, s = ref.quantize_rows_int8(W)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.all(np.abs(q.astype(int)) <= 127)
+    err = np.abs(ref.dequantize_rows(q, s) - W.astype(np.float64))
+    assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 1e-5) + 1e-30)
+    nz = s > 0
+    assert np.all(np.abs(q[nz].astype(int)).max(axis=1) == 127)
+    assert s[5] == 0 and np.all(q[5] == 0)
+
+
+def test_int8_rows_exact_on_the_grid():
+    # weights that are integer multiples of a power-of-two step with max |k| = 127 come
+    # back exactly (s = step exactly, w / s exact)
+    rng = np.random.default_rng(6)
+    k = rng.integers(-127, 128, size=(9, 40))
+    k[:, 0] = 127
+    step = 2.0 ** -rng.integers(1, 12, size=(9, 1))
+    W = (k * step).astype(np.float32)
+    q, s = ref.quantize_rows_int8(W)
+    assert np.array_equal(q.astype(int), k)
+    assert np.array_equal(s.astype(np.float64), step[:, 0])
+    # and a planted mistake (truncation instead of rounding) breaks the half-step bound
+    Wr = rng.standard_normal((8, 64)).astype(np.float32)
+    q2, s2 = ref.quantize_rows_int8(Wr)
+    trunc = np.trunc(Wr / s2[:, None])
+    assert not np.array_equal(trunc, q2.astype(np.float32))
+
+
 @pytest.mark.parametrize("k", [2, 4])
 def test_spectrum_bounds_with_cnp(k):
     # P6 with the truncated G: each factor has singular values in [1-eps, 1+eps],
