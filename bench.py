@@ -544,6 +544,39 @@ def run_poetx(args):
         if P.device_status(stream) != P.POETX_OK:
             raise RuntimeError("device status not OK after the outer merge")
 
+    # the same step with the int8 merged weight (POET-XQ reading), CUDA-graph replay
+    xq = None
+    if s.dtype == "bf16" and args.graph:
+        lq = P.PoetxLinear(to(inp.W0, act), to(inp.theta_P, torch.float32),
+                           to(inp.theta_R, torch.float32), pP, pR, s.b, s.k, s.T,
+                           int8_weight=True)
+        for i in range(3):
+            lq.step(xs[i % nsets], dys[i % nsets], y, dx, stream)
+        torch.cuda.synchronize(dev)
+        gq = []
+        for i in range(nsets):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                lq.step(xs[i], dys[i], y, dx, torch.cuda.current_stream(dev))
+            gq.append(gr)
+        for i in range(3):
+            gq[i % nsets].replay()
+        nq = min(args.steps, 500)
+        q0 = torch.cuda.Event(enable_timing=True)
+        q1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        q0.record(stream)
+        for i in range(nq):
+            gq[i % nsets].replay()
+        q1.record(stream)
+        torch.cuda.synchronize(dev)
+        if P.device_status(stream) != P.POETX_OK:
+            raise RuntimeError("device status not OK after the int8-weight steps")
+        qms = q0.elapsed_time(q1) / nq
+        xq = {"ms_per_step": qms, "tokens_per_s": s.T / (qms / 1e3), "steps": nq,
+              "weight": "int8 W0' (per-row scales), dequantised into scratch per call"}
+        del gq
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_throughput(s, args.oracle_budget)
@@ -570,6 +603,7 @@ def run_poetx(args):
         "cpu_baseline": cpu,
         "kernels": breakdown,
         "outer_merge": outer,
+        "int8_weight_step": xq,
         "cnp_blocks_per_s": world * nblk * args.steps / (max_ms / 1e3),
     }
     if rank == 0:

@@ -269,6 +269,40 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
                      size_t ws_bytes, void* stream);
 
 /*
+ * Int8 base weight (POET-X technical summary section 2.6, POET-XQ: training on a low-bit
+ * base model, whose weight is dequantised on the fly only where it is needed and never
+ * stored in high precision).  The pages give no scheme; here one fp32 scale per output
+ * channel (row of W0'):
+ *   scales[i] = max_j |W[i, j]| / 127,   q[i, j] = round_to_nearest_even(W[i, j] / scales[i])
+ * clamped to [-127, 127] (an all-zero row: scale 0, codes 0).  Scale and codes are decided
+ * in fp32 with IEEE division, so they are reproducible bit for bit.
+ *   W       device [m, n] (dtype POETX_BF16 or POETX_F32), read.
+ *   q       device int8 [m, n], written.     scales  device fp32 [m], written.
+ *   Errors: INVALID_ARG, DTYPE, ALIGN, CUDA.
+ */
+int poetx_quantize_rows(const void* W, int8_t* q, float* scales, int32_t m, int32_t n, int dtype,
+                        void* stream);
+
+/*
+ * The bf16 layer with the int8 merged weight (codes and scales from poetx_quantize_rows
+ * of W0').  Each call first writes bf16(scales[i] * q[i, j]) into the first
+ * poetx_linear_q8_scratch(d) bytes of ws (for that call only), then runs
+ * poetx_linear_fwd / poetx_linear_bwd with it; the rest of ws is their scratch, so ws_bytes
+ * must be at least poetx_linear_q8_scratch(d) + poetx_linear_{fwd,bwd}_workspace(d, ...).
+ *   W0q device int8 [m, n], scales device fp32 [m]: read.  Other arguments as the bf16
+ *   entry points.  d->dtype must be POETX_BF16 (else DTYPE).
+ *   Errors: as poetx_linear_fwd / poetx_linear_bwd.
+ */
+size_t poetx_linear_q8_scratch(const poetx_linear_desc* d);
+int poetx_linear_fwd_q8(const poetx_linear_desc* d, const void* x, const void* G_P,
+                        const void* G_R, const int8_t* W0q, const float* scales, void* y,
+                        void* save_u, void* save_w, void* ws, size_t ws_bytes, void* stream);
+int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* dy,
+                        const void* G_P, const void* G_R, const int8_t* W0q, const float* scales,
+                        const void* save_u, const void* save_w, void* dx, float* dG_P,
+                        float* dG_R, int accumulate, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Reads and clears the device-side error flag that kernels with bounded barrier waits
  * set on a timeout.  Synchronises the given stream first.  Returns POETX_OK or
  * POETX_ERR_TIMEOUT (or POETX_ERR_CUDA if the synchronisation itself failed).

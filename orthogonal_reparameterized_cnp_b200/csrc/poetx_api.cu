@@ -1087,6 +1087,64 @@ int poetx_outer_merge(const void* W0p, const void* G_P, const void* G_R, int32_t
   return POETX_OK;
 }
 
+int poetx_quantize_rows(const void* W, int8_t* q, float* scales, int32_t m, int32_t n, int dtype,
+                        void* stream) {
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m < 0 || n < 0) return fail(POETX_ERR_INVALID_ARG, "negative size");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!W || !q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(q) || !aligned16(scales))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  POETX_CUDA(launch_quantize_rows(W, q, scales, m, n, dtype == POETX_BF16 ? 2 : 4,
+                                  static_cast<cudaStream_t>(stream)),
+             "quantize rows");
+  return POETX_OK;
+}
+
+size_t poetx_linear_q8_scratch(const poetx_linear_desc* d) {
+  if (!d || d->dtype != POETX_BF16 || d->m <= 0 || d->n <= 0) return 0;
+  return align_up((size_t)d->m * d->n * 2);
+}
+
+int poetx_linear_fwd_q8(const poetx_linear_desc* d, const void* x, const void* G_P,
+                        const void* G_R, const int8_t* W0q, const float* scales, void* y,
+                        void* save_u, void* save_w, void* ws, size_t ws_bytes, void* stream) {
+  int st = linear_validate(d);
+  if (st != POETX_OK) return st;
+  if (d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "int8 base weight needs bf16");
+  if (d->T == 0) return POETX_OK;
+  if (!W0q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W0q) || !aligned16(scales) || !aligned16(ws))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const size_t q8 = poetx_linear_q8_scratch(d);
+  if (!ws || ws_bytes < q8) return fail(POETX_ERR_WORKSPACE, "scratch too small");
+  // the dequantised weight lives in the first part of the scratch for this call only
+  POETX_CUDA(launch_dequant_rows(W0q, scales, ws, d->m, d->n, static_cast<cudaStream_t>(stream)),
+             "dequantise W0'");
+  return poetx_linear_fwd(d, x, G_P, G_R, ws, y, save_u, save_w,
+                          static_cast<char*>(ws) + q8, ws_bytes - q8, stream);
+}
+
+int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* dy,
+                        const void* G_P, const void* G_R, const int8_t* W0q, const float* scales,
+                        const void* save_u, const void* save_w, void* dx, float* dG_P,
+                        float* dG_R, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+  int st = linear_validate(d);
+  if (st != POETX_OK) return st;
+  if (d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "int8 base weight needs bf16");
+  if (!W0q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W0q) || !aligned16(scales) || !aligned16(ws))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const size_t q8 = poetx_linear_q8_scratch(d);
+  if (!ws || ws_bytes < q8) return fail(POETX_ERR_WORKSPACE, "scratch too small");
+  if (d->T > 0)
+    POETX_CUDA(launch_dequant_rows(W0q, scales, ws, d->m, d->n,
+                                   static_cast<cudaStream_t>(stream)),
+               "dequantise W0'");
+  return poetx_linear_bwd(d, x, dy, G_P, G_R, ws, save_u, save_w, dx, dG_P, dG_R, accumulate,
+                          static_cast<char*>(ws) + q8, ws_bytes - q8, stream);
+}
+
 int poetx_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");

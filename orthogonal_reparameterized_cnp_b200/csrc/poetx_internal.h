@@ -37,6 +37,14 @@ cudaError_t launch_gather(const void* in, void* out, const int32_t* row_idx,
 cudaError_t launch_compose_perm(const int32_t* outer, const int32_t* inner, int32_t* out, int n,
                                 cudaStream_t s);
 
+// ---- int8 base weight (kernels_quant.cu) -----------------------------------------
+// per-row symmetric int8: s_i = max|w_i.| / 127, q = rint(w / s) in [-127, 127]
+cudaError_t launch_quantize_rows(const void* W, int8_t* q, float* s, int m, int n,
+                                 int elem_bytes, cudaStream_t st);
+// out (bf16) = s_i * q_ij
+cudaError_t launch_dequant_rows(const int8_t* q, const float* s, void* out, int m, int n,
+                                cudaStream_t st);
+
 // ---- fp32 SIMT batched GEMM (kernels_sgemm.cu) -----------------------------------
 enum SgemmMode { SG_FULL = 0, SG_SYM = 1, SG_SYMSKEW = 2 };
 

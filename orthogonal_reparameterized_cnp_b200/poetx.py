@@ -66,6 +66,12 @@ SIGNATURES = {
     "poetx_linear_bwd": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "poetx_device_status": (_c_int, [_vp]),
+    "poetx_quantize_rows": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
+    "poetx_linear_q8_scratch": (_c_size, [ctypes.POINTER(LinearDesc)]),
+    "poetx_linear_fwd_q8": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _c_size, _vp]),
+    "poetx_linear_bwd_q8": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "poetx_launch_count": (_c_u64, []),
     "poetx_profile_begin": (_c_int, [ctypes.c_char_p]),
     "poetx_profile_end": (_c_int, [_i32p, ctypes.POINTER(ctypes.c_double)]),
@@ -280,6 +286,39 @@ def linear_bwd(desc: LinearDesc, x, dy, G_P, G_R, W0p, save_u, save_w, dx, dG_P,
                                     _stream(stream)), "poetx_linear_bwd")
 
 
+def quantize_rows(W, q, scales, stream=None):
+    """Per-row symmetric int8 codes and fp32 scales of W (see the header)."""
+    _require_cuda()
+    m, n = W.shape
+    _check(_load().poetx_quantize_rows(_ptr(W), _ptr(q), _ptr(scales), m, n, _dtype_code(W),
+                                       _stream(stream)), "poetx_quantize_rows")
+
+
+def linear_q8_scratch(desc: LinearDesc) -> int:
+    return int(_load().poetx_linear_q8_scratch(ctypes.byref(desc)))
+
+
+def linear_fwd_q8(desc: LinearDesc, x, G_P, G_R, W0q, scales, y, save_u, save_w, ws,
+                  stream=None):
+    _require_cuda()
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_linear_fwd_q8(ctypes.byref(desc), _ptr(x), _ptr(G_P), _ptr(G_R),
+                                       _ptr(W0q), _ptr(scales), _ptr(y), _ptr(save_u),
+                                       _ptr(save_w), _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_linear_fwd_q8")
+
+
+def linear_bwd_q8(desc: LinearDesc, x, dy, G_P, G_R, W0q, scales, save_u, save_w, dx, dG_P,
+                  dG_R, accumulate: int, ws, stream=None):
+    _require_cuda()
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_linear_bwd_q8(ctypes.byref(desc), _ptr(x), _ptr(dy), _ptr(G_P),
+                                       _ptr(G_R), _ptr(W0q), _ptr(scales), _ptr(save_u),
+                                       _ptr(save_w), _ptr(dx), _ptr(dG_P), _ptr(dG_R),
+                                       accumulate, _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_linear_bwd_q8")
+
+
 def device_status(stream=None) -> int:
     _require_cuda()
     return int(_load().poetx_device_status(_stream(stream)))
@@ -305,7 +344,7 @@ class PoetxLinear:
     """
 
     def __init__(self, W0, theta_P, theta_R, perm_P, perm_R, b: int, k: int, T: int,
-                 save_activations: bool = True):
+                 save_activations: bool = True, int8_weight: bool = False):
         import torch
         _require_cuda()
         dev = W0.device
@@ -349,7 +388,19 @@ class PoetxLinear:
             self.U = self.Wsave = None
         fwd_ws = linear_fwd_workspace(self.desc, self.save, self.save)
         bwd_ws = linear_bwd_workspace(self.desc, self.save, self.save)
-        self.ws = torch.empty(max(fwd_ws, bwd_ws, 16), dtype=torch.uint8, device=dev)
+        # int8 merged weight (POET-XQ): codes + per-row scales; the bf16 weight exists only
+        # inside each layer call's scratch
+        self.int8 = int8_weight
+        q8 = 0
+        if int8_weight:
+            if not self.bf16:
+                raise ValueError("the int8 base weight needs the bf16 layer")
+            self.W0q = torch.empty((self.m, self.n), dtype=torch.int8, device=dev)
+            self.scales = torch.empty((self.m,), **f32)
+            q8 = linear_q8_scratch(self.desc)
+        self.ws = torch.empty(max(fwd_ws, bwd_ws, 16) + q8, dtype=torch.uint8, device=dev)
+        if int8_weight:  # the bf16 merged weight is only a step of merge(): it lives in scratch
+            self.W0p = self.ws[: self.m * self.n * 2].view(W0.dtype).view(self.m, self.n)
 
     def G_ops(self):
         G = self.G_lp if self.bf16 else self.G
@@ -357,6 +408,8 @@ class PoetxLinear:
 
     def merge(self, stream=None):
         merge_perm(self.W0, self.W0p, self.perm_R, self.perm_P, stream)
+        if self.int8:
+            quantize_rows(self.W0p, self.W0q, self.scales, stream)
 
     def cnp_forward(self, stream=None):
         cnp_fwd_save(self.theta, self.G, self.G_lp, self.S_save, self.F_save, self.b, self.k,
@@ -364,12 +417,21 @@ class PoetxLinear:
 
     def forward(self, x, y, stream=None):
         GP, GR = self.G_ops()
-        linear_fwd(self.desc, x, GP, GR, self.W0p, y, self.U, self.Wsave, self.ws, stream)
+        if self.int8:
+            linear_fwd_q8(self.desc, x, GP, GR, self.W0q, self.scales, y, self.U, self.Wsave,
+                          self.ws, stream)
+        else:
+            linear_fwd(self.desc, x, GP, GR, self.W0p, y, self.U, self.Wsave, self.ws, stream)
 
     def backward(self, x, dy, dx, accumulate=0, stream=None):
         GP, GR = self.G_ops()
-        linear_bwd(self.desc, x, dy, GP, GR, self.W0p, self.U, self.Wsave, dx,
-                   self.dG[: self.nP], self.dG[self.nP:], accumulate, self.ws, stream)
+        if self.int8:
+            linear_bwd_q8(self.desc, x, dy, GP, GR, self.W0q, self.scales, self.U, self.Wsave,
+                          dx, self.dG[: self.nP], self.dG[self.nP:], accumulate, self.ws,
+                          stream)
+        else:
+            linear_bwd(self.desc, x, dy, GP, GR, self.W0p, self.U, self.Wsave, dx,
+                       self.dG[: self.nP], self.dG[self.nP:], accumulate, self.ws, stream)
 
     def cnp_backward(self, stream=None):
         """dtheta from dG; reads S and F' of the last cnp_forward (theta unchanged since)."""

@@ -1,0 +1,83 @@
+"""GPU parity of the int8 base weight (POET-XQ reading): codes and scales bit-exact with
+the oracle's fp32 decision, and the bf16 layer run on the int8 merged weight against the
+float64 oracle layer on the dequantised weight (normalised max error <= 2e-2)."""
+import numpy as np
+import pytest
+
+from oracle import poetx_ref as ref
+from poetx_inputs import LayerShape, layer_inputs, round_to_bf16
+
+from .gpu_harness import host, norm_max_err, tensor
+
+pytestmark = pytest.mark.gpu
+
+BF16_NORM = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    P.lib()  # fails loudly if the library is missing
+    yield
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("m,n", [(1, 16), (300, 520), (64, 2048), (7, 33)])
+def test_quantize_rows_bit_exact(dtype, m, n):
+    import torch
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    rng = np.random.default_rng(m * 31 + n)
+    W = rng.standard_normal((m, n)) * rng.uniform(1e-3, 5.0, (m, 1))
+    if m > 3:
+        W[3] = 0.0
+    W = round_to_bf16(W) if dtype == "bf16" else W.astype(np.float32).astype(np.float64)
+    Wd = tensor(W, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    q = torch.empty((m, n), dtype=torch.int8, device="cuda")
+    s = torch.empty((m,), dtype=torch.float32, device="cuda")
+    P.quantize_rows(Wd, q, s)
+    torch.cuda.synchronize()
+    q_ref, s_ref = ref.quantize_rows_int8(W)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("T,n,m,b", [(256, 512, 384, 128), (320, 512, 768, 256)])
+def test_int8_layer_matches_oracle(T, n, m, b):
+    import torch
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    s = LayerShape(f"xq-{n}x{m}-b{b}", T=T, n=n, m=m, b=b, k=4, dtype="bf16", config_id=11,
+                   std_theta=0.01)
+    inp = layer_inputs(s)
+    dev = torch.device("cuda")
+    pP, _ = P.make_perm(inp.seed_P, n)
+    pR, _ = P.make_perm(inp.seed_R, m)
+    layer = P.PoetxLinear(tensor(inp.W0, torch.bfloat16), tensor(inp.theta_P, torch.float32),
+                          tensor(inp.theta_R, torch.float32), pP, pR, b, 4, T, int8_weight=True)
+    x = tensor(inp.x, torch.bfloat16)
+    dy = tensor(inp.dy, torch.bfloat16)
+    y = torch.empty((T, m), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((T, n), dtype=torch.bfloat16, device=dev)
+    layer.step(x, dy, y, dx)
+    torch.cuda.synchronize()
+    assert P.device_status() == P.POETX_OK
+    # oracle: its own permutations, merge, quantisation and CNP; layer on s * q
+    oP, _ = ref.make_perm(inp.seed_P, n)
+    oR, _ = ref.make_perm(inp.seed_R, m)
+    W0p = ref.merge_perm(inp.W0, oR, oP)
+    q, sc = ref.quantize_rows_int8(W0p)
+    assert np.array_equal(layer.W0q.cpu().numpy(), q) and np.array_equal(layer.scales.cpu().numpy(), sc)
+    Wdq = ref.dequantize_rows(q, sc)
+    G_P, G_R = ref.cnp_forward(inp.theta_P, b, 4), ref.cnp_forward(inp.theta_R, b, 4)
+    x64, dy64 = inp.x.astype(np.float64), inp.dy.astype(np.float64)
+    Y, U, V, W = ref.layer_forward(x64, Wdq, G_P, G_R, oP, oR)
+    dX, dG_P, dG_R = ref.layer_backward(x64, dy64, Wdq, G_P, G_R, oP, oR, U=U, W=W)
+    dth = np.concatenate([ref.cnp_backward(inp.theta_P, dG_P, b, 4),
+                          ref.cnp_backward(inp.theta_R, dG_R, b, 4)])
+    errs = {"y": norm_max_err(host(y), Y), "dx": norm_max_err(host(dx), dX),
+            "dG_P": norm_max_err(host(layer.dG[: n // b]), dG_P),
+            "dG_R": norm_max_err(host(layer.dG[n // b:]), dG_R),
+            "dtheta": norm_max_err(host(layer.dtheta), dth)}
+    assert all(v <= BF16_NORM for v in errs.values()), errs

@@ -143,6 +143,28 @@ def test_outer_merge_validation_before_launch():
     assert P.outer_merge_workspace(0, 2048, P.POETX_BF16) == 0
 
 
+def test_int8_weight_validation_before_launch():
+    lib = P.lib()
+    f = ctypes.c_void_p(0x70000)
+    assert lib.poetx_quantize_rows(f, f, f, 4, 8, 9, None) == P.POETX_ERR_DTYPE
+    assert lib.poetx_quantize_rows(None, f, f, 4, 8, P.POETX_BF16, None) == \
+        P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_quantize_rows(ctypes.c_void_p(0x70004), f, f, 4, 8, P.POETX_BF16, None) == \
+        P.POETX_ERR_ALIGN
+    assert lib.poetx_quantize_rows(f, f, f, 0, 8, P.POETX_BF16, None) == P.POETX_OK
+    d32 = _desc(dtype=P.POETX_F32)
+    assert P.linear_q8_scratch(d32) == 0
+    d = _desc(T=64, n=512, m=256, b=128)
+    assert P.linear_q8_scratch(d) >= 512 * 256 * 2
+    ws = ctypes.c_void_p(0x80000)
+    assert lib.poetx_linear_fwd_q8(ctypes.byref(d32), f, f, f, f, f, f, None, None, ws, 1 << 40,
+                                   None) == P.POETX_ERR_DTYPE
+    assert lib.poetx_linear_fwd_q8(ctypes.byref(d), f, f, f, None, f, f, None, None, ws, 1 << 40,
+                                   None) == P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_linear_fwd_q8(ctypes.byref(d), f, f, f, f, f, f, None, None, ws, 16,
+                                   None) == P.POETX_ERR_WORKSPACE
+
+
 def test_profile_and_launch_counter_without_launches():
     n0 = P.launch_count()
     assert P.launch_count() == n0
