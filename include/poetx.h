@@ -195,23 +195,24 @@ int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nb
                   int32_t k, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * The same CNP pair with the forward's S = Q^2 and F' kept for the backward (POET-X
+ * The same CNP pair with the forward's Q, S = Q^2 and F' kept for the backward (POET-X
  * technical summary section 2.5 trades recomputation against memory the same way for the
  * layer's activations): with theta unchanged between the two calls, the backward reads
- * S and F' instead of recomputing Q^2, the higher powers and F', and its result is
- * bit-identical to poetx_cnp_bwd.  F' = F(S) - f_0 I, where G = E(S) + Q F(S) splits the
- * CNP polynomial into its even and odd parts in Q (f_0 = 2, the coefficient of Q).
- *   S_save, F_save    device fp32 [nblk, b, b] each, written by poetx_cnp_fwd_save.
- *   S_saved, F_saved  the same buffers, read by poetx_cnp_bwd_saved (theta unchanged).
- *   Other arguments and errors as poetx_cnp_fwd / poetx_cnp_bwd (NULL save buffers with
+ * Q, S and F' instead of expanding theta and recomputing Q^2, the higher powers and F',
+ * and its result is bit-identical to poetx_cnp_bwd.  F' = F(S) - f_0 I, where
+ * G = E(S) + Q F(S) splits the CNP polynomial into its even and odd parts in Q (f_0 = 2,
+ * the coefficient of Q).
+ *   Q_save, S_save, F_save     device fp32 [nblk, b, b] each, written by poetx_cnp_fwd_save.
+ *   Q_saved, S_saved, F_saved  the same buffers, read by poetx_cnp_bwd_saved.
+ *   Other arguments and errors as poetx_cnp_fwd / poetx_cnp_bwd (a NULL save buffer with
  *   nblk > 0: INVALID_ARG).
  */
-int poetx_cnp_fwd_save(const float* theta, float* G, void* G_bf16, float* S_save, float* F_save,
-                       int32_t nblk, int32_t b, int32_t k, void* ws, size_t ws_bytes,
-                       void* stream);
-int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* S_saved,
-                        const float* F_saved, float* dtheta, int32_t nblk, int32_t b, int32_t k,
-                        void* ws, size_t ws_bytes, void* stream);
+int poetx_cnp_fwd_save(const float* theta, float* G, void* G_bf16, float* Q_save, float* S_save,
+                       float* F_save, int32_t nblk, int32_t b, int32_t k, void* ws,
+                       size_t ws_bytes, void* stream);
+int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* Q_saved,
+                        const float* S_saved, const float* F_saved, float* dtheta, int32_t nblk,
+                        int32_t b, int32_t k, void* ws, size_t ws_bytes, void* stream);
 
 /* Shape, precision and index maps of one POET-X linear (index maps in device memory). */
 typedef struct poetx_linear_desc {

@@ -379,7 +379,7 @@ int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* F
 
 struct BwdMats {
   float *Q, *P[4], *Fp, *D, *dGt, *N[4], *Pm, *R, *R2, *T, *T2, *A;
-  bool saved = false;  // P[1] = S and Fp = F' are given (from the forward): no power jobs
+  bool saved = false;  // Q, P[1] = S and Fp = F' are given (from the forward)
 };
 
 int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdMats& M,
@@ -389,19 +389,23 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   g.nblk = nb;
   g.b = b;
   g.counters = counters;
-  CnpJob ex;
-  ex.type = JOB_EXPAND;
-  ex.A = theta;
-  ex.C = M.Q;
-  g.job[g.njobs++] = ex;
+  // with Q, S and F' saved by the forward there is no expansion and there are no power
+  // jobs; otherwise job 0 expands theta into Q
+  if (!M.saved) {
+    CnpJob ex;
+    ex.type = JOB_EXPAND;
+    ex.A = theta;
+    ex.C = M.Q;
+    g.job[g.njobs++] = ex;
+  }
+  const unsigned dQ = M.saved ? 0u : 1u;  // dependency bit on Q
   int idx[4] = {0, 0, 0, 0};
   // jobs are queued level by level so independent work is not stuck behind tiles that
   // wait: S and D (both need only Q), then the higher powers, then the Horner terms.
-  // With S and F' saved by the forward there are no power jobs at all.
   if (!M.saved) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 1, 1);
   // D = Q dG (the adjoint reaching F is Q^T dG = -D)
   const int jD = g.njobs;
-  g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, 1u);
+  g.job[g.njobs++] = prod_job(M.Q, -1, dg, M.D, SG_FULL, dQ);
   if (!M.saved && d >= 2) graph_powers(g, 0, M.Q, M.P, M.Fp, P, idx, 2, d);
   // dependency bits on S and on F' (none when they are inputs)
   const unsigned dS = M.saved ? 0u : 1u << idx[1];
@@ -475,7 +479,7 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   }
   // A = f_0 dG + dG F' - Y Q; dtheta_(i,j) = A_ij - A_ji
   const int jA = g.njobs;
-  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL, 1u | (1u << jN) | dF | (1u << jY));
+  CnpJob ja = prod_job(M.dGt, 2, M.Fp, M.A, SG_FULL, dQ | (1u << jN) | dF | (1u << jY));
   ja.A2 = Y;
   ja.a2_sym = 1;
   ja.B2 = M.Q;
@@ -498,15 +502,15 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
 
 extern "C" {
 
-// S_save / F_save (optional, both or neither): receive S = Q^2 and F' per block.
-static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* S_save, float* F_save,
-                        int32_t nblk, int32_t b, int32_t k, void* ws, size_t ws_bytes,
-                        void* stream) {
+// Q_save / S_save / F_save (optional, all or none): receive Q, S = Q^2 and F' per block.
+static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* Q_save, float* S_save,
+                        float* F_save, int32_t nblk, int32_t b, int32_t k, void* ws,
+                        size_t ws_bytes, void* stream) {
   int st = cnp_validate(theta, G, nblk, b, k);
   if (st != POETX_OK) return st;
   if (nblk == 0) return POETX_OK;
   if (!aligned16(theta) || !aligned16(G) || (G_bf16 && !aligned16(G_bf16)) ||
-      !aligned16(S_save) || !aligned16(F_save))
+      !aligned16(Q_save) || !aligned16(S_save) || !aligned16(F_save))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CnpPoly P = cnp_poly(k);
@@ -519,6 +523,7 @@ static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* S_sav
     for (int j = 1; j <= d; ++j) Pw[j] = static_cast<float*>(cv.take(bb * 4 * nb));
     float* Fp = static_cast<float*>(cv.take(bb * 4 * nb));
     if (S_save) {  // the saved matrices are written in place of the scratch copies
+      Q = Q_save + b0 * bb;
       Pw[1] = S_save + b0 * bb;
       Fp = F_save + b0 * bb;
     }
@@ -552,26 +557,30 @@ static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* S_sav
 
 int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int32_t b, int32_t k,
                   void* ws, size_t ws_bytes, void* stream) {
-  return cnp_fwd_impl(theta, G, G_bf16, nullptr, nullptr, nblk, b, k, ws, ws_bytes, stream);
+  return cnp_fwd_impl(theta, G, G_bf16, nullptr, nullptr, nullptr, nblk, b, k, ws, ws_bytes,
+                      stream);
 }
 
-int poetx_cnp_fwd_save(const float* theta, float* G, void* G_bf16, float* S_save, float* F_save,
-                       int32_t nblk, int32_t b, int32_t k, void* ws, size_t ws_bytes,
-                       void* stream) {
-  if (nblk > 0 && (!S_save || !F_save)) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  return cnp_fwd_impl(theta, G, G_bf16, S_save, F_save, nblk, b, k, ws, ws_bytes, stream);
+int poetx_cnp_fwd_save(const float* theta, float* G, void* G_bf16, float* Q_save, float* S_save,
+                       float* F_save, int32_t nblk, int32_t b, int32_t k, void* ws,
+                       size_t ws_bytes, void* stream) {
+  if (nblk > 0 && (!Q_save || !S_save || !F_save))
+    return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  return cnp_fwd_impl(theta, G, G_bf16, Q_save, S_save, F_save, nblk, b, k, ws, ws_bytes,
+                      stream);
 }
 
-// S_saved / F_saved (optional, both or neither): S and F' of the forward on the same theta.
-static int cnp_bwd_impl(const float* theta, const float* dG, const float* S_saved,
-                        const float* F_saved, float* dtheta, int32_t nblk, int32_t b, int32_t k,
-                        void* ws, size_t ws_bytes, void* stream) {
+// Q_saved / S_saved / F_saved (optional, all or none): Q, S and F' of the forward on the
+// same theta.
+static int cnp_bwd_impl(const float* theta, const float* dG, const float* Q_saved,
+                        const float* S_saved, const float* F_saved, float* dtheta, int32_t nblk,
+                        int32_t b, int32_t k, void* ws, size_t ws_bytes, void* stream) {
   int st = cnp_validate(theta, dtheta, nblk, b, k);
   if (st != POETX_OK) return st;
   if (nblk == 0) return POETX_OK;
   if (!dG) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(theta) || !aligned16(dG) || !aligned16(dtheta) || !aligned16(S_saved) ||
-      !aligned16(F_saved))
+  if (!aligned16(theta) || !aligned16(dG) || !aligned16(dtheta) || !aligned16(Q_saved) ||
+      !aligned16(S_saved) || !aligned16(F_saved))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const CnpPoly P = cnp_poly(k);
@@ -595,7 +604,8 @@ static int cnp_bwd_impl(const float* theta, const float* dG, const float* S_save
     float* A = mat();
     const float* dg = dG + b0 * bb;
     const bool saved = S_saved != nullptr;
-    if (saved) {  // S and F' come from the forward; the backward reads nothing else of them
+    if (saved) {  // Q, S and F' come from the forward (read only)
+      Q = const_cast<float*>(Q_saved) + b0 * bb;
       Pw[1] = const_cast<float*>(S_saved) + b0 * bb;
       Fp = const_cast<float*>(F_saved) + b0 * bb;
     }
@@ -612,8 +622,8 @@ static int cnp_bwd_impl(const float* theta, const float* dG, const float* S_save
       M.saved = saved;
       return run_bwd_graph(theta + b0 * ntri, dg, dtheta + b0 * ntri, M, counters, P, nb, b, s);
     }
-    POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
     if (!saved) {
+      POETX_CUDA(launch_theta_to_Q(theta + b0 * ntri, Q, nb, b, s), "cnp theta->Q");
       int st2 = cnp_powers(Q, Pw, Fp, P, nb, b, s);
       if (st2 != POETX_OK) return st2;
     }
@@ -700,14 +710,17 @@ static int cnp_bwd_impl(const float* theta, const float* dG, const float* S_save
 
 int poetx_cnp_bwd(const float* theta, const float* dG, float* dtheta, int32_t nblk, int32_t b,
                   int32_t k, void* ws, size_t ws_bytes, void* stream) {
-  return cnp_bwd_impl(theta, dG, nullptr, nullptr, dtheta, nblk, b, k, ws, ws_bytes, stream);
+  return cnp_bwd_impl(theta, dG, nullptr, nullptr, nullptr, dtheta, nblk, b, k, ws, ws_bytes,
+                      stream);
 }
 
-int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* S_saved,
-                        const float* F_saved, float* dtheta, int32_t nblk, int32_t b, int32_t k,
-                        void* ws, size_t ws_bytes, void* stream) {
-  if (nblk > 0 && (!S_saved || !F_saved)) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  return cnp_bwd_impl(theta, dG, S_saved, F_saved, dtheta, nblk, b, k, ws, ws_bytes, stream);
+int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* Q_saved,
+                        const float* S_saved, const float* F_saved, float* dtheta, int32_t nblk,
+                        int32_t b, int32_t k, void* ws, size_t ws_bytes, void* stream) {
+  if (nblk > 0 && (!Q_saved || !S_saved || !F_saved))
+    return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  return cnp_bwd_impl(theta, dG, Q_saved, S_saved, F_saved, dtheta, nblk, b, k, ws, ws_bytes,
+                      stream);
 }
 
 }  // extern "C"

@@ -55,9 +55,9 @@ SIGNATURES = {
     "poetx_cnp_fwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
     "poetx_cnp_bwd": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size, _vp]),
     "poetx_cnp_fwd_static": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp]),
-    "poetx_cnp_fwd_save": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size,
-                                    _vp]),
-    "poetx_cnp_bwd_saved": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp,
+    "poetx_cnp_fwd_save": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp,
+                                    _c_size, _vp]),
+    "poetx_cnp_bwd_saved": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_i32, _c_i32, _c_i32, _vp,
                                      _c_size, _vp]),
     "poetx_linear_fwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
     "poetx_linear_bwd_workspace": (_c_size, [ctypes.POINTER(LinearDesc), _c_int, _c_int]),
@@ -248,24 +248,25 @@ def cnp_bwd(theta, dG, dtheta, b: int, k: int, ws, stream=None):
                                  ws_bytes, _stream(stream)), "poetx_cnp_bwd")
 
 
-def cnp_fwd_save(theta, G, G_bf16, S_save, F_save, b: int, k: int, ws, stream=None):
-    """CNP forward that also keeps S = Q^2 and F' for poetx_cnp_bwd_saved."""
+def cnp_fwd_save(theta, G, G_bf16, Q_save, S_save, F_save, b: int, k: int, ws, stream=None):
+    """CNP forward that also keeps Q, S = Q^2 and F' for poetx_cnp_bwd_saved."""
     _require_cuda()
     nblk = theta.shape[0]
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _check(_load().poetx_cnp_fwd_save(_ptr(theta), _ptr(G), _ptr(G_bf16), _ptr(S_save),
-                                      _ptr(F_save), nblk, b, k, _ptr(ws), ws_bytes,
+    _check(_load().poetx_cnp_fwd_save(_ptr(theta), _ptr(G), _ptr(G_bf16), _ptr(Q_save),
+                                      _ptr(S_save), _ptr(F_save), nblk, b, k, _ptr(ws), ws_bytes,
                                       _stream(stream)), "poetx_cnp_fwd_save")
 
 
-def cnp_bwd_saved(theta, dG, S_saved, F_saved, dtheta, b: int, k: int, ws, stream=None):
-    """CNP backward reading the forward's S and F' (theta unchanged since)."""
+def cnp_bwd_saved(theta, dG, Q_saved, S_saved, F_saved, dtheta, b: int, k: int, ws,
+                  stream=None):
+    """CNP backward reading the forward's Q, S and F' (theta unchanged since)."""
     _require_cuda()
     nblk = theta.shape[0]
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _check(_load().poetx_cnp_bwd_saved(_ptr(theta), _ptr(dG), _ptr(S_saved), _ptr(F_saved),
-                                       _ptr(dtheta), nblk, b, k, _ptr(ws), ws_bytes,
-                                       _stream(stream)), "poetx_cnp_bwd_saved")
+    _check(_load().poetx_cnp_bwd_saved(_ptr(theta), _ptr(dG), _ptr(Q_saved), _ptr(S_saved),
+                                       _ptr(F_saved), _ptr(dtheta), nblk, b, k, _ptr(ws),
+                                       ws_bytes, _stream(stream)), "poetx_cnp_bwd_saved")
 
 
 def linear_fwd(desc: LinearDesc, x, G_P, G_R, W0p, y, save_u, save_w, ws, stream=None):
@@ -372,7 +373,8 @@ class PoetxLinear:
         self.G_lp = torch.empty((nblk, b, b), dtype=W0.dtype, device=dev) if self.bf16 else None
         self.dG = torch.empty((nblk, b, b), **f32)
         self.dtheta = torch.empty((nblk, ntri), **f32)
-        # S = Q^2 and F' of the last CNP forward, read by the CNP backward of the same step
+        # Q, S = Q^2 and F' of the last CNP forward, read by the CNP backward of the same step
+        self.Q_save = torch.empty((nblk, b, b), **f32)
         self.S_save = torch.empty((nblk, b, b), **f32)
         self.F_save = torch.empty((nblk, b, b), **f32)
         self.cnp_ws = torch.empty(max(cnp_workspace(nblk, b, k), 16), dtype=torch.uint8,
@@ -412,8 +414,8 @@ class PoetxLinear:
             quantize_rows(self.W0p, self.W0q, self.scales, stream)
 
     def cnp_forward(self, stream=None):
-        cnp_fwd_save(self.theta, self.G, self.G_lp, self.S_save, self.F_save, self.b, self.k,
-                     self.cnp_ws, stream)
+        cnp_fwd_save(self.theta, self.G, self.G_lp, self.Q_save, self.S_save, self.F_save,
+                     self.b, self.k, self.cnp_ws, stream)
 
     def forward(self, x, y, stream=None):
         GP, GR = self.G_ops()
@@ -434,9 +436,9 @@ class PoetxLinear:
                        self.dG[: self.nP], self.dG[self.nP:], accumulate, self.ws, stream)
 
     def cnp_backward(self, stream=None):
-        """dtheta from dG; reads S and F' of the last cnp_forward (theta unchanged since)."""
-        cnp_bwd_saved(self.theta, self.dG, self.S_save, self.F_save, self.dtheta, self.b,
-                      self.k, self.cnp_ws, stream)
+        """dtheta from dG; reads Q, S and F' of the last cnp_forward (theta unchanged)."""
+        cnp_bwd_saved(self.theta, self.dG, self.Q_save, self.S_save, self.F_save, self.dtheta,
+                      self.b, self.k, self.cnp_ws, stream)
 
     def step(self, x, dy, y, dx, stream=None):
         """One pass of the whole path: merge, CNP forward, layer forward and backward,

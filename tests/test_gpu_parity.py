@@ -116,7 +116,7 @@ def test_cnp_matches_oracle(b, k):
 
 @pytest.mark.parametrize("b,k", [(64, 6), (100, 4), (256, 4), (128, 1)])
 def test_cnp_saved_pair_is_bit_identical(b, k):
-    # the forward keeps S = Q^2 and F'; the backward that reads them must give exactly
+    # the forward keeps Q, S = Q^2 and F'; the backward that reads them must give exactly
     # the dtheta of the recomputing backward (task graph: b % 64 == 0; b = 100 takes the
     # per-step path), and S must be Q^2
     import torch
@@ -128,17 +128,19 @@ def test_cnp_saved_pair_is_bit_identical(b, k):
     G, _, dth = _cnp_gpu(theta, dG, b, k)
     th = tensor(theta, torch.float32)
     G2 = torch.empty_like(G)
+    Qs = torch.empty_like(G)
     S = torch.empty_like(G)
     F = torch.empty_like(G)
     dth2 = torch.empty_like(th)
     ws = torch.empty(max(P.cnp_workspace(nblk, b, k), 16), dtype=torch.uint8, device="cuda")
-    P.cnp_fwd_save(th, G2, None, S, F, b, k, ws)
-    P.cnp_bwd_saved(th, tensor(dG, torch.float32), S, F, dth2, b, k, ws)
+    P.cnp_fwd_save(th, G2, None, Qs, S, F, b, k, ws)
+    P.cnp_bwd_saved(th, tensor(dG, torch.float32), Qs, S, F, dth2, b, k, ws)
     torch.cuda.synchronize()
     assert P.device_status() == P.POETX_OK
     assert torch.equal(G2, G)
     assert torch.equal(dth2, dth)
     Q = np.stack([ref.theta_to_Q(t, b) for t in theta.astype(np.float64)])
+    assert np.array_equal(host(Qs), Q)  # the packing, bit-exact (fp32 theta is exact in fp64)
     assert np.abs(host(S) - Q @ Q).max() <= CNP_ABS
 
 
