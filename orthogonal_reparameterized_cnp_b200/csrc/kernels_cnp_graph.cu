@@ -549,6 +549,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
   __shared__ __align__(16) int s_job[(sizeof(CnpJob) + 3) / 4];
   int* ticket = g.counters + g.njobs * g.nblk;
   const int total = g.item_start[g.njobs];
+  pdl_trigger();
+  pdl_wait();
   if (threadIdx.x == 0) s_next = atomicAdd(ticket, 1);
   for (;;) {
     __syncthreads();  // smem of the previous item is free; s_next is visible
@@ -609,6 +611,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
 }
 
 __global__ void k_zero_ints(int* p, int n) {
+  pdl_trigger();
+  pdl_wait();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
 }
 
@@ -640,9 +644,9 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   g.err = device_error_flag();
   const int ncount = g.njobs * g.nblk + 1;
   begin_launch("cnp_elementwise", s);
-  k_zero_ints<<<(ncount + 255) / 256, 256, 0, s>>>(g.counters, ncount);
+  cudaError_t e = launch_pdl(k_zero_ints, dim3((ncount + 255) / 256), dim3(256), 0, s,
+                             g.counters, ncount);
   end_launch("cnp_elementwise", s);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // persistent grid: never more CTAs than can be resident at once
   static int per_sm_dev[64] = {0};  // once per device, outside any stream capture
@@ -663,9 +667,9 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   const int total = g.item_start[g.njobs];
   if (grid > total) grid = total;
   begin_launch("cnp_sgemm", s);
-  k_cnp_graph<<<grid, kThreads, kSmemBytes, s>>>(g);
+  e = launch_pdl(k_cnp_graph, dim3(grid), dim3(kThreads), kSmemBytes, s, g);
   end_launch("cnp_sgemm", s);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace poetx

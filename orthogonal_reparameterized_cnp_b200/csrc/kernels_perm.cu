@@ -199,6 +199,8 @@ __global__ void __launch_bounds__(kIlThreads, 1)
   uint16_t* const stage0 = reinterpret_cast<uint16_t*>(smem_raw);
   uint4* const il = reinterpret_cast<uint4*>(smem_raw + (size_t)NS * 8 * cols * 2);
   const int nchunk = cols / 8;
+  pdl_trigger();
+  pdl_wait();
   const unsigned ucols = (unsigned)cols;
   // slots of the source columns of the output chunks this thread owns (2 x 16 bit a word)
   uint32_t src[MAXC][4];
@@ -312,11 +314,11 @@ cudaError_t il8_launch(const void* in, void* out, const int32_t* row_idx, const 
   int grid = num_sms() * per_sm;
   if (grid > ngroups) grid = ngroups;
   begin_launch("permute", s);
-  k_gather_il8<MAXC, NS><<<grid, kIlThreads, smem, s>>>(
-      static_cast<const uint16_t*>(in), static_cast<uint16_t*>(out), row_idx, col_idx, rows,
-      cols, ld_in, ld_out);
+  const cudaError_t e = launch_pdl(k_gather_il8<MAXC, NS>, dim3(grid), dim3(kIlThreads), smem, s,
+                                   static_cast<const uint16_t*>(in), static_cast<uint16_t*>(out),
+                                   row_idx, col_idx, rows, cols, ld_in, ld_out);
   end_launch("permute", s);
-  return cudaGetLastError();
+  return e;
 }
 
 // Rows too wide for shared memory: gather straight from global memory (L2 absorbs the

@@ -722,6 +722,8 @@ __global__ void __launch_bounds__(256) k_pack_skew(const float* __restrict__ A,
 
 __global__ void k_split_reduce(const float* __restrict__ src, int nsplit, int64_t stride,
                                float* __restrict__ dst, int64_t count, int accumulate) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t n4 = count / 4;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -920,9 +922,10 @@ cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, fl
   if (blocks < 1) blocks = 1;
   if (blocks > num_sms() * 8) blocks = num_sms() * 8;
   begin_launch("reduce", s);
-  k_split_reduce<<<(unsigned)blocks, 256, 0, s>>>(src, nsplit, stride, dst, count, accumulate);
+  const cudaError_t e = launch_pdl(k_split_reduce, dim3((unsigned)blocks), dim3(256), 0, s, src,
+                                   nsplit, stride, dst, count, accumulate);
   end_launch("reduce", s);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s) {

@@ -347,6 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot_ptr;
+  // set-up done: from here on the previous kernel's results are read
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -605,9 +608,10 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
     attr_done[dev] = true;
   }
   begin_launch(family, s);
-  kern<<<grid, kThreads, Cfg<BN, B_RES>::SMEM_BYTES, s>>>(ma, mb, md, p);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), Cfg<BN, B_RES>::SMEM_BYTES, s,
+                                   ma, mb, md, p);
   end_launch(family, s);
-  return cudaGetLastError();
+  return e;
 }
 
 template <int BN>

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "../../include/poetx.h"
 
@@ -27,6 +28,35 @@ int* device_error_flag();
 
 // Number of SMs of the current device.
 int num_sms();
+
+// ---- programmatic dependent launch ------------------------------------------------
+// Kernels of the layer step are launched so that a kernel may start (and do its set-up)
+// while the previous kernel on the stream is still finishing.  Every kernel launched this
+// way calls pdl_wait() before its first access to global memory: that waits until the
+// previous kernel has completed and its writes are visible, so stream order is kept.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+#ifdef __CUDACC__
+// lets the next kernel on the stream be scheduled once every CTA of this one got here
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// waits until the previous kernel on the stream has completed (its writes visible)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+#endif
 
 // ---- permutation / gather kernels (kernels_perm.cu) ------------------------------
 // out[r, c] = in[row_idx ? row_idx[r] : r, col_idx[c]]
