@@ -44,7 +44,7 @@ SM_MAX_MHZ = 1965.0
 # DRAM bytes (read + write) per launch of a family's kernel from one ncu capture of the
 # current kernel (cold caches; mean over the family's launches in one step); families
 # without a capture of their current kernel report null.
-MEASURED_TRAFFIC = {"cnp_sgemm": (2.140e6 + 0.0003e6 + 16.828e6 + 0.515e6) / 2}
+MEASURED_TRAFFIC = {"cnp_sgemm": (2.141e6 + 0.0008e6 + 16.829e6 + 0.504e6) / 2}
 
 
 def parse_args(argv=None):
