@@ -10,12 +10,17 @@
 //   * the block-gradient contractions dG_j = sum_t g_t^T h_t over tokens, split over the
 //     token axis into fixed partial sums.
 //
-// Structure: one persistent CTA per SM, 192 threads.
+// Structure: one persistent CTA per SM, 320 threads.
 //   warp 0      TMA producer (one lane): A/B k-chunks of 64 into a STAGES-deep smem ring
+//               (or, for the block-diagonal products, A only with the item's whole B
+//               resident)
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x (M=128, N=BN, K=16) per chunk
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, convert, store to global
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator, convert, stage each 32 x 64
+//               piece in a 128-byte-swizzled 4 KB tile, TMA tensor store
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap the main loop
-// of tile t+1.  Operands may be K-major or MN-major (transposed) in global memory; both
+// of tile t+1.  The kernel is launched as a programmatic dependent of the previous kernel
+// on the stream: set-up (barriers, TMEM, tensor-map prefetch) runs before
+// griddepcontrol.wait, global memory only after it.  Operands may be K-major or MN-major (transposed) in global memory; both
 // are staged with the 128-byte swizzle the UMMA smem descriptors expect.
 //
 // Every mbarrier wait is bounded: after kWaitLimitNs the waiting role records
