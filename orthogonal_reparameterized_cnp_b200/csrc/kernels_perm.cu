@@ -5,9 +5,12 @@
 //
 // The permutation acts along the contiguous feature axis of a row-major matrix, so a
 // direct gather from global memory would touch a 32-byte sector per element.  Instead
-// each CTA stages whole source rows in shared memory with coalesced 16-byte loads and
-// writes the permuted row with coalesced 16-byte stores; the random access happens only
-// in shared memory.  HBM traffic is exactly one read and one write of the matrix.
+// source rows are staged in shared memory with coalesced 16-byte loads and the permuted
+// rows written with coalesced 16-byte stores; the random access happens only in shared
+// memory.  HBM traffic is exactly one read and one write of the matrix.  For 2-byte
+// elements (the bf16 layer) k_gather_il8 interleaves 8 rows per shared-memory word so
+// that one access serves a column of 8 rows; the row-staged kernels cover fp32 and rows
+// too wide for its stages.
 #include <cuda_bf16.h>
 
 #include "poetx_internal.h"

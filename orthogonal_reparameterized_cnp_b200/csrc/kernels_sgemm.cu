@@ -1,6 +1,8 @@
 // fp32 SIMT kernels: a batched FFMA GEMM with structured (symmetric / symmetric+skew)
 // outputs, and the small elementwise kernels of the Cayley-Neumann parameterisation
-// (POET-X technical summary, section 2.4).
+// (POET-X technical summary, section 2.4).  They run the fp32 layer and the CNP shapes
+// outside the one-launch task graph (b % 64 != 0 or more than three powers of S), plus
+// the fixed-order reduction of split token sums.
 //
 // The CNP works on b x b blocks in fp32.  Its products are between polynomials in the
 // skew-symmetric Q, so most outputs are symmetric (even powers of Q) or skew (odd
