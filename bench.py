@@ -2,27 +2,39 @@
 """POET-X linear forward + backward throughput on B200 (tokens/s), with roofline figures.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl poetx|reference]
+                    [--workload llama13b-block|llama8b-up|llama1b-attn|fp32-small]
 
-One step is one pass of the whole path over one batch of synthetic tokens:
-merge of the two permutations into W0' -> CNP forward (input and output blocks) ->
-layer forward (gather, block product, W0' GEMM, block product, scatter) -> layer
-backward (dG_R, dW, dV, dU, dG_P, dX) -> CNP backward (dtheta).
+One step is one pass of the per-step path over one batch of synthetic tokens: CNP forward
+(every block of the workload, one call) -> every linear's forward (gather, block product,
+W0' GEMM, block product, scatter) -> every linear's backward (dG_R, dW, dV, dU, dG_P, dX)
+-> CNP backward (dtheta of every block, one call).  The permutations are drawn and merged
+into W0' once per set of permutations (once per outer iteration), so that merge is not
+part of the step; its time is reported separately.
 
-Workload: the Llama-1B-shaped attention projection, n = m = 2048, b = 256, k = 4,
-T = 8192 tokens (4 x 2048), bf16 activations, fp32 theta / CNP.  Inputs rotate over three
-seeded sets (192 MB of x and dy, larger than the 126 MB L2) between steps.
+Default workload: the Llama-13B-shaped decoder block, all 7 linears as POET-X layers
+(q, k, v, o 5120 -> 5120; gate, up 5120 -> 13824; down 13824 -> 5120), b = 256, k = 4,
+T = 8192 tokens, bf16 activations, fp32 theta / CNP, 382 CNP blocks.  The step touches
+several GB, far more than the 126 MB L2, so consecutive steps never find their inputs in
+L2; workloads whose inputs fit in L2 rotate over three input sets instead.
+
+Besides the headline line the run measures: the layer-only figure (forward + backward
+without the CNP), CNP-only forward and backward (blocks/s), per-kernel-family device time
+from CUDA-graph replays, the FP32 FMA peak of the device, and (default workload only, under
+"also") the Llama-8B up-projection step, the fp32 small layer's CUDA-graph latency and the
+CNP sweep over b in {64, 128, 256, 512} and k in {2, 4, 6}.
 
 Under torchrun (N > 1) the step is data parallel (weak scaling): every rank takes its own
 T tokens with theta, G and W0' replicated, and the step ends with one NCCL sum all-reduce
-of dtheta; the step time is the maximum over ranks.  The outer-loop merge (once per inner
-loop, outside the step) is timed separately after the timed region.  ``--impl reference``
-times the float64 CPU oracle instead (rank 0 only) on a bounded token sample per step.
+of dtheta; the step time is the maximum over ranks.  ``--impl reference`` times the float64
+CPU oracle instead (rank 0 only) on a bounded token sample per step.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -40,34 +52,53 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 SM_MAX_MHZ = 1965.0
-
-# DRAM bytes (read + write) per launch of a family's kernel from one ncu capture of the
-# current kernel (cold caches; mean over the family's launches in one step); families
-# without a capture of their current kernel report null.
-MEASURED_TRAFFIC = {"cnp_sgemm": (2.141e6 + 0.0008e6 + 16.829e6 + 0.504e6) / 2}
+L2_BYTES = 126 << 20
+FAMILIES = ["gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm", "cnp_elementwise",
+            "reduce"]
+WORKLOADS = ["llama13b-block", "llama8b-up", "llama1b-attn", "fp32-small"]
+# kernel source of each family: a committed DRAM-traffic figure applies only while the
+# source it was captured from is unchanged
+FAMILY_SOURCES = {
+    "gemm_w0": "kernels_umma.cu", "gemm_blockdiag": "kernels_umma.cu",
+    "gemm_dG": "kernels_umma.cu", "permute": "kernels_perm.cu",
+    "cnp_sgemm": "kernels_cnp_graph.cu", "reduce": "kernels_sgemm.cu",
+}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.md")
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
-    ap.add_argument("--workload", default="llama1b-attn",
-                    choices=["llama1b-attn", "llama8b-up", "fp32-small"])
+    ap.add_argument("--workload", default="llama13b-block", choices=WORKLOADS)
+    ap.add_argument("--no-also", dest="also", action="store_false",
+                    help="skip the secondary workloads of the default run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-budget", type=float, default=20.0,
                     help="seconds of CPU work for the oracle baseline")
-    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every kernel from the host instead of replaying CUDA graphs")
     return ap.parse_args(argv)
 
 
 def workload(name):
-    from poetx_inputs import workload_llama1b_attn, workload_llama8b_up, workload_small_fp32
-    return {"llama1b-attn": workload_llama1b_attn, "llama8b-up": workload_llama8b_up,
-            "fp32-small": workload_small_fp32}[name]()
+    """The linears of a named workload (LayerShape list; one entry except the 13B block)."""
+    from poetx_inputs import (workload_llama13b_block, workload_llama1b_attn,
+                              workload_llama8b_up, workload_small_fp32)
+    if name == "llama13b-block":
+        return workload_llama13b_block()
+    return [{"llama8b-up": workload_llama8b_up, "llama1b-attn": workload_llama1b_attn,
+             "fp32-small": workload_small_fp32}[name]()]
+
+
+def workload_name(name, shapes):
+    s = shapes[0]
+    if name == "llama13b-block":
+        return f"llama13b-block-7linears-d5120-ffn13824-b{s.b}-k{s.k}-T{s.T}"
+    return s.name
 
 
 def load_peaks():
@@ -75,8 +106,30 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        return d, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json on this box)"
+
+
+def source_sha(fname: str) -> str:
+    path = os.path.join(ROOT, "orthogonal_reparameterized_cnp_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(family: str, workload_key: str):
+    """DRAM bytes (read + write) per launch of `family` on `workload_key` from the committed
+    ncu summary, or None when there is none or its kernel source has changed since."""
+    if not os.path.exists(TRAFFIC_FILE) or family not in FAMILY_SOURCES:
+        return None
+    sha = source_sha(FAMILY_SOURCES[family])
+    pat = re.compile(r"^\|\s*" + re.escape(family) + r"\s*\|\s*" + re.escape(workload_key) +
+                     r"\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]{16})\s*\|")
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            m = pat.match(line.strip())
+            if m and m.group(2) == sha:
+                return float(m.group(1))
+    return None
 
 
 # ------------------------------------------------------------------ clocks sampler
@@ -137,35 +190,50 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ algorithmic work
-def family_work(s, ksplit_R=1, ksplit_P=1):
-    """Algorithmic FLOPs / bytes per step for each kernel family of the bf16 path."""
-    T, n, m, b, k = s.T, s.n, s.m, s.b, s.k
-    es = 2 if s.dtype == "bf16" else 4
-    nP, nR = n // b, m // b
+def cnp_flops_per_block(b: int, k: int):
+    """(forward, backward) FLOPs of one block as the library computes it, counting a
+    product whose result is symmetric (or symmetric + skew) as half a product: forward
+    d + 1 half products (the d powers of S = Q^2, the last emitting E and F', then G);
+    backward with Q, S and F' kept: D = Q dG (2 b^3), the Horner terms of the adjoint
+    through S (d = 2: N_2 S, 2 b^3; d = 3: three more full products and one half
+    product: 7 b^3 in all), A = f_0 dG + dG F' - Y Q (4 b^3)."""
     d = (k + 1) // 2
-    cnp_fwd = (d + 1) * b ** 3                        # d symmetric powers + G (half products)
-    y_terms = 0 if d == 1 else (2 * b ** 3 + (d - 2) * 3 * b ** 3)
-    # the backward reads S and F' kept by the forward: D, the Horner terms, A
-    cnp_bwd = 2 * b ** 3 + y_terms + 4 * b ** 3
+    fwd = (d + 1) * b ** 3
+    horner = {1: 0, 2: 2, 3: 7}[d] * b ** 3
+    return float(fwd), float(2 * b ** 3 + horner + 4 * b ** 3)
+
+
+def family_work(shapes):
+    """Algorithmic FLOPs / bytes per step (all linears of the workload) of each kernel
+    family, and its launches per step."""
+    es = 2 if shapes[0].dtype == "bf16" else 4
+    T, b, k = shapes[0].T, shapes[0].b, shapes[0].k
+    w0 = bd = dg = perm = 0.0
+    nblk = 0
+    for s in shapes:
+        n, m = s.n, s.m
+        nP, nR = n // b, m // b
+        nblk += nP + nR
+        w0 += 2 * (2.0 * T * n * m)
+        # F1, F3, B1, B3: read and write one activation each, plus the G blocks
+        bd += 2.0 * es * T * (2 * n + 2 * m) + 2.0 * es * (nP + nR) * b * b
+        # dG_R, dG_P: read both activations, write the fp32 block gradients
+        dg += 2.0 * es * T * (n + m) + 4.0 * (nP + nR) * b * b
+        # gathers of x and dy, scatters of y and dx: one read and one write each
+        perm += 2.0 * es * (2 * T * n + 2 * T * m)
+    L = len(shapes)
+    cf, cb = cnp_flops_per_block(b, k)
     return {
-        "gemm_w0": {"bound": "tensor", "flops": 2 * (2.0 * T * n * m), "launches": 2},
-        "gemm_blockdiag": {"bound": "hbm", "launches": 4,
-                           "bytes": 2.0 * es * T * (2 * n + 2 * m) + 2.0 * es * (nP + nR) * b * b},
-        "gemm_dG": {"bound": "hbm", "launches": 2,
-                    "bytes": 2.0 * es * T * (n + m) + 4.0 * (nP + nR) * b * b},
-        "permute": {"bound": "hbm", "launches": 5,
-                    "bytes": 2.0 * es * (m * n + 2 * T * n + 2 * T * m)},
-        "cnp_sgemm": {"bound": "alu", "flops": float(nP + nR) * (cnp_fwd + cnp_bwd)},
+        "gemm_w0": {"bound": "tensor", "flops": w0, "launches": 2 * L},
+        "gemm_blockdiag": {"bound": "hbm", "bytes": bd, "launches": 4 * L},
+        "gemm_dG": {"bound": "hbm", "bytes": dg, "launches": 2 * L},
+        "permute": {"bound": "hbm", "bytes": perm, "launches": 4 * L},
+        "cnp_sgemm": {"bound": "alu", "flops": nblk * (cf + cb), "launches": 2,
+                      "flops_fwd": nblk * cf, "flops_bwd": nblk * cb},
     }
 
 
 # ------------------------------------------------------------------ oracle timing
-def oracle_inputs(s, T_sample=None):
-    from poetx_inputs import layer_inputs
-    inp = layer_inputs(s)
-    return inp
-
-
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -178,66 +246,80 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def oracle_step_sampler(s, inp, perms, budget_per_step):
-    """Returns (run_one_step, tokens_per_step): the oracle on a token window of T_s tokens
-    plus the amortised share of the per-step CNP work (b x b blocks, forward + backward)."""
-    from oracle import poetx_ref as ref
-    pP, pR = perms
-    nblk = s.n // s.b + s.m // s.b
-    theta = np.concatenate([inp.theta_P, inp.theta_R])
-    W0p = ref.merge_perm(inp.W0, pR, pP)
-    G_P = ref.cnp_forward(inp.theta_P, s.b, s.k)
-    G_R = ref.cnp_forward(inp.theta_R, s.b, s.k)
-    # calibration: one CNP block forward + backward, and the layer on 64 tokens
-    t0 = time.perf_counter()
-    g1 = ref.cnp_forward(theta[:1], s.b, s.k)
-    ref.cnp_backward(theta[:1], g1, s.b, s.k)
-    t_blk = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    Tc = min(64, s.T)
-    ref.layer_forward(inp.x[:Tc], W0p, G_P, G_R, pP, pR)
-    ref.layer_backward(inp.x[:Tc], inp.dy[:Tc], W0p, G_P, G_R, pP, pR)
-    t_tok = (time.perf_counter() - t0) / Tc
-    per_tok = t_tok + t_blk * nblk / s.T
-    T_s = int(max(1, min(s.T, budget_per_step / per_tok)))
-    state = {"credit": 0.0, "t0": 0}
+class OracleSampler:
+    """The float64 oracle on token windows of every linear of the workload, plus the
+    per-token share of the per-step CNP work (forward + backward of each b x b block)."""
 
-    def run_one():
-        a = state["t0"] % s.T
-        e = min(s.T, a + T_s)
-        x, dy = inp.x[a:e], inp.dy[a:e]
-        state["t0"] = e % s.T
-        W0p_ = ref.merge_perm(inp.W0, pR, pP)
-        y, U, V, W = ref.layer_forward(x, W0p_, G_P, G_R, pP, pR)
-        ref.layer_backward(x, dy, W0p_, G_P, G_R, pP, pR, U=U, W=W)
-        state["credit"] += nblk * (e - a) / s.T
-        while state["credit"] >= 1.0:
-            j = int(state["credit"] * 7919) % nblk
-            G = ref.cnp_forward(theta[j:j + 1], s.b, s.k)
-            ref.cnp_backward(theta[j:j + 1], G, s.b, s.k)
-            state["credit"] -= 1.0
+    def __init__(self, shapes, budget_per_step: float):
+        from oracle import poetx_ref as ref
+        from poetx_inputs import layer_inputs
+        self.ref = ref
+        self.shapes = shapes
+        self.T = shapes[0].T
+        self.b, self.k = shapes[0].b, shapes[0].k
+        self.lin = []
+        thetas = []
+        for s in shapes:
+            inp = layer_inputs(s)
+            pP, _ = ref.make_perm(inp.seed_P, s.n)
+            pR, _ = ref.make_perm(inp.seed_R, s.m)
+            W0p = ref.merge_perm(inp.W0.astype(np.float64), pR, pP)
+            G_P = ref.cnp_forward(inp.theta_P, s.b, s.k)
+            G_R = ref.cnp_forward(inp.theta_R, s.b, s.k)
+            self.lin.append((inp.x, inp.dy, W0p, G_P, G_R, pP, pR))
+            thetas += [inp.theta_P, inp.theta_R]
+        self.theta = np.concatenate(thetas)
+        self.nblk = len(self.theta)
+        # calibration: one CNP block forward + backward, and every linear on 32 tokens
+        t0 = time.perf_counter()
+        g1 = ref.cnp_forward(self.theta[:1], self.b, self.k)
+        ref.cnp_backward(self.theta[:1], g1, self.b, self.k)
+        t_blk = time.perf_counter() - t0
+        Tc = min(32, self.T)
+        t0 = time.perf_counter()
+        self._layers(0, Tc)
+        t_tok = (time.perf_counter() - t0) / Tc
+        per_tok = t_tok + t_blk * self.nblk / self.T
+        self.T_s = int(max(1, min(self.T, budget_per_step / per_tok)))
+        self.credit = 0.0
+        self.t0 = 0
+
+    def _layers(self, a, e):
+        ref = self.ref
+        for x, dy, W0p, G_P, G_R, pP, pR in self.lin:
+            y, U, V, W = ref.layer_forward(x[a:e], W0p, G_P, G_R, pP, pR)
+            ref.layer_backward(x[a:e], dy[a:e], W0p, G_P, G_R, pP, pR, U=U, W=W)
+
+    def run_one(self) -> int:
+        ref = self.ref
+        a = self.t0 % self.T
+        e = min(self.T, a + self.T_s)
+        self.t0 = e % self.T
+        self._layers(a, e)
+        self.credit += self.nblk * (e - a) / self.T
+        while self.credit >= 1.0:
+            j = int(self.credit * 7919) % self.nblk
+            G = ref.cnp_forward(self.theta[j:j + 1], self.b, self.k)
+            ref.cnp_backward(self.theta[j:j + 1], G, self.b, self.k)
+            self.credit -= 1.0
         return e - a
 
-    return run_one, T_s
+    def describe(self, name):
+        return (f"{name}: float64 oracle on windows of {self.T_s} of {self.T} tokens through "
+                f"all {len(self.shapes)} linear(s) (forward + backward) plus the per-token "
+                f"share of the CNP forward + backward of the {self.nblk} b={self.b} blocks")
 
 
-def oracle_throughput(s, budget_s):
+def oracle_throughput(name, shapes, budget_s):
     """Oracle tokens/s on a bounded sample of the workload (about budget_s of CPU work)."""
-    from oracle import poetx_ref as ref
-    inp = oracle_inputs(s)
-    pP, _ = ref.make_perm(inp.seed_P, s.n)
-    pR, _ = ref.make_perm(inp.seed_R, s.m)
-    run_one, T_s = oracle_step_sampler(s, inp, (pP, pR), budget_per_step=budget_s / 4)
-    run_one()  # warm
+    smp = OracleSampler(shapes, budget_per_step=budget_s / 4)
+    smp.run_one()  # warm
     tokens, t0 = 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s * 0.75:
-        tokens += run_one()
+        tokens += smp.run_one()
     dt = time.perf_counter() - t0
     return {"value": tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{s.name}: float64 oracle on windows of {T_s} of {s.T} tokens (fwd+bwd, "
-                      f"merge each window) plus the per-token share of the CNP forward+backward "
-                      f"of the {s.n // s.b + s.m // s.b} b={s.b} blocks; {tokens} tokens in "
-                      f"{dt:.1f} s"}
+            "sample": smp.describe(name) + f"; {tokens} tokens in {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -245,19 +327,15 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    s = workload(args.workload)
-    from oracle import poetx_ref as ref
-    inp = oracle_inputs(s)
-    pP, _ = ref.make_perm(inp.seed_P, s.n)
-    pR, _ = ref.make_perm(inp.seed_R, s.m)
+    shapes = workload(args.workload)
+    name = workload_name(args.workload, shapes)
     budget_total = 150.0
-    run_one, T_s = oracle_step_sampler(s, inp, (pP, pR),
-                                       budget_per_step=budget_total / max(1, args.steps + args.warmup))
+    smp = OracleSampler(shapes, budget_per_step=budget_total / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        run_one()
+        smp.run_one()
     tokens, t0 = 0, time.perf_counter()
     for _ in range(args.steps):
-        tokens += run_one()
+        tokens += smp.run_one()
     dt = time.perf_counter() - t0
     value = tokens / dt
     cores = blas_threads()
@@ -266,16 +344,22 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": s.name, "T": s.T, "n": s.n, "m": s.m, "b": s.b, "k": s.k,
-                   "tokens_per_step": T_s},
+        "config": workload_config(args.workload, shapes),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{T_s} of {s.T} tokens per step plus the per-token share of "
-                                   f"the CNP work, {args.steps} steps"},
+                         "sample": smp.describe(name) + f"; {args.steps} steps"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def workload_config(key, shapes):
+    s = shapes[0]
+    cfg = {"workload": workload_name(key, shapes), "T": s.T, "b": s.b, "k": s.k,
+           "linears": [[x.n, x.m] for x in shapes],
+           "cnp_blocks_per_step": sum(x.n // x.b + x.m // x.b for x in shapes)}
+    return cfg
 
 
 # ------------------------------------------------------------------ multi-rank timing
@@ -296,13 +380,235 @@ def job_tokens_per_s(world: int, tokens_per_rank_step: int, steps: int, max_ms: 
     return world * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
+# ------------------------------------------------------------------ GPU helpers
+def graph_of(fn, stream):
+    """Captures fn(stream) into a CUDA graph (on the current device)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(stream)
+    return g
+
+
+def time_graphs(graphs, reps, stream):
+    """Device time (ms) of `reps` back-to-back replays cycling over `graphs`."""
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(reps):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def measure_fma_peak(P, dev):
+    """FP32 FMA TFLOP/s of this device: the library's probe kernel, 2 CTAs of 512 threads
+    per SM, best of 5 launches timed with events."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ctas, iters = 2 * sms, 20000
+    out = torch.empty(ctas * 512, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    P.fma_probe(out, ctas, 200, stream)
+    best = 0.0
+    for _ in range(5):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        P.fma_probe(out, ctas, iters, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        best = max(best, ctas * 512 * 16 * iters * 2 / (ms / 1e3) / 1e12)
+    return best
+
+
+class Workload:
+    """Device state of one workload: the group of linears and its input sets."""
+
+    def __init__(self, key, dev, int8=False, device_inputs=False, seed=0):
+        import torch
+
+        from orthogonal_reparameterized_cnp_b200 import poetx as P
+        from poetx_inputs import layer_inputs
+        self.key = key
+        self.shapes = workload(key)
+        s0 = self.shapes[0]
+        self.T, self.b, self.k = s0.T, s0.b, s0.k
+        self.bf16 = s0.dtype == "bf16"
+        self.act = torch.bfloat16 if self.bf16 else torch.float32
+        to = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
+        specs, xs, dys, self.host_inputs = [], [], [], []
+        gen = torch.Generator(device=dev)
+        for i, s in enumerate(self.shapes):
+            pP, _ = P.make_perm((s.config_id << 32) | (s.linear_id << 8) | 0, s.n)
+            pR, _ = P.make_perm((s.config_id << 32) | (s.linear_id << 8) | 1, s.m)
+            if device_inputs:
+                # seeded draws on the device at the workload's scales (timing-only runs)
+                gen.manual_seed(seed * 1000 + i)
+                rn = lambda shape, std, dt: (torch.randn(shape, generator=gen, device=dev)  # noqa: E731
+                                             * std).to(dt)
+                W0 = rn((s.m, s.n), 1.0 / np.sqrt(s.n), self.act)
+                tP = rn((s.nblk_P, s.ntri), s.std_theta, torch.float32)
+                tR = rn((s.nblk_R, s.ntri), s.std_theta, torch.float32)
+                x = rn((s.T, s.n), 1.0, self.act)
+                dy = rn((s.T, s.m), 1.0, self.act)
+            else:
+                inp = layer_inputs(s)
+                W0, tP, tR = to(inp.W0, self.act), to(inp.theta_P, torch.float32), \
+                    to(inp.theta_R, torch.float32)
+                x, dy = to(inp.x, self.act), to(inp.dy, self.act)
+            specs.append((W0, tP, tR, pP, pR))
+            xs.append(x)
+            dys.append(dy)
+        self.group = P.PoetxLinearGroup(specs, self.b, self.k, self.T, int8_weight=int8)
+        es = 2 if self.bf16 else 4
+        in_bytes = sum(s.T * (s.n + s.m) * es for s in self.shapes)
+        # inputs larger than L2 per step need no rotation; small ones rotate over 3 sets
+        self.nsets = 1 if in_bytes > 2 * L2_BYTES else 3
+        self.xs, self.dys = [xs], [dys]
+        for r in range(1, self.nsets):
+            self.xs.append([torch.roll(t, shifts=r, dims=0).contiguous() for t in xs])
+            self.dys.append([torch.roll(t, shifts=r, dims=0).contiguous() for t in dys])
+        self.ys = [torch.empty((s.T, s.m), dtype=self.act, device=dev) for s in self.shapes]
+        self.dxs = [torch.empty((s.T, s.n), dtype=self.act, device=dev) for s in self.shapes]
+        self.in_bytes = in_bytes
+        self.nblk = self.group.cnp.nblk
+
+    def step(self, i, stream):
+        self.group.step(self.xs[i % self.nsets], self.dys[i % self.nsets], self.ys, self.dxs,
+                        stream)
+
+    def layer_only(self, i, stream):
+        g = self.group
+        xs, dys = self.xs[i % self.nsets], self.dys[i % self.nsets]
+        g.forward(xs, self.ys, stream)
+        g.backward(xs, dys, self.dxs, 0, stream)
+
+    def l2_note(self):
+        if self.nsets == 1:
+            return (f"each step reads {self.in_bytes >> 20} MB of inputs and touches several "
+                    f"times that (> 126 MB L2): no step finds its inputs in L2")
+        return (f"inputs rotate over {self.nsets} sets "
+                f"({self.nsets * self.in_bytes >> 20} MB > 126 MB L2)")
+
+
+def check_status(P, stream, where):
+    if P.device_status(stream) != P.POETX_OK:
+        raise RuntimeError(f"device status not OK after {where}")
+
+
+def family_attribution(P, wl, stream, reps):
+    """Per-family device time of one step from CUDA-graph replays: the step is captured
+    once per family with CUDA events around that family's launches (event nodes of the
+    graph), replayed `reps` times, and the bracketed times of each replay summed."""
+    import torch
+    out = {}
+    for fam in FAMILIES:
+        P.profile_begin(fam)
+        g = graph_of(lambda st: wl.step(0, st), stream)
+        P.profile_begin(None)
+        tot, launches = 0.0, 0
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            n, ms = P.profile_end()
+            tot += ms
+            launches = n
+        out[fam] = {"launches_per_step": launches, "ms_per_step": tot / reps,
+                    "avg_launch_ms": (tot / reps / launches) if launches else None}
+        del g
+    check_status(P, stream, "the attribution replays")
+    return out
+
+
+def cnp_only(P, wl, stream, reps):
+    """CNP forward and backward alone (one call each over every block), CUDA-graph replay."""
+    c = wl.group.cnp
+    gf = graph_of(lambda st: c.forward(st), stream)
+    gb = graph_of(lambda st: c.backward(st), stream)
+    time_graphs([gf, gb], 2, stream)
+    fms = time_graphs([gf], reps, stream) / reps
+    bms = time_graphs([gb], reps, stream) / reps
+    check_status(P, stream, "the CNP-only replays")
+    cf, cb = cnp_flops_per_block(wl.b, wl.k)
+    return {"blocks": c.nblk, "b": wl.b, "k": wl.k, "fwd_ms": fms, "bwd_ms": bms,
+            "fwd_blocks_per_s": c.nblk / (fms / 1e3), "bwd_blocks_per_s": c.nblk / (bms / 1e3),
+            "fwd_tflops": c.nblk * cf / (fms / 1e3) / 1e12,
+            "bwd_tflops": c.nblk * cb / (bms / 1e3) / 1e12}
+
+
+def cnp_sweep(P, dev, stream, fma_peak):
+    """The CNP-only sweep: b in {64, 128, 256, 512}, k in {2, 4, 6}; block count = both
+    sides of all 7 linears x 32 layers of Llama-8B shapes; seeded device inputs at the
+    sweep's scales (theta ~ N(0, 0.01^2), dG ~ N(0, 1))."""
+    import torch
+
+    from orthogonal_reparameterized_cnp_b200 import poetx as P_
+    from poetx_inputs import cnp_sweep_blocks
+    res = []
+    gen = torch.Generator(device=dev)
+    for b in (64, 128, 256, 512):
+        nblk = cnp_sweep_blocks(b)
+        gen.manual_seed(b)
+        c = P_.CnpBuffers(nblk, b, 2, dev)
+        c.theta.copy_(torch.randn(c.theta.shape, generator=gen, device=dev) * 0.01)
+        c.dG.copy_(torch.randn(c.dG.shape, generator=gen, device=dev))
+        for k in (2, 4, 6):
+            c.set_order(k)
+            c.forward(stream)
+            c.backward(stream)
+            gf = graph_of(lambda st: c.forward(st), stream)
+            gb = graph_of(lambda st: c.backward(st), stream)
+            time_graphs([gf, gb], 1, stream)
+            reps = 3
+            fms = time_graphs([gf], reps, stream) / reps
+            bms = time_graphs([gb], reps, stream) / reps
+            cf, cb = cnp_flops_per_block(b, k)
+            res.append({"b": b, "k": k, "blocks": nblk,
+                        "fwd_blocks_per_s": nblk / (fms / 1e3),
+                        "bwd_blocks_per_s": nblk / (bms / 1e3),
+                        "fwd_frac_fma": nblk * cf / (fms / 1e3) / 1e12 / fma_peak,
+                        "bwd_frac_fma": nblk * cb / (bms / 1e3) / 1e12 / fma_peak})
+            del gf, gb
+        del c
+        torch.cuda.empty_cache()
+    check_status(P, stream, "the CNP sweep")
+    return res
+
+
+def secondary_step(P, key, dev, stream, reps):
+    """Step and layer-only throughput of a secondary workload, CUDA-graph replay, seeded
+    device inputs (timing only; parity of these shapes is checked by the tests)."""
+    import torch
+    wl = Workload(key, dev, device_inputs=True, seed=7)
+    for i in range(3):
+        wl.step(i, stream)
+    torch.cuda.synchronize()
+    gs = [graph_of(lambda st, i=i: wl.step(i, st), stream) for i in range(wl.nsets)]
+    gl = [graph_of(lambda st, i=i: wl.layer_only(i, st), stream) for i in range(wl.nsets)]
+    time_graphs(gs, 3, stream)
+    ms = time_graphs(gs, reps, stream) / reps
+    lms = time_graphs(gl, reps, stream) / reps
+    check_status(P, stream, f"the {key} replays")
+    out = {"workload": workload_name(key, wl.shapes), "ms_per_step": ms,
+           "tokens_per_s": wl.T / (ms / 1e3), "layer_only_tokens_per_s": wl.T / (lms / 1e3),
+           "launch": "cuda_graph", "l2": wl.l2_note(), "steps": reps}
+    del gs, gl, wl
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_poetx(args):
     import torch
     import torch.distributed as dist
 
+    from orthogonal_reparameterized_cnp_b200 import dp
     from orthogonal_reparameterized_cnp_b200 import poetx as P
-    from poetx_inputs import layer_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -316,150 +622,89 @@ def run_poetx(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    s = workload(args.workload)
-    inp = layer_inputs(s)
-    act = torch.bfloat16 if s.dtype == "bf16" else torch.float32
-    to = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)  # noqa: E731
-    pP, _ = P.make_perm(inp.seed_P, s.n)
-    pR, _ = P.make_perm(inp.seed_R, s.m)
-    layer = P.PoetxLinear(to(inp.W0, act), to(inp.theta_P, torch.float32),
-                          to(inp.theta_R, torch.float32), pP, pR, s.b, s.k, s.T)
-    nsets = 3
-    xs = [to(inp.x, act)]
-    dys = [to(inp.dy, act)]
-    for i in range(1, nsets):  # further sets: the same values rolled by i tokens
-        xs.append(torch.roll(xs[0], shifts=i, dims=0).contiguous())
-        dys.append(torch.roll(dys[0], shifts=i, dims=0).contiguous())
-    y = torch.empty((s.T, s.m), dtype=act, device=dev)
-    dx = torch.empty((s.T, s.n), dtype=act, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    fma_peak = measure_fma_peak(P, dev)
 
-    from orthogonal_reparameterized_cnp_b200 import dp
+    wl = Workload(args.workload, dev)
+    shapes = wl.shapes
+    T = wl.T
 
     def exchange():  # the data-parallel step's one collective (a no-op on one rank)
         if world > 1:
-            dp.allreduce_dtheta(layer.dtheta)
-
-    def step(i):
-        layer.step(xs[i % nsets], dys[i % nsets], y, dx, stream)
-        exchange()
+            dp.allreduce_dtheta(wl.group.cnp.dtheta)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # warm-up
+    # warm-up (eager), then the step captured once per input set
     for i in range(max(3, args.warmup)):
-        step(i)
+        wl.step(i, stream)
+        exchange()
     torch.cuda.synchronize(dev)
-    if P.device_status(stream) != P.POETX_OK:
-        raise RuntimeError("device status not OK after warm-up")
-
-    # per-family breakdown (short profiled pass, outside the timed region)
-    work = family_work(s)
-    breakdown = {}
-    for fam in ["gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm",
-                "cnp_elementwise", "reduce"]:
-        P.profile_begin(fam)
-        nprof = 10
-        for i in range(nprof):
-            step(i)
+    check_status(P, stream, "warm-up")
+    graphs = None
+    graph_launches = 0
+    if args.graph:
+        graphs = []
+        for i in range(wl.nsets):
+            n0 = P.launch_count()
+            graphs.append(graph_of(lambda st, i=i: wl.step(i, st), stream))
+            graph_launches = P.launch_count() - n0
+        for i in range(3):
+            with torch.cuda.stream(stream):
+                graphs[i % wl.nsets].replay()
+            exchange()
         torch.cuda.synchronize(dev)
-        launches, ms = P.profile_end()
-        breakdown[fam] = {"launches_per_step": launches / nprof, "ms_per_step": ms / nprof}
-    dominant = max(breakdown, key=lambda f: breakdown[f]["ms_per_step"])
+        check_status(P, stream, "graph warm-up")
 
     # timed region
     props = torch.cuda.get_device_properties(dev)
     uuid = str(getattr(props, "uuid", "") or "")
     gpu_id = (uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if uuid else str(local)
     sampler = ClockSampler(gpu_id)
-    # the whole step captured once per input set and replayed (no per-kernel host work)
-    graphs = None
-    graph_launches = 0
-    if args.graph:
-        graphs = []
-        for i in range(nsets):
-            gr = torch.cuda.CUDAGraph()
-            n0 = P.launch_count()
-            with torch.cuda.graph(gr):
-                layer.step(xs[i], dys[i], y, dx, torch.cuda.current_stream(dev))
-            graph_launches = P.launch_count() - n0
-            graphs.append(gr)
-        for i in range(3):
-            graphs[i % nsets].replay()
-            exchange()
-        torch.cuda.synchronize(dev)
-        if P.device_status(stream) != P.POETX_OK:
-            raise RuntimeError("device status not OK after graph warm-up")
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
     time.sleep(0.3)
     launches0 = P.launch_count()
-    if not graphs:
-        P.profile_begin(dominant)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for i in range(args.steps):
-        if graphs:
-            graphs[i % nsets].replay()  # the layer's kernels; the collective stays outside
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(args.steps):
+            if graphs:
+                graphs[i % wl.nsets].replay()  # the layers' kernels; the collective outside
+            else:
+                wl.step(i, stream)
             exchange()
-        else:
-            step(i)
-    ev1.record(stream)
+        ev1.record(stream)
     torch.cuda.synchronize(dev)
-    if graphs:
-        launches = graph_launches * args.steps  # libpoetx kernels in the replayed graphs
-    else:
-        dom_launches, dom_ms = P.profile_end()
-        launches = P.launch_count() - launches0
+    launches = graph_launches * args.steps if graphs else P.launch_count() - launches0
     barrier()
     clocks = sampler.stop()
     elapsed_ms = ev0.elapsed_time(ev1)
-    if graphs:
-        # per-launch device time of the dominant family: eager steps right after the timed
-        # region, each of its launches bracketed by CUDA events on the launch stream
-        P.profile_begin(dominant)
-        for i in range(min(args.steps, 300)):
-            step(i)
-        torch.cuda.synchronize(dev)
-        dom_launches, dom_ms = P.profile_end()
     max_ms = max_over_ranks(elapsed_ms, dist if world > 1 else None, dev)
-    if P.device_status(stream) != P.POETX_OK:
-        raise RuntimeError("device status not OK after the timed region")
+    check_status(P, stream, "the timed region")
     ms_per_step = max_ms / args.steps
-    value = job_tokens_per_s(world, s.T, args.steps, max_ms)
+    value = job_tokens_per_s(world, T, args.steps, max_ms)
 
-    # roofline of the dominant kernel family
+    reps = max(10, min(args.steps, 50))
+    # layer-only figure: forward + backward of every linear without the CNP
+    gl = [graph_of(lambda st, i=i: wl.layer_only(i, st), stream) for i in range(wl.nsets)]
+    time_graphs(gl, 3, stream)
+    lms = time_graphs(gl, reps, stream) / reps
+    check_status(P, stream, "the layer-only replays")
+    del gl
+    cnp = cnp_only(P, wl, stream, reps)
+
+    # per-family device time and the roofline of the dominant family
+    work = family_work(shapes)
+    breakdown = family_attribution(P, wl, stream, reps=min(reps, 20))
+    dominant = max(breakdown, key=lambda f: breakdown[f]["ms_per_step"])
     peaks, peak_src = load_peaks()
-    avg_launch_ms = dom_ms / max(1, dom_launches)
-    w = work.get(dominant)
-    roof = None
-    if w is not None:
-        # launches of the family per step (exact, from the profiled pre-pass); the event
-        # pool may bracket fewer launches than the timed region makes
-        per_launch_steps = breakdown[dominant]["launches_per_step"]
-        if w["bound"] == "tensor":
-            achieved = w["flops"] / per_launch_steps / (avg_launch_ms / 1e3) / 1e12 \
-                if per_launch_steps else 0.0
-            peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-            unit = "TFLOP/s"
-        elif w["bound"] == "hbm":
-            achieved = w["bytes"] / per_launch_steps / (avg_launch_ms / 1e3) / 1e9
-            peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-            unit = "GB/s"
-        else:
-            achieved = w["flops"] / per_launch_steps / (avg_launch_ms / 1e3) / 1e12
-            peak = SM_COUNT * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
-            unit = "TFLOP/s"
-        roof = {"kernel": dominant, "bound": w["bound"], "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak if peak else None,
-                "traffic": MEASURED_TRAFFIC.get(dominant),
-                "peak_source": peak_src if w["bound"] != "alu" else
-                "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz",
-                "avg_launch_ms": avg_launch_ms, "launches": dom_launches}
+    wkey = workload_name(args.workload, shapes)
     for fam, bd in breakdown.items():
         ww = work.get(fam)
         if ww and bd["ms_per_step"] > 0:
@@ -467,27 +712,52 @@ def run_poetx(args):
                 bd["achieved_tflops"] = ww["flops"] / (bd["ms_per_step"] / 1e3) / 1e12
             if "bytes" in ww:
                 bd["achieved_gbs"] = ww["bytes"] / (bd["ms_per_step"] / 1e3) / 1e9
+    roof = None
+    w = work.get(dominant)
+    bd = breakdown[dominant]
+    if w is not None and bd["launches_per_step"]:
+        per_launch_s = bd["avg_launch_ms"] / 1e3
+        nl = bd["launches_per_step"]
+        if w["bound"] == "tensor":
+            achieved = w["flops"] / nl / per_launch_s / 1e12
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            unit, psrc = "TFLOP/s", peak_src + ", bf16 burst"
+        elif w["bound"] == "hbm":
+            achieved = w["bytes"] / nl / per_launch_s / 1e9
+            peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+            unit, psrc = "GB/s", peak_src
+        else:
+            achieved = w["flops"] / nl / per_launch_s / 1e12
+            peak = fma_peak
+            unit, psrc = "TFLOP/s", "measured: FP32 FMA probe kernel on this device"
+        roof = {"kernel": dominant, "bound": w["bound"], "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak if peak else None,
+                "traffic": committed_traffic(dominant, wkey),
+                "peak_source": psrc, "avg_launch_ms": bd["avg_launch_ms"],
+                "launches_per_step": nl,
+                "timing": "CUDA events around each launch of the family, as event nodes of "
+                          "the captured step graph, averaged over replays"}
+        if w["bound"] == "tensor":
+            sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+            roof["frac_of_sustained"] = achieved / sus
 
     # end to end through the public API with host buffers (pinned), copies timed: every
-    # step uploads its x, dy, theta and downloads y, dx, dtheta; the host pipeline runs
-    # the uploads of the next step and the downloads of the previous one on the two copy
-    # engines while a step computes
+    # step uploads every linear's x and dy and theta, and downloads y, dx and dtheta; the
+    # host pipeline overlaps the uploads of the next step and the downloads of the previous
+    # one with the step's kernels (two copy engines)
     e2e = None
     if args.e2e_steps > 0:
         from orthogonal_reparameterized_cnp_b200.host_pipeline import HostPipeline
-        hx = [xs[i].cpu().pin_memory() for i in range(nsets)]
-        hdy = [dys[i].cpu().pin_memory() for i in range(nsets)]
-        hth = layer.theta.cpu().pin_memory()
-        hy = torch.empty(y.shape, dtype=act).pin_memory()
-        hdx = torch.empty(dx.shape, dtype=act).pin_memory()
-        hdth = torch.empty(layer.dtheta.shape, dtype=torch.float32).pin_memory()
-        pipe = HostPipeline(layer, nbuf=2, exchange=exchange if world > 1 else None)
-
-        def e2e_step(i):
-            pipe.submit(i, hx[i % nsets], hdy[i % nsets], hth, hy, hdx, hdth)
-
+        g = wl.group
+        hx = [t.cpu().pin_memory() for t in wl.xs[0]]
+        hdy = [t.cpu().pin_memory() for t in wl.dys[0]]
+        hth = g.cnp.theta.cpu().pin_memory()
+        hy = [torch.empty(t.shape, dtype=wl.act).pin_memory() for t in wl.ys]
+        hdx = [torch.empty(t.shape, dtype=wl.act).pin_memory() for t in wl.dxs]
+        hdth = torch.empty(g.cnp.dtheta.shape, dtype=torch.float32).pin_memory()
+        pipe = HostPipeline(g, nbuf=2, exchange=exchange if world > 1 else None)
         for i in range(3):
-            e2e_step(i)
+            pipe.submit(i, hx, hdy, hth, hy, hdx, hdth)
         pipe.synchronize()
         barrier()
         torch.cuda.synchronize(dev)
@@ -495,116 +765,118 @@ def run_poetx(args):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(pipe.h2d)  # every step's first operation (its upload) follows this
         for i in range(args.e2e_steps):
-            e2e_step(i)
+            pipe.submit(i, hx, hdy, hth, hy, hdx, hdth)
         e1.record(pipe.d2h)  # the last download is the last operation of the last step
         pipe.synchronize()
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
-        h2d = hx[0].numel() * hx[0].element_size() + hdy[0].numel() * hdy[0].element_size() + \
-            hth.numel() * 4
-        d2h = hy.numel() * hy.element_size() + hdx.numel() * hdx.element_size() + hdth.numel() * 4
-        e2e = {"value": job_tokens_per_s(world, s.T, args.e2e_steps, e_ms), "unit": "tokens/s",
+        nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)  # noqa: E731
+        h2d = nbytes(hx) + nbytes(hdy) + hth.numel() * 4
+        d2h = nbytes(hy) + nbytes(hdx) + hdth.numel() * 4
+        e2e = {"value": job_tokens_per_s(world, T, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps, "copies": "overlapped with compute (2 buffer sets)"}
-        if P.device_status(stream) != P.POETX_OK:
-            raise RuntimeError("device status not OK after the end-to-end steps")
+        check_status(P, stream, "the end-to-end steps")
+        del pipe, hx, hdy, hy, hdx
 
-    # outer-loop merge (once per inner loop, not part of the step): device time per call
+    # the merge of the permutations into W0' (S1: once per set of permutations, every
+    # linear of the workload), and the outer-loop merge of the first linear (once per
+    # inner loop); device time per call
+    merge = None
+    gm = graph_of(lambda st: wl.group.merge(st), stream)
+    time_graphs([gm], 2, stream)
+    mms = time_graphs([gm], 10, stream) / 10
+    mbytes = sum(2.0 * s.m * s.n * (2 if wl.bf16 else 4) for s in shapes)
+    merge = {"ms": mms, "achieved_gbs": mbytes / (mms / 1e3) / 1e9}
+    del gm
     outer = None
-    if s.dtype == "bf16":
-        pP2, _ = P.make_perm(inp.seed_P + 1000003, s.n)
-        pR2, _ = P.make_perm(inp.seed_R + 1000003, s.m)
+    if wl.bf16:
+        L0 = wl.group.layers[0]
+        s = shapes[0]
+        pP2, _ = P.make_perm(12345 + 1000003, s.n)
+        pR2, _ = P.make_perm(12346 + 1000003, s.m)
         i32 = lambda a: torch.as_tensor(np.asarray(a, dtype=np.int32), device=dev)  # noqa: E731
         pP2d, pR2d = i32(pP2), i32(pR2)
-        W0p_new = torch.empty_like(layer.W0p)
+        W0p_new = torch.empty_like(L0.W0p)
         mws = torch.empty(P.outer_merge_workspace(s.m, s.n, P.POETX_BF16), dtype=torch.uint8,
                           device=dev)
-        GP, GR = layer.G_ops()
-
-        def merge_call():
-            P.outer_merge(layer.W0p, GP, GR, s.b, layer.inv_P, layer.inv_R, pP2d, pR2d,
-                          W0p_new, mws, stream)
-
-        for _ in range(3):
-            merge_call()
-        reps = 20
-        m0 = torch.cuda.Event(enable_timing=True)
-        m1 = torch.cuda.Event(enable_timing=True)
-        m0.record(stream)
-        for _ in range(reps):
-            merge_call()
-        m1.record(stream)
-        torch.cuda.synchronize(dev)
-        mms = m0.elapsed_time(m1) / reps
-        # algorithmic: read W0' and write W0'_new (bf16), read both G; 2 b-wide products
-        mbytes = 2 * s.m * s.n * 2 + (s.n + s.m) * s.b * 2
-        outer = {"ms": mms, "achieved_gbs": mbytes / (mms / 1e3) / 1e9,
-                 "achieved_tflops": 4.0 * s.m * s.n * s.b / (mms / 1e3) / 1e12,
-                 "launches": 5}
-        if P.device_status(stream) != P.POETX_OK:
-            raise RuntimeError("device status not OK after the outer merge")
+        GP, GR = L0.G_ops()
+        go = graph_of(lambda st: P.outer_merge(L0.W0p, GP, GR, s.b, L0.inv_P, L0.inv_R, pP2d,
+                                               pR2d, W0p_new, mws, st), stream)
+        time_graphs([go], 2, stream)
+        oms = time_graphs([go], 10, stream) / 10
+        mb = 2 * s.m * s.n * 2 + (s.n + s.m) * s.b * 2
+        outer = {"linear": [s.n, s.m], "ms": oms, "achieved_gbs": mb / (oms / 1e3) / 1e9,
+                 "achieved_tflops": 4.0 * s.m * s.n * s.b / (oms / 1e3) / 1e12}
+        check_status(P, stream, "the outer merge")
+        del go, W0p_new, mws
 
     # the same step with the int8 merged weight (POET-XQ reading), CUDA-graph replay
     xq = None
-    if s.dtype == "bf16" and args.graph:
-        lq = P.PoetxLinear(to(inp.W0, act), to(inp.theta_P, torch.float32),
-                           to(inp.theta_R, torch.float32), pP, pR, s.b, s.k, s.T,
-                           int8_weight=True)
+    if wl.bf16 and args.graph:
+        wq = Workload(args.workload, dev, int8=True, device_inputs=True, seed=3)
         for i in range(3):
-            lq.step(xs[i % nsets], dys[i % nsets], y, dx, stream)
+            wq.step(i, stream)
         torch.cuda.synchronize(dev)
-        gq = []
-        for i in range(nsets):
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr):
-                lq.step(xs[i], dys[i], y, dx, torch.cuda.current_stream(dev))
-            gq.append(gr)
-        for i in range(3):
-            gq[i % nsets].replay()
-        nq = min(args.steps, 500)
-        q0 = torch.cuda.Event(enable_timing=True)
-        q1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(dev)
-        q0.record(stream)
-        for i in range(nq):
-            gq[i % nsets].replay()
-        q1.record(stream)
-        torch.cuda.synchronize(dev)
-        if P.device_status(stream) != P.POETX_OK:
-            raise RuntimeError("device status not OK after the int8-weight steps")
-        qms = q0.elapsed_time(q1) / nq
-        xq = {"ms_per_step": qms, "tokens_per_s": s.T / (qms / 1e3), "steps": nq,
-              "weight": "int8 W0' (per-row scales), dequantised into scratch per call"}
-        del gq
+        gq = [graph_of(lambda st, i=i: wq.step(i, st), stream) for i in range(wq.nsets)]
+        time_graphs(gq, 3, stream)
+        qms = time_graphs(gq, reps, stream) / reps
+        check_status(P, stream, "the int8-weight steps")
+        xq = {"ms_per_step": qms, "tokens_per_s": T / (qms / 1e3), "steps": reps,
+              "weight": "int8 W0' (per-row scales)"}
+        del gq, wq
+        torch.cuda.empty_cache()
+
+    also = None
+    if args.also and args.workload == "llama13b-block" and world == 1:
+        also = {}
+        del graphs
+        graphs = None
+        torch.cuda.empty_cache()
+        for key in ("llama8b-up", "fp32-small"):
+            try:
+                also[key] = secondary_step(P, key, dev, stream,
+                                           reps=20 if key == "llama8b-up" else 200)
+            except Exception as exc:  # reported in the line; the headline stands on its own
+                also[key] = {"error": f"{type(exc).__name__}: {exc}"}
+        if "ms_per_step" in also.get("fp32-small", {}):
+            also["fp32-small"]["latency_us"] = 1e3 * also["fp32-small"]["ms_per_step"]
+        try:
+            also["cnp_sweep"] = cnp_sweep(P, dev, stream, fma_peak)
+        except Exception as exc:
+            also["cnp_sweep"] = {"error": f"{type(exc).__name__}: {exc}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_throughput(s, args.oracle_budget)
+        cpu = oracle_throughput(wkey, shapes, args.oracle_budget)
 
-    nblk = s.n // s.b + s.m // s.b
+    cfg = workload_config(args.workload, shapes)
+    cfg.update({
+        "l2": wl.l2_note(), "parallelism": f"dp{world}" if world > 1 else "single",
+        "launch": "cuda_graph" if args.graph else "eager",
+        "step": "CNP forward (one call, every block) + every linear's forward + every "
+                "linear's backward + CNP backward (one call); the merge of the "
+                "permutations is once per set of permutations, reported under 'merge'"})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if s.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": s.name, "T": s.T, "n": s.n, "m": s.m, "b": s.b, "k": s.k,
-                   "cnp_blocks_per_step": nblk,
-                   "l2": f"inputs rotate over {nsets} sets of x and dy "
-                         f"({nsets * (s.T * (s.n + s.m) * (2 if s.dtype == 'bf16' else 4)) >> 20} MB"
-                         f" > 126 MB L2)",
-                   "parallelism": f"dp{world}" if world > 1 else "single",
-                   "launch": "cuda_graph" if graphs else "eager",
-                   "roofline_timing": ("eager steps after the timed region" if graphs
-                                       else "inside the timed region")},
+        "dtype": "bf16" if wl.bf16 else "f32", "data": "synthetic",
+        "config": cfg,
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": int(launches),
         "roofline": roof,
         "cpu_baseline": cpu,
+        "layer_only": {"tokens_per_s": world * T / (lms / 1e3), "ms_per_step": lms,
+                       "what": "every linear's forward + backward, no CNP (CUDA graph)"},
+        "cnp": cnp,
+        "fma_peak_tflops": fma_peak,
         "kernels": breakdown,
+        "merge": merge,
         "outer_merge": outer,
         "int8_weight_step": xq,
-        "cnp_blocks_per_s": world * nblk * args.steps / (max_ms / 1e3),
+        "also": also,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

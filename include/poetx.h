@@ -93,6 +93,17 @@ const char* poetx_version(void);
 int poetx_make_perm(uint64_t seed, int32_t n, int32_t* perm, int32_t* inv);
 
 /*
+ * Inverse of a given index map, in HOST memory (POET-X section 2.2: Pi^T is applied as the
+ * gather by the inverse map, inv[perm[i]] = i).  The map is checked first: every entry must
+ * lie in [0, n) and appear once (a bijection), else nothing is written.
+ *   perm: caller-owned host array of n int32, read.  inv: host array of n int32, written;
+ *   must not be perm.
+ *   Errors: POETX_ERR_INVALID_ARG for n < 0, NULL arrays with n > 0, perm == inv, an entry
+ *   out of range or repeated (the detail text names it).
+ */
+int poetx_invert_perm(const int32_t* perm, int32_t n, int32_t* inv);
+
+/*
  * Permutation reduction (POET-X section 2.2): W0' = Pi_R W0 Pi_P^T, i.e.
  * W0p[i, j] = W0[perm_R[i], perm_P[j]].  Run once per outer iteration.
  *   W0   device [m, n] (dtype), read.      W0p  device [m, n] (dtype), written.
@@ -165,12 +176,14 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
  * counterpart: this entry point exists for callers that cannot allocate device memory
  * where they need G (a host framework that owns all device memory in its own pool and
  * exposes none to this call site, or a loop that must not call cudaMalloc because it
- * would synchronise the device).  Same arguments and result as poetx_cnp_fwd, minus
- * (ws, ws_bytes).
+ * would synchronise the device).  Same arguments and result as poetx_cnp_fwd (bit for
+ * bit: the same kernels on the same chunks of blocks), minus (ws, ws_bytes).
  *   Scratch: a fixed 32 MiB array of the library's own device memory, present on every
- *   GPU that loads the library until the process exits.  One block's scratch must fit
- *   it (poetx_cnp_workspace(1, b, k) <= 32 MiB: every k for b <= 512); larger b returns
- *   POETX_ERR_WORKSPACE with a message.  Any number of blocks is processed in chunks.
+ *   GPU that loads the library until the process exits.  One block's forward scratch must
+ *   fit it: (d + 2) b x b fp32 matrices plus 64 bytes of counters and a fixed 256 bytes,
+ *   with d = floor((k + 1) / 2) -- every k <= 16 for b <= 512, k <= 5 for b = 1024;
+ *   b = 1024 with k >= 6 returns POETX_ERR_WORKSPACE with a message.  Any number of
+ *   blocks is processed in chunks.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before any
  *   stream capture.  The call allocates nothing and calls no allocating routine.
@@ -304,6 +317,43 @@ int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* d
                         float* dG_R, int accumulate, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Time limit of every bounded wait in the library's kernels (mbarrier waits of the tensor-core
+ * GEMM, dependency waits of the CNP task graph), in nanoseconds; 0 restores the default of
+ * 2 s.  Kernels read the limit when they are launched (a CUDA graph keeps the value it was
+ * captured with).  Not thread-safe against concurrent launches that expect the old value.
+ *   previous: receives the limit before this call (may be NULL).
+ *   Errors: POETX_ERR_INVALID_ARG above 60 s.
+ */
+int poetx_set_wait_limit(uint64_t ns, uint64_t* previous);
+
+/*
+ * Self-test of the bounded waits (no counterpart in the pages): runs the CNP forward task
+ * graph of nblk blocks with the done-counter of block 0's first step started far below
+ * reach, so the first item that depends on it waits until the time limit, records
+ * POETX_ERR_TIMEOUT in the device flag and the launch returns.  Nothing faults and nothing
+ * waits without a bound; G holds partial results afterwards.  poetx_device_status then
+ * reports (and clears) the timeout, and later calls run normally.
+ *   theta device fp32 [nblk, b(b-1)/2], G device fp32 [nblk, b, b] (written, partially).
+ *   ws: scratch holding every block at once: nblk * (d + 2) b x b fp32 matrices (d =
+ *   floor((k + 1) / 2)) plus 64 bytes of counters per block and 256 bytes;
+ *   poetx_cnp_workspace(nblk, b, k) is enough whenever nblk * b * b * 4 <= 256 MiB.
+ *   Shapes: b % 64 == 0 and k <= 6 (the task-graph shapes), nblk >= 1.
+ *   Errors: INVALID_ARG, SHAPE, ALIGN, WORKSPACE, CUDA.
+ */
+int poetx_selftest_wait_timeout(const float* theta, float* G, int32_t nblk, int32_t b, int32_t k,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * FP32 FMA throughput probe (no counterpart in the pages; the measured peak of the pipe that
+ * bounds the SIMT CNP kernels): one launch of `ctas` CTAs x 512 threads, every thread running
+ * 16 independent chains of `iters` fused multiply-adds, i.e. ctas * 512 * 16 * iters * 2
+ * FLOPs.  Time it with events on `stream`.
+ *   out: device fp32 [ctas * 512], written (the chains' sums).
+ *   Errors: INVALID_ARG, ALIGN, CUDA.
+ */
+int poetx_fma_probe(float* out, int32_t ctas, int32_t iters, void* stream);
+
+/*
  * Reads and clears the device-side error flag that kernels with bounded barrier waits
  * set on a timeout.  Synchronises the given stream first.  Returns POETX_OK or
  * POETX_ERR_TIMEOUT (or POETX_ERR_CUDA if the synchronisation itself failed).
@@ -316,9 +366,13 @@ int poetx_device_status(void* stream);
  *   poetx_profile_begin(name) starts bracketing every launch of the kernel family
  *   `name` ("gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm", ...) with
  *   CUDA events on the launch stream (NULL or "" turns this off); poetx_profile_end()
- *   synchronises those events and reports the number of bracketed launches and their
- *   summed device time in milliseconds.  Events come from a fixed pool of 32768 pairs;
- *   launches beyond it are not bracketed (the count reports how many were).
+ *   stops bracketing, synchronises those events and reports the number of bracketed
+ *   launches and their summed device time in milliseconds.  Launches made while the
+ *   stream is captured into a CUDA graph get event nodes in the graph: each replay of the
+ *   graph records them again, and a further poetx_profile_end() (without a new
+ *   poetx_profile_begin) reports the launches of the latest replay.  Events come from a
+ *   fixed pool of 32768 pairs; launches beyond it are not bracketed (the count reports
+ *   how many were).
  */
 uint64_t poetx_launch_count(void);
 int poetx_profile_begin(const char* name);

@@ -48,7 +48,6 @@ static_assert(kRedFloats + kMirFloats <= kRingFloats,
 static_assert(kPairFloats <= kSmemFloats, "symmetrising job staging must fit");
 constexpr int kSmemBytes = kSmemFloats * 4;
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 227 * 1024, "shared memory per SM");
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;  // 64 x 64 tile-pair jobs
 
 __device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
@@ -585,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
         while (ld_acquire(cnt) < need) {
           if ((++spins & 31u) == 0) {
             if (*reinterpret_cast<volatile int*>(g.err) != 0 ||
-                gtimer() - t0 > kWaitLimitNs) {
+                gtimer() - t0 > g.wait_ns) {
               atomicCAS(g.err, 0, (int)POETX_ERR_TIMEOUT);
               s_ok = 0;
               break;
@@ -610,10 +609,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
   }
 }
 
-__global__ void k_zero_ints(int* p, int n) {
+// p[0] = first, p[1..n) = 0
+__global__ void k_zero_ints(int* p, int n, int first) {
   pdl_trigger();
   pdl_wait();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    p[i] = i == 0 ? first : 0;
 }
 
 }  // namespace
@@ -642,10 +643,12 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
       return cudaErrorInvalidValue;
   }
   g.err = device_error_flag();
+  if (!g.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
+  g.wait_ns = wait_limit_ns();
   const int ncount = g.njobs * g.nblk + 1;
   begin_launch("cnp_elementwise", s);
   cudaError_t e = launch_pdl(k_zero_ints, dim3((ncount + 255) / 256), dim3(256), 0, s,
-                             g.counters, ncount);
+                             g.counters, ncount, g.first_counter);
   end_launch("cnp_elementwise", s);
   if (e != cudaSuccess) return e;
   // persistent grid: never more CTAs than can be resident at once

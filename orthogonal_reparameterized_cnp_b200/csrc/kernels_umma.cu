@@ -23,7 +23,8 @@
 // griddepcontrol.wait, global memory only after it.  Operands may be K-major or MN-major (transposed) in global memory; both
 // are staged with the 128-byte swizzle the UMMA smem descriptors expect.
 //
-// Every mbarrier wait is bounded: after kWaitLimitNs the waiting role records
+// Every mbarrier wait is bounded: after the wait limit (Params::wait_ns, 2 s unless the
+// library's poetx_set_wait_limit changed it) the waiting role records
 // POETX_ERR_TIMEOUT in a device flag and leaves its loop; the CTA then drains its
 // outstanding TMA loads and MMAs (again with bounded waits), frees TMEM and returns.
 // No cluster multicast is used anywhere.
@@ -42,7 +43,6 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 constexpr int kThreads = 320;  // 2 control warps + 8 epilogue warps
 constexpr int kEpiWarps = 8;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // B_RES: the B operand of a whole item (K <= 256) stays in shared memory while the CTA
 // works through consecutive items that share it (the block-diagonal products: one G_j
@@ -69,6 +69,7 @@ struct Params {
   int out_f32;
   long long ldd, d_boff_col, d_boff, d_split;
   int* err;
+  unsigned long long wait_ns;  // bound of every mbarrier wait
   int y_per_bz, y_per_split;  // output tensor rows per batch entry / per split
 };
 
@@ -103,14 +104,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   return t;
 }
 // Bounded wait: false after a timeout (flag set) or when another CTA reported a failure.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err,
+                                       unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   unsigned spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 63u) == 0) {
       if (*reinterpret_cast<volatile int*>(err) != 0) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         atomicCAS(err, 0, (int)POETX_ERR_TIMEOUT);
         return false;
       }
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key = b_key(p, item);
         if (key != cur_key) {
           ++brun;
-          if (!mbar_wait(bempty_bar, (brun & 1) ^ 1, p.err)) {
+          if (!mbar_wait(bempty_bar, (brun & 1) ^ 1, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int kc = kc0; kc < kc1; ++kc, ++it) {
         const int s = it % C::STAGES, r = it / C::STAGES;
-        if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err)) {
+        if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -444,14 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         key = b_key(p, item);
         if (key != cur_key) {
           ++brun;
-          if (!mbar_wait(bfull_bar, brun & 1, p.err)) {
+          if (!mbar_wait(bfull_bar, brun & 1, p.err, p.wait_ns)) {
             ok = false;
             break;
           }
           cur_key = key;
         }
       }
-      if (!mbar_wait(tempty_bar(acc), (ra & 1) ^ 1, p.err)) {
+      if (!mbar_wait(tempty_bar(acc), (ra & 1) ^ 1, p.err, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
       for (int kc = kc0; kc < kc1; ++kc, ++it) {
         const int s = it % C::STAGES, r = it / C::STAGES;
-        if (!mbar_wait(full_bar(s), r & 1, p.err)) {
+        if (!mbar_wait(full_bar(s), r & 1, p.err, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -504,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = tcount & 1, ra = tcount >> 1;
       // one lane waits so that the warp stays converged for the .sync.aligned loads
       int ready = 0;
-      if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err) ? 1 : 0;
+      if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err, p.wait_ns) ? 1 : 0;
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (!ready) break;
       tc_fence_after();
@@ -701,6 +703,8 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   p.d_boff = g.d_boff;
   p.d_split = g.d_split;
   p.err = device_error_flag();
+  if (!p.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
+  p.wait_ns = wait_limit_ns();
   // output as a 2-D row-major tensor: batch entries / splits are row offsets (d_boff,
   // d_split multiples of ldd) or column offsets (d_boff_col)
   if (g.ldd <= 0 || g.d_boff % g.ldd != 0 || g.d_split % g.ldd != 0) return cudaErrorInvalidValue;

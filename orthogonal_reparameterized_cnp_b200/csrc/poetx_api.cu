@@ -44,6 +44,10 @@ int* device_error_flag() {
   return ptrs[dev];
 }
 
+static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};  // 2 s
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -66,18 +70,29 @@ static constexpr int kEventPairs = 32768;
 static std::vector<cudaEvent_t> g_ev_start, g_ev_stop;
 static int g_prof_used = 0;
 
+// While a stream is being captured into a CUDA graph the events are recorded as event
+// nodes of the graph (cudaEventRecordExternal), so every replay of the graph re-records
+// them and the elapsed times describe the launches of the latest replay.
+static void record_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, s);
+}
+
 void begin_launch(const char* family, cudaStream_t s) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (!g_prof_on) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (g_prof_on && g_prof_family == family && g_prof_used < kEventPairs)
-    cudaEventRecord(g_ev_start[g_prof_used], s);
+    record_event(g_ev_start[g_prof_used], s);
 }
 void end_launch(const char* family, cudaStream_t s) {
   if (!g_prof_on) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (g_prof_on && g_prof_family == family && g_prof_used < kEventPairs)
-    cudaEventRecord(g_ev_stop[g_prof_used++], s);
+    record_event(g_ev_stop[g_prof_used++], s);
 }
 
 // ------------------------------------------------------------------ helpers
@@ -173,6 +188,13 @@ int cnp_chunks(int nblk, int b, int k, bool backward, void* ws, size_t ws_bytes,
   return POETX_OK;
 }
 
+}  // namespace
+
+size_t cnp_fwd_block_bytes(int b, int k) { return cnp_per_block(b, k, false); }
+size_t cnp_fixed_bytes() { return kCnpFixedBytes; }
+
+namespace {
+
 SgemmArgs sq_gemm(const float* A, int tA, const float* B, int tB, float* C, int nb, int b,
                   int mode) {
   SgemmArgs g;
@@ -231,6 +253,36 @@ int poetx_make_perm(uint64_t seed, int32_t n, int32_t* perm, int32_t* inv) {
   }
   if (inv)
     for (int32_t i = 0; i < n; ++i) inv[perm[i]] = i;
+  return POETX_OK;
+}
+
+int poetx_invert_perm(const int32_t* perm, int32_t n, int32_t* inv) {
+  if (n < 0) return fail(POETX_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return POETX_OK;
+  if (!perm || !inv) return fail(POETX_ERR_INVALID_ARG, "perm and inv must be given");
+  if (perm == inv) return fail(POETX_ERR_INVALID_ARG, "perm and inv must be distinct arrays");
+  // every index in range and taken once: the map is a bijection of {0..n-1}
+  std::vector<unsigned char> seen((size_t)n, 0);
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t p = perm[i];
+    if (p < 0 || p >= n)
+      return fail(POETX_ERR_INVALID_ARG, "perm[" + std::to_string(i) + "] = " +
+                                             std::to_string(p) + " is outside [0, n)");
+    if (seen[(size_t)p])
+      return fail(POETX_ERR_INVALID_ARG, "perm is not a bijection: index " + std::to_string(p) +
+                                             " appears twice");
+    seen[(size_t)p] = 1;
+  }
+  for (int32_t i = 0; i < n; ++i) inv[perm[i]] = i;
+  return POETX_OK;
+}
+
+int poetx_set_wait_limit(uint64_t ns, uint64_t* previous) {
+  if (ns > 60ull * 1000000000ull)
+    return fail(POETX_ERR_INVALID_ARG, "wait limit above 60 s");
+  const unsigned long long v = ns ? ns : 2000000000ull;
+  const unsigned long long old = g_wait_limit_ns.exchange(v);
+  if (previous) *previous = old;
   return POETX_OK;
 }
 
@@ -349,12 +401,13 @@ void graph_powers(CnpGraph& g, int jQ, const float* Q, float* const* Pw, float* 
 
 int run_fwd_graph(const float* theta, const float* Q, float* const* Pw, float* Fp, float* G,
                   __nv_bfloat16* Gb, int* counters, const CnpPoly& P, int nb, int b,
-                  cudaStream_t s) {
+                  cudaStream_t s, int first_counter = 0) {
   const int d = P.d;
   CnpGraph g;
   g.nblk = nb;
   g.b = b;
   g.counters = counters;
+  g.first_counter = first_counter;
   CnpJob ex;
   ex.type = JOB_EXPAND;
   ex.A = theta;
@@ -721,6 +774,33 @@ int poetx_cnp_bwd_saved(const float* theta, const float* dG, const float* Q_save
     return fail(POETX_ERR_INVALID_ARG, "null pointer");
   return cnp_bwd_impl(theta, dG, Q_saved, S_saved, F_saved, dtheta, nblk, b, k, ws, ws_bytes,
                       stream);
+}
+
+int poetx_selftest_wait_timeout(const float* theta, float* G, int32_t nblk, int32_t b, int32_t k,
+                                void* ws, size_t ws_bytes, void* stream) {
+  int st = cnp_validate(theta, G, nblk, b, k);
+  if (st != POETX_OK) return st;
+  if (nblk < 1) return fail(POETX_ERR_INVALID_ARG, "nblk must be >= 1");
+  if (!cnp_graph_ok(b, k))
+    return fail(POETX_ERR_SHAPE, "the self-test needs the task-graph shapes (b % 64 == 0, k <= 6)");
+  if (!aligned16(theta) || !aligned16(G)) return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const size_t per = cnp_per_block(b, k, false);
+  if (!ws || ws_bytes < (size_t)nblk * per + kCnpFixedBytes)
+    return fail(POETX_ERR_WORKSPACE, "self-test scratch must hold every block (no chunking)");
+  if (!aligned16(ws)) return fail(POETX_ERR_ALIGN, "scratch must be 16-byte aligned");
+  const CnpPoly P = cnp_poly(k);
+  const int d = P.d;
+  const int64_t bb = (int64_t)b * b;
+  Carve cv(ws);
+  float* Q = static_cast<float*>(cv.take(bb * 4 * nblk));
+  std::vector<float*> Pw(d + 1, nullptr);
+  for (int j = 1; j <= d; ++j) Pw[j] = static_cast<float*>(cv.take(bb * 4 * nblk));
+  float* Fp = static_cast<float*>(cv.take(bb * 4 * nblk));
+  int* counters = static_cast<int*>(cv.take(kCnpCounterBytesPerBlock * nblk + 4));
+  // the expansion of block 0 can never be counted as done, so the first item that reads
+  // it waits until the time limit
+  return run_fwd_graph(theta, Q, Pw.data(), Fp, G, nullptr, counters, P, nblk, b,
+                       static_cast<cudaStream_t>(stream), INT32_MIN / 2);
 }
 
 }  // extern "C"

@@ -23,11 +23,20 @@ int cuda_fail(cudaError_t e, const char* what);
 void begin_launch(const char* family, cudaStream_t s);
 void end_launch(const char* family, cudaStream_t s);
 
-// Device error flag (set by kernels whose bounded waits time out).
+// Device error flag (set by kernels whose bounded waits time out).  nullptr when the flag's
+// device address cannot be looked up; launchers then refuse to launch.
 int* device_error_flag();
+
+// Time limit of every bounded wait in the kernels, in nanoseconds (poetx_set_wait_limit).
+unsigned long long wait_limit_ns();
 
 // Number of SMs of the current device.
 int num_sms();
+
+// CNP forward scratch: bytes per block (its matrices and task-graph counters) and the
+// fixed part of a call (the chunking of poetx_cnp_fwd works in these units).
+size_t cnp_fwd_block_bytes(int b, int k);
+size_t cnp_fixed_bytes();
 
 // ---- programmatic dependent launch ------------------------------------------------
 // Kernels of the layer step are launched so that a kernel may start (and do its set-up)
@@ -178,6 +187,11 @@ struct CnpGraph {
   int item_start[kCnpMaxJobs + 1] = {0};
   int* counters = nullptr;  // scratch: njobs * nblk done-counters + 1 ticket
   int* err = nullptr;
+  unsigned long long wait_ns = 0;  // bound of every dependency wait
+  // initial value of the done-counter of job 0, block 0 (0 in every product call; the
+  // wait-timeout self-test starts it far below reach so that the first dependent item's
+  // wait runs out)
+  int first_counter = 0;
 };
 // Zeroes the counters and runs the graph (two launches).
 cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s);

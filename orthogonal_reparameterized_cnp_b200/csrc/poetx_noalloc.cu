@@ -50,9 +50,10 @@ extern "C" int poetx_cnp_fwd_static(const float* theta, float* G, void* G_bf16, 
   if (nblk < 0) return poetx::fail(POETX_ERR_INVALID_ARG, "nblk must be >= 0");
   if (b < 1 || b > 1024 || k < 1 || k > 16)
     return poetx::fail(POETX_ERR_SHAPE, "block size b must be in [1, 1024], k in [1, 16]");
-  // One block's scratch must fit the fixed array; larger counts run in chunks inside it.
-  const size_t one_block = poetx_cnp_workspace(1, b, k);
-  if (one_block == 0 || one_block > kStaticScratchBytes)
+  // One block's forward scratch (its d + 2 matrices and counters, plus the call's fixed
+  // part) must fit the fixed array; larger counts run in chunks inside it.
+  const size_t one_block = poetx::cnp_fwd_block_bytes(b, k) + poetx::cnp_fixed_bytes();
+  if (one_block > kStaticScratchBytes)
     return poetx::fail(POETX_ERR_WORKSPACE,
                        "poetx_cnp_fwd_static: one block of size b=" + std::to_string(b) +
                            ", k=" + std::to_string(k) + " needs " + std::to_string(one_block) +

@@ -34,8 +34,8 @@ def allreduce_dtheta(dtheta, group=None) -> None:
 
 
 def dp_step(layer, x, dy, y, dx, stream=None, group=None) -> None:
-    """One data-parallel step of a PoetxLinear on this rank's tokens: the whole path
-    (merge, CNP forward, layer forward and backward, CNP backward), then the all-reduce
-    of dtheta."""
+    """One data-parallel step of a PoetxLinear (or, with lists of tensors, a
+    PoetxLinearGroup) on this rank's tokens: CNP forward, layer forward and backward, CNP
+    backward, then the all-reduce of dtheta (every block of the layer or group at once)."""
     layer.step(x, dy, y, dx, stream)
-    allreduce_dtheta(layer.dtheta, group)
+    allreduce_dtheta(layer.cnp.dtheta if hasattr(layer, "layers") else layer.dtheta, group)

@@ -46,6 +46,7 @@ SIGNATURES = {
     "poetx_last_error": (ctypes.c_char_p, []),
     "poetx_version": (ctypes.c_char_p, []),
     "poetx_make_perm": (_c_int, [_c_u64, _c_i32, _i32p, _i32p]),
+    "poetx_invert_perm": (_c_int, [_i32p, _c_i32, _i32p]),
     "poetx_merge_perm": (_c_int, [_vp, _vp, _c_i32, _c_i32, _vp, _vp, _c_int, _vp]),
     "poetx_permute_cols": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
     "poetx_outer_merge_workspace": (_c_size, [_c_i32, _c_i32, _c_int]),
@@ -66,6 +67,10 @@ SIGNATURES = {
     "poetx_linear_bwd": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                   _vp, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "poetx_device_status": (_c_int, [_vp]),
+    "poetx_set_wait_limit": (_c_int, [_c_u64, ctypes.POINTER(_c_u64)]),
+    "poetx_selftest_wait_timeout": (_c_int, [_vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size,
+                                             _vp]),
+    "poetx_fma_probe": (_c_int, [_vp, _c_i32, _c_i32, _vp]),
     "poetx_quantize_rows": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
     "poetx_linear_q8_scratch": (_c_size, [ctypes.POINTER(LinearDesc)]),
     "poetx_linear_fwd_q8": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp,
@@ -150,6 +155,26 @@ def make_perm(seed: int, n: int):
                              perm.ctypes.data_as(_i32p), inv.ctypes.data_as(_i32p)),
            "poetx_make_perm")
     return perm, inv
+
+
+def invert_perm(perm) -> np.ndarray:
+    """Inverse of an index map (numpy int32), computed and validated by the library: a map
+    that is not a bijection of range(n) raises PoetxError (POETX_ERR_INVALID_ARG)."""
+    L = _load()
+    p = np.ascontiguousarray(np.asarray(perm), dtype=np.int32)
+    if p.ndim != 1:
+        raise ValueError("an index map is a 1-D array")
+    inv = np.empty_like(p)
+    _check(L.poetx_invert_perm(p.ctypes.data_as(_i32p), len(p), inv.ctypes.data_as(_i32p)),
+           "poetx_invert_perm")
+    return inv
+
+
+def set_wait_limit(ns: int) -> int:
+    """Sets the kernels' bounded-wait limit (0: the 2 s default); returns the previous one."""
+    prev = _c_u64(0)
+    _check(_load().poetx_set_wait_limit(int(ns), ctypes.byref(prev)), "poetx_set_wait_limit")
+    return int(prev.value)
 
 
 def cnp_workspace(nblk: int, b: int, k: int) -> int:
@@ -320,65 +345,121 @@ def linear_bwd_q8(desc: LinearDesc, x, dy, G_P, G_R, W0q, scales, save_u, save_w
            "poetx_linear_bwd_q8")
 
 
+def selftest_wait_timeout(theta, G, b: int, k: int, ws, stream=None):
+    """Runs the CNP forward with a dependency that is never met (see the header)."""
+    _require_cuda()
+    nblk = theta.shape[0]
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_load().poetx_selftest_wait_timeout(_ptr(theta), _ptr(G), nblk, b, k, _ptr(ws),
+                                               ws_bytes, _stream(stream)),
+           "poetx_selftest_wait_timeout")
+
+
+def fma_probe(out, ctas: int, iters: int, stream=None):
+    """FP32 FMA throughput probe: ctas * 512 * 16 * iters * 2 FLOPs into out[ctas * 512]."""
+    _require_cuda()
+    _check(_load().poetx_fma_probe(_ptr(out), ctas, iters, _stream(stream)), "poetx_fma_probe")
+
+
 def device_status(stream=None) -> int:
     _require_cuda()
     return int(_load().poetx_device_status(_stream(stream)))
 
 
-# ------------------------------------------------------------------------ a layer object
-@dataclass
-class PoetxLinearState:
-    """Device buffers of one POET-X linear for a fixed token count (allocated by torch)."""
-    T: int
-    n: int
-    m: int
-    b: int
-    k: int
-    dtype: str
+# ------------------------------------------------------------------------ layer objects
+class CnpBuffers:
+    """Device buffers of the Cayley-Neumann parameterisation of nblk b x b blocks: theta,
+    G (fp32 and, for the bf16 layer, its bf16 copy), the upstream dG, dtheta, and the Q,
+    S = Q^2 and F' that the forward keeps for the backward.  One forward call and one
+    backward call cover every block, whichever layers the blocks belong to."""
+
+    def __init__(self, nblk: int, b: int, k: int, device, lowp_dtype=None):
+        import torch
+        self.nblk, self.b, self.k = nblk, b, k
+        f32 = dict(dtype=torch.float32, device=device)
+        ntri = b * (b - 1) // 2
+        self.theta = torch.zeros((nblk, ntri), **f32)
+        self.G = torch.empty((nblk, b, b), **f32)
+        self.G_lp = torch.empty((nblk, b, b), dtype=lowp_dtype, device=device) \
+            if lowp_dtype is not None else None
+        self.dG = torch.zeros((nblk, b, b), **f32)
+        self.dtheta = torch.empty((nblk, ntri), **f32)
+        self.Q_save = torch.empty((nblk, b, b), **f32)
+        self.S_save = torch.empty((nblk, b, b), **f32)
+        self.F_save = torch.empty((nblk, b, b), **f32)
+        self.ws = None
+        self.set_order(k)
+
+    def set_order(self, k: int):
+        """Neumann order of the following calls (the scratch is resized to it)."""
+        import torch
+        self.k = k
+        self.ws = None
+        self.ws = torch.empty(max(cnp_workspace(self.nblk, self.b, k), 16), dtype=torch.uint8,
+                              device=self.G.device)
+
+    def forward(self, stream=None):
+        cnp_fwd_save(self.theta, self.G, self.G_lp, self.Q_save, self.S_save, self.F_save,
+                     self.b, self.k, self.ws, stream)
+
+    def backward(self, stream=None):
+        """dtheta from dG; reads the Q, S and F' of the last forward (theta unchanged)."""
+        cnp_bwd_saved(self.theta, self.dG, self.Q_save, self.S_save, self.F_save, self.dtheta,
+                      self.b, self.k, self.ws, stream)
+
+
+def _layer_scratch_bytes(desc, save: bool, int8: bool) -> int:
+    q8 = linear_q8_scratch(desc) if int8 else 0
+    return max(linear_fwd_workspace(desc, save, save), linear_bwd_workspace(desc, save, save),
+               16) + q8
 
 
 class PoetxLinear:
     """One POET-X linear on the GPU: merged weight, CNP blocks, forward and backward.
 
     All buffers are torch tensors on the current device; every computation is a libpoetx
-    call.  ``theta`` holds the input-side blocks first, then the output-side blocks.
+    call.  The CNP blocks are the input-side blocks first, then the output-side blocks, in
+    ``cnp`` (a CnpBuffers of this layer alone unless one is shared, see PoetxLinearGroup);
+    ``theta``, ``G``, ``dG``, ``dtheta`` are this layer's rows of it.  The inverse index
+    maps come from the library, which rejects a perm_P or perm_R that is not a bijection.
+    The permutations are merged into W0' once, at construction (and again by merge()).
     """
 
     def __init__(self, W0, theta_P, theta_R, perm_P, perm_R, b: int, k: int, T: int,
-                 save_activations: bool = True, int8_weight: bool = False):
+                 save_activations: bool = True, int8_weight: bool = False, cnp=None,
+                 first_block: int = 0, ws=None):
         import torch
+        self.m, self.n = W0.shape
+        # the index maps are checked (bijections) and inverted by the library, on the host,
+        # before any device work
+        pP = np.ascontiguousarray(np.asarray(perm_P), dtype=np.int32)
+        pR = np.ascontiguousarray(np.asarray(perm_R), dtype=np.int32)
+        if pP.shape != (self.n,) or pR.shape != (self.m,):
+            raise ValueError("perm_P must have n entries and perm_R m entries")
+        iP, iR = invert_perm(pP), invert_perm(pR)
         _require_cuda()
         dev = W0.device
-        self.m, self.n = W0.shape
         self.b, self.k, self.T = b, k, T
         self.bf16 = W0.dtype == torch.bfloat16
         self.nP, self.nR = self.n // b, self.m // b
         nblk = self.nP + self.nR
-        ntri = b * (b - 1) // 2
         i32 = dict(dtype=torch.int32, device=dev)
-        pP = torch.as_tensor(np.asarray(perm_P, dtype=np.int32), **i32)
-        pR = torch.as_tensor(np.asarray(perm_R, dtype=np.int32), **i32)
-        self.perm_P, self.perm_R = pP, pR
-        self.inv_P = torch.empty_like(pP)
-        self.inv_P[pP.long()] = torch.arange(self.n, **i32)
-        self.inv_R = torch.empty_like(pR)
-        self.inv_R[pR.long()] = torch.arange(self.m, **i32)
+        self.perm_P, self.inv_P = torch.as_tensor(pP, **i32), torch.as_tensor(iP, **i32)
+        self.perm_R, self.inv_R = torch.as_tensor(pR, **i32), torch.as_tensor(iR, **i32)
         self.W0 = W0
         self.W0p = torch.empty_like(W0)
-        f32 = dict(dtype=torch.float32, device=dev)
-        self.theta = torch.empty((nblk, ntri), **f32)
+        if cnp is None:
+            cnp = CnpBuffers(nblk, b, k, dev, W0.dtype if self.bf16 else None)
+            first_block = 0
+        if cnp.b != b or cnp.k != k or first_block + nblk > cnp.nblk:
+            raise ValueError("the CNP buffers do not hold this layer's blocks")
+        self.cnp = cnp
+        rows = slice(first_block, first_block + nblk)
+        self.theta, self.G, self.dG, self.dtheta = (cnp.theta[rows], cnp.G[rows], cnp.dG[rows],
+                                                    cnp.dtheta[rows])
+        self.G_lp = cnp.G_lp[rows] if cnp.G_lp is not None else None
         self.theta[: self.nP] = theta_P
         self.theta[self.nP:] = theta_R
-        self.G = torch.empty((nblk, b, b), **f32)
-        self.G_lp = torch.empty((nblk, b, b), dtype=W0.dtype, device=dev) if self.bf16 else None
-        self.dG = torch.empty((nblk, b, b), **f32)
-        self.dtheta = torch.empty((nblk, ntri), **f32)
-        # Q, S = Q^2 and F' of the last CNP forward, read by the CNP backward of the same step
-        self.Q_save = torch.empty((nblk, b, b), **f32)
-        self.S_save = torch.empty((nblk, b, b), **f32)
-        self.F_save = torch.empty((nblk, b, b), **f32)
-        self.cnp_ws = torch.empty(max(cnp_workspace(nblk, b, k), 16), dtype=torch.uint8,
-                                  device=dev)
         self.desc = linear_desc(T, self.n, self.m, b, POETX_BF16 if self.bf16 else POETX_F32,
                                 self.perm_P, self.inv_P, self.perm_R, self.inv_R)
         act = W0.dtype
@@ -388,34 +469,36 @@ class PoetxLinear:
             self.Wsave = torch.empty((T, self.m), dtype=act, device=dev)
         else:
             self.U = self.Wsave = None
-        fwd_ws = linear_fwd_workspace(self.desc, self.save, self.save)
-        bwd_ws = linear_bwd_workspace(self.desc, self.save, self.save)
         # int8 merged weight (POET-XQ): codes + per-row scales; the bf16 weight exists only
         # inside each layer call's scratch
         self.int8 = int8_weight
-        q8 = 0
         if int8_weight:
             if not self.bf16:
                 raise ValueError("the int8 base weight needs the bf16 layer")
             self.W0q = torch.empty((self.m, self.n), dtype=torch.int8, device=dev)
-            self.scales = torch.empty((self.m,), **f32)
-            q8 = linear_q8_scratch(self.desc)
-        self.ws = torch.empty(max(fwd_ws, bwd_ws, 16) + q8, dtype=torch.uint8, device=dev)
+            self.scales = torch.empty((self.m,), dtype=torch.float32, device=dev)
+        need = _layer_scratch_bytes(self.desc, self.save, int8_weight)
+        if ws is None:
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        elif ws.numel() * ws.element_size() < need:
+            raise ValueError("shared layer scratch too small")
+        self.ws = ws
         if int8_weight:  # the bf16 merged weight is only a step of merge(): it lives in scratch
             self.W0p = self.ws[: self.m * self.n * 2].view(W0.dtype).view(self.m, self.n)
+        self.merge()
 
     def G_ops(self):
         G = self.G_lp if self.bf16 else self.G
         return G[: self.nP], G[self.nP:]
 
     def merge(self, stream=None):
+        """W0' = Pi_R W0 Pi_P^T (and its int8 codes): once per set of permutations."""
         merge_perm(self.W0, self.W0p, self.perm_R, self.perm_P, stream)
         if self.int8:
             quantize_rows(self.W0p, self.W0q, self.scales, stream)
 
     def cnp_forward(self, stream=None):
-        cnp_fwd_save(self.theta, self.G, self.G_lp, self.Q_save, self.S_save, self.F_save,
-                     self.b, self.k, self.cnp_ws, stream)
+        self.cnp.forward(stream)
 
     def forward(self, x, y, stream=None):
         GP, GR = self.G_ops()
@@ -437,14 +520,72 @@ class PoetxLinear:
 
     def cnp_backward(self, stream=None):
         """dtheta from dG; reads Q, S and F' of the last cnp_forward (theta unchanged)."""
-        cnp_bwd_saved(self.theta, self.dG, self.Q_save, self.S_save, self.F_save, self.dtheta,
-                      self.b, self.k, self.cnp_ws, stream)
+        self.cnp.backward(stream)
 
     def step(self, x, dy, y, dx, stream=None):
-        """One pass of the whole path: merge, CNP forward, layer forward and backward,
-        CNP backward."""
-        self.merge(stream)
+        """One pass of the per-step path: CNP forward, layer forward and backward, CNP
+        backward (the merge of the permutations is per set of permutations, not per step)."""
         self.cnp_forward(stream)
         self.forward(x, y, stream)
         self.backward(x, dy, dx, 0, stream)
+        self.cnp_backward(stream)
+
+
+class PoetxLinearGroup:
+    """Several POET-X linears (e.g. the seven of a decoder block) whose CNP forward and
+    backward each run as one call over all of their blocks, and whose layer calls share one
+    scratch buffer (they run one after another on one stream).
+
+    specs: list of (W0, theta_P, theta_R, perm_P, perm_R) per linear.
+    """
+
+    def __init__(self, specs, b: int, k: int, T: int, save_activations: bool = True,
+                 int8_weight: bool = False):
+        import torch
+        _require_cuda()
+        W0s = [sp[0] for sp in specs]
+        dev = W0s[0].device
+        bf16 = W0s[0].dtype == torch.bfloat16
+        nblks = [(W.shape[1] + W.shape[0]) // b for W in W0s]
+        self.cnp = CnpBuffers(sum(nblks), b, k, dev, W0s[0].dtype if bf16 else None)
+        need = 16
+        for W in W0s:
+            m, n = W.shape
+            d = LinearDesc(T, n, m, b, POETX_BF16 if bf16 else POETX_F32, None, None, None, None)
+            need = max(need, _layer_scratch_bytes(d, save_activations, int8_weight))
+        self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.layers = []
+        off = 0
+        for sp, nb in zip(specs, nblks):
+            W0, tP, tR, pP, pR = sp
+            self.layers.append(PoetxLinear(W0, tP, tR, pP, pR, b, k, T, save_activations,
+                                           int8_weight, cnp=self.cnp, first_block=off,
+                                           ws=self.ws))
+            off += nb
+        self.b, self.k, self.T = b, k, T
+
+    def merge(self, stream=None):
+        for L in self.layers:
+            L.merge(stream)
+
+    def cnp_forward(self, stream=None):
+        self.cnp.forward(stream)
+
+    def forward(self, xs, ys, stream=None):
+        for L, x, y in zip(self.layers, xs, ys):
+            L.forward(x, y, stream)
+
+    def backward(self, xs, dys, dxs, accumulate=0, stream=None):
+        for L, x, dy, dx in reversed(list(zip(self.layers, xs, dys, dxs))):
+            L.backward(x, dy, dx, accumulate, stream)
+
+    def cnp_backward(self, stream=None):
+        self.cnp.backward(stream)
+
+    def step(self, xs, dys, ys, dxs, stream=None):
+        """CNP forward (every block, one call), every layer's forward, every layer's
+        backward (last layer first), CNP backward (one call)."""
+        self.cnp_forward(stream)
+        self.forward(xs, ys, stream)
+        self.backward(xs, dys, dxs, 0, stream)
         self.cnp_backward(stream)

@@ -13,7 +13,7 @@ from poetx_inputs import (LayerShape, cnp_inputs, cnp_sweep_blocks, layer_inputs
                           workload_llama13b_block, workload_llama1b_attn, workload_llama8b_up,
                           workload_small_fp32)
 
-from .gpu_harness import host, norm_max_err, run_layer, tensor
+from .gpu_harness import host, norm_max_err, run_group, run_layer, tensor
 
 pytestmark = pytest.mark.gpu
 
@@ -305,63 +305,64 @@ def test_empty_token_set():
     assert torch.count_nonzero(layer.dG).item() == 0
 
 
-# ------------------------------------------------------------------ full-size, sampled
-def _sampled_checks(out, s, inp, rows, tol=BF16_NORM):
+# ------------------------------------------------------------------ full size, every element
+def _full_checks(out, s, inp, tol=BF16_NORM):
+    """Every output element of one linear against the full float64 oracle: y, dX, and every
+    block of dG_P, dG_R, dtheta_P, dtheta_R (normalised per tensor and per block), G to
+    CNP_ABS, and W0' bit-exact."""
     pP = out["perm_P"].astype(np.int64)
     pR = out["perm_R"].astype(np.int64)
-    W0p = ref.merge_perm(inp.W0, pR, pP)
-    G_P = ref.cnp_forward(inp.theta_P, s.b, s.k)
-    G_R = ref.cnp_forward(inp.theta_R, s.b, s.k)
-    y_ref = ref.layer_forward_rows(inp.x[rows], W0p, G_P, G_R, pP, pR)
-    dx_ref = ref.layer_backward_dx_rows(inp.dy[rows], W0p, G_P, G_R, pP, pR)
-    assert norm_max_err(out["y"][rows], y_ref) <= tol
-    assert norm_max_err(out["dx"][rows], dx_ref) <= tol
-    assert np.abs(out["G"] - np.concatenate([G_P, G_R])).max() <= CNP_ABS
-    # <dY, Y> = <dX, X> = sum <dG_P, G_P> = sum <dG_R, G_R> (linearity in each factor).
-    # These sums cancel heavily, so the error scale is the sum of |terms|, not |L|.
-    terms = inp.dy.astype(np.float64) * out["y"]
-    L = float(np.sum(terms))
-    scale = float(np.sum(np.abs(terms)))
-    G_used = out.get("G_lp", out["G"])
-    nP = s.n // s.b
-    for v in [float(np.sum(inp.x.astype(np.float64) * out["dx"])),
-              float(np.sum(out["dG_P"] * G_used[:nP])),
-              float(np.sum(out["dG_R"] * G_used[nP:]))]:
-        assert abs(v - L) <= tol * scale
-    return W0p, G_P, G_R
+    o = ref.full_step(inp.x, inp.W0, inp.theta_P, inp.theta_R, inp.dy, pP, pR, s.b, s.k)
+    assert np.array_equal(out["W0p"], o["W0p"])
+    assert np.abs(out["G"] - np.concatenate([o["G_P"], o["G_R"]])).max() <= CNP_ABS
+    errs = {key: norm_max_err(out[key], o[key])
+            for key in ["y", "dx", "dG_P", "dG_R", "dtheta_P", "dtheta_R"]}
+    bad = {kk: v for kk, v in errs.items() if not v <= tol}
+    assert not bad, f"{s.name}: normalised max errors above {tol}: {errs}"
+    worst = {}
+    for key in ["dG_P", "dG_R", "dtheta_P", "dtheta_R"]:
+        per_block = [norm_max_err(out[key][j], o[key][j]) for j in range(len(o[key]))]
+        worst[key] = max(per_block)
+        assert worst[key] <= tol, f"{s.name}: {key} block {int(np.argmax(per_block))}: " \
+                                  f"{worst[key]:.3e} > {tol}"
+    return errs, worst
 
 
-def _block_grad_checks(out, s, inp, W0p, G_P, G_R, jR, jP):
-    pP = out["perm_P"].astype(np.int64)
-    pR = out["perm_R"].astype(np.int64)
-    gP, gR = ref.layer_block_grads(inp.x, inp.dy, W0p, G_P, G_R, pP, pR, jR, jP)
-    assert norm_max_err(out["dG_R"][jR], gR) <= BF16_NORM
-    assert norm_max_err(out["dG_P"][jP], gP) <= BF16_NORM
-    dthR = ref.cnp_backward(inp.theta_R[jR:jR + 1], gR[None], s.b, s.k)[0]
-    dthP = ref.cnp_backward(inp.theta_P[jP:jP + 1], gP[None], s.b, s.k)[0]
-    assert norm_max_err(out["dtheta_R"][jR], dthR) <= BF16_NORM
-    assert norm_max_err(out["dtheta_P"][jP], dthP) <= BF16_NORM
-
-
-def test_layer_bf16_llama8b_up_sampled():
-    """n = 4096 -> m = 14336, b = 256, T = 16384: sampled rows of y and dX, the inner
-    product identities, and the first/last blocks' dG over all tokens."""
+@pytest.mark.slow
+def test_layer_bf16_llama8b_up_full():
+    """n = 4096 -> m = 14336, b = 256, T = 16384: every element of y and dX and every one of
+    the 16 + 56 blocks of dG and dtheta against the full float64 oracle."""
     s = workload_llama8b_up()
     inp = layer_inputs(s)
     out = run_layer(inp)
-    rng = np.random.default_rng(3)
-    rows = np.sort(np.concatenate([[0, s.T - 1], rng.choice(s.T, 62, replace=False)]))
-    W0p, G_P, G_R = _sampled_checks(out, s, inp, rows)
-    _block_grad_checks(out, s, inp, W0p, G_P, G_R, s.m // s.b - 1, 0)
+    out.pop("layer")
+    _full_checks(out, s, inp)
 
 
-@pytest.mark.parametrize("idx", range(7))
-def test_layer_bf16_llama13b_block_sampled(idx):
-    s = workload_llama13b_block()[idx]
-    inp = layer_inputs(s)
-    out = run_layer(inp)
-    rng = np.random.default_rng(idx)
-    rows = np.sort(np.concatenate([[0, s.T - 1], rng.choice(s.T, 30, replace=False)]))
-    W0p, G_P, G_R = _sampled_checks(out, s, inp, rows)
-    nP, nR = s.n // s.b, s.m // s.b
-    _block_grad_checks(out, s, inp, W0p, G_P, G_R, (5 * idx + 1) % nR, (3 * idx) % nP)
+@pytest.mark.slow
+def test_layer_bf16_llama13b_block_full():
+    """The 7 linears of the 13B decoder block as one group (one CNP call over all 382
+    blocks, as the bench runs it): every element of every linear's y and dX and every
+    block of its dG and dtheta against the full float64 oracle."""
+    shapes = workload_llama13b_block()
+    inps = [layer_inputs(s) for s in shapes]
+    outs, g = run_group(inps)
+    del g
+    for s, inp, out in zip(shapes, inps, outs):
+        _full_checks(out, s, inp)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_group_matches_separate_layers_bit_for_bit(dtype):
+    """One CNP call over the blocks of several linears and a shared layer scratch give
+    exactly what separate layers (each with its own CNP call and scratch) give."""
+    b = 128 if dtype == "bf16" else 32
+    shapes = [LayerShape(f"grp{i}", T=300, n=n, m=m, b=b, k=4, dtype=dtype, config_id=400,
+                         linear_id=i)
+              for i, (n, m) in enumerate([(256, 256), (256, 512), (512, 256)])]
+    inps = [layer_inputs(s) for s in shapes]
+    outs, g = run_group(inps)
+    for inp, o in zip(inps, outs):
+        r = run_layer(inp)
+        for key in ["W0p", "G", "y", "dx", "dG_P", "dG_R", "dtheta_P", "dtheta_R"]:
+            assert np.array_equal(o[key], r[key]), key

@@ -168,3 +168,72 @@ def test_int8_weight_validation_before_launch():
 def test_profile_and_launch_counter_without_launches():
     n0 = P.launch_count()
     assert P.launch_count() == n0
+
+
+def test_invert_perm_matches_the_generators_inverse():
+    for seed, n in [(0, 1), (7, 64), (123, 5120)]:
+        p, inv = P.make_perm(seed, n)
+        assert np.array_equal(P.invert_perm(p), inv)
+    assert P.invert_perm(np.zeros(0, dtype=np.int32)).shape == (0,)
+
+
+def test_invert_perm_rejects_maps_that_are_not_bijections():
+    lib = P.lib()
+    with pytest.raises(P.PoetxError) as e:
+        P.invert_perm([0, 2, 2, 1])              # 2 twice, 3 missing
+    assert e.value.status == P.POETX_ERR_INVALID_ARG and "twice" in str(e.value)
+    with pytest.raises(P.PoetxError) as e:
+        P.invert_perm([0, 1, 4])                 # out of range
+    assert e.value.status == P.POETX_ERR_INVALID_ARG and "outside" in str(e.value)
+    with pytest.raises(P.PoetxError):
+        P.invert_perm([-1, 0])
+    a = (ctypes.c_int32 * 3)(0, 1, 2)
+    assert lib.poetx_invert_perm(a, 3, a) == P.POETX_ERR_INVALID_ARG   # in place
+    assert lib.poetx_invert_perm(None, 3, a) == P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_invert_perm(a, -1, a) == P.POETX_ERR_INVALID_ARG
+    # nothing is written when the map is rejected
+    inv = (ctypes.c_int32 * 3)(-7, -7, -7)
+    bad = (ctypes.c_int32 * 3)(1, 1, 0)
+    assert lib.poetx_invert_perm(bad, 3, inv) == P.POETX_ERR_INVALID_ARG
+    assert list(inv) == [-7, -7, -7]
+
+
+def test_layer_object_validates_index_maps_before_any_device_work():
+    # PoetxLinear takes the inverse maps from the library; a map with a duplicate entry is
+    # rejected there (the CUDA check comes after, so this holds without a GPU too)
+    with pytest.raises(P.PoetxError) as e:
+        P.PoetxLinear.__init__(object.__new__(P.PoetxLinear), _FakeW0(), None, None,
+                               [0, 0, 1, 2], [0, 1, 2, 3], 2, 4, 8)
+    assert e.value.status == P.POETX_ERR_INVALID_ARG and "bijection" in str(e.value)
+
+
+class _FakeW0:
+    shape = (4, 4)
+    device = "cpu"
+    dtype = None
+
+
+def test_wait_limit_setter():
+    prev = P.set_wait_limit(50_000_000)
+    try:
+        assert P.set_wait_limit(0) == 50_000_000   # 0 restores the 2 s default
+        assert P.set_wait_limit(0) == 2_000_000_000
+        with pytest.raises(P.PoetxError):
+            P.set_wait_limit(61 * 10 ** 9)
+    finally:
+        P.set_wait_limit(prev)
+
+
+def test_new_entry_points_validate_before_launch():
+    lib = P.lib()
+    f = ctypes.c_void_p(0x90000)
+    assert lib.poetx_fma_probe(f, 0, 10, None) == P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_fma_probe(None, 1, 10, None) == P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_fma_probe(ctypes.c_void_p(0x90004), 1, 10, None) == P.POETX_ERR_ALIGN
+    # the timeout self-test runs only on task-graph shapes and needs room for every block
+    assert lib.poetx_selftest_wait_timeout(f, f, 2, 100, 4, f, 1 << 30, None) == \
+        P.POETX_ERR_SHAPE
+    assert lib.poetx_selftest_wait_timeout(f, f, 2, 64, 4, f, 1024, None) == \
+        P.POETX_ERR_WORKSPACE
+    assert lib.poetx_selftest_wait_timeout(f, f, 0, 64, 4, f, 1 << 30, None) == \
+        P.POETX_ERR_INVALID_ARG

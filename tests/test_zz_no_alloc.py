@@ -2,7 +2,9 @@
 device memory (their device memory belongs to a host framework's pool they cannot reach
 from the call site, or the call sits in a loop where cudaMalloc would synchronise the
 device).  Its scratch is a fixed array of the library's own device memory instead of a
-caller buffer.  Checked through the C ABI against poetx_cnp_fwd on two calls in a row.
+caller buffer.  Checked through the C ABI on two calls in a row: bit for bit against
+poetx_cnp_fwd (the same kernels on the same chunks of blocks) and against the float64
+oracle within the CNP bar.
 
 This file is collected last on purpose (the name sorts after the others).
 """
@@ -10,6 +12,8 @@ import ctypes
 
 import numpy as np
 import pytest
+
+from oracle import poetx_ref as ref
 
 pytestmark = pytest.mark.gpu
 
@@ -40,11 +44,12 @@ def test_static_scratch_forward_matches_buffered_forward(P):
     lib = P.lib()
     stream = torch.cuda.current_stream().cuda_stream
     # first call: 40 blocks of 256 need two passes through the 32 MiB array;
-    # second call: other sizes, reusing the array the first call left behind
-    for nblk, b, k, seed in [(40, 256, 4, 1), (7, 64, 6, 2)]:
+    # second call: other sizes, reusing the array the first call left behind;
+    # third call: b = 1024, one block per pass (its forward scratch is 16 MiB + counters)
+    for nblk, b, k, seed in [(40, 256, 4, 1), (7, 64, 6, 2), (2, 1024, 4, 3)]:
         rng = np.random.default_rng(seed)
-        theta = torch.from_numpy(
-            (rng.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)).cuda()
+        th_np = (rng.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+        theta = torch.from_numpy(th_np).cuda()
         G_ref, Gb_ref = _buffered(P, theta, nblk, b, k)
         G = torch.full((nblk, b, b), float("nan"), dtype=torch.float32, device="cuda")
         Gb = torch.zeros((nblk, b, b), dtype=torch.bfloat16, device="cuda")
@@ -53,12 +58,18 @@ def test_static_scratch_forward_matches_buffered_forward(P):
         assert st == P.POETX_OK, lib.poetx_last_error()
         torch.cuda.synchronize()
         assert P.device_status() == P.POETX_OK
-        assert (G - G_ref).abs().max().item() <= CNP_ABS
-        assert (Gb.float() - Gb_ref.float()).abs().max().item() <= 2 ** -7
+        assert torch.equal(G, G_ref)
+        assert torch.equal(Gb, Gb_ref)
+        # the oracle on the first and the last block
+        for j in (0, nblk - 1):
+            G_o = ref.cnp_forward(th_np[j:j + 1], b, k)[0]
+            assert np.abs(G[j].double().cpu().numpy() - G_o).max() <= CNP_ABS
 
 
 def test_static_scratch_rejects_blocks_above_its_size(P):
     lib = P.lib()
     fake = ctypes.c_void_p(0x10000)
-    assert lib.poetx_cnp_fwd_static(fake, fake, None, 1, 1024, 4, None) == P.POETX_ERR_WORKSPACE
+    # b = 1024, k = 16: 10 matrices of 4 MiB per block do not fit the 32 MiB array
+    assert lib.poetx_cnp_fwd_static(fake, fake, None, 1, 1024, 16, None) == P.POETX_ERR_WORKSPACE
     assert b"fixed" in lib.poetx_last_error()
+    assert lib.poetx_cnp_fwd_static(fake, fake, None, 1, 1024, 6, None) == P.POETX_ERR_WORKSPACE
