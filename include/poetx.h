@@ -298,6 +298,19 @@ int poetx_quantize_rows(const void* W, int8_t* q, float* scales, int32_t m, int3
                         void* stream);
 
 /*
+ * Permutation reduction straight into the int8 merged weight (POET-X section 2.2 with the
+ * section 2.6 base weight): the codes and scales that poetx_quantize_rows gives for
+ * W0' = Pi_R W0 Pi_P^T, bit for bit, without forming W0' in high precision.  A permutation
+ * of a row does not change its largest magnitude, so row i's scale is that of source row
+ * perm_R[i]; each source row is staged on chip and gathered there.
+ *   W0 device [m, n] (dtype POETX_BF16 or POETX_F32), read; perm_R device int32 [m],
+ *   perm_P device int32 [n]; W0q device int8 [m, n], scales device fp32 [m], written.
+ *   Rows up to 200 KB (n * element size).  Errors: INVALID_ARG, SHAPE, DTYPE, ALIGN, CUDA.
+ */
+int poetx_merge_perm_q8(const void* W0, int8_t* W0q, float* scales, int32_t m, int32_t n,
+                        const int32_t* perm_R, const int32_t* perm_P, int dtype, void* stream);
+
+/*
  * The bf16 layer with the int8 merged weight (codes and scales from poetx_quantize_rows
  * of W0').  Each call first writes bf16(scales[i] * q[i, j]) into the first
  * poetx_linear_q8_scratch(d) bytes of ws (for that call only), then runs

@@ -6,6 +6,16 @@
 // jobs it reads have finished for its own block (per-(job, block) counters), so the
 // blocks flow through the chain independently and no launch boundary separates steps.
 //
+// Two shapes of product item:
+//   * 64 x 64 output tiles, 512 threads, K split over four 128-thread groups whose partial
+//     tiles are summed through shared memory in a fixed order; one CTA per SM.  Used when
+//     the call has few blocks (a level of the chain then still has ~one item per SM).
+//   * 128 x 128 output tiles, 256 threads, one 8 x 8 register tile per thread over the
+//     whole K (no partial-tile reduction), structured epilogue straight from registers;
+//     two CTAs per SM, so one CTA's operand waits and epilogue overlap the other's FMAs.
+//     Used when the call has enough blocks to fill the GPU with these larger items.
+// The elementwise jobs work on 64 x 64 tile pairs in both.
+//
 // Deadlock freedom: tickets are taken in increasing order by CTAs that are running, and
 // an item only waits on items with smaller tickets, so the lowest unfinished ticket can
 // always run (the grid is also sized to the CTAs that fit on the GPU at once).  Every wait is bounded anyway: after the
@@ -20,13 +30,12 @@
 namespace poetx {
 namespace {
 
+// ---- 64 x 64 items ------------------------------------------------------------------
 // kGroups groups of 128 threads per CTA; in a product tile every group accumulates the
 // whole 64 x 64 tile over its own share of K (own cp.async ring), then the partial tiles
-// are summed through shared memory in a fixed order.  kCtasPerSm CTAs share an SM so that
-// one item's load / epilogue latency overlaps another item's arithmetic.
+// are summed through shared memory in a fixed order.
 constexpr int kGroups = 4;
 constexpr int kThreads = kGroups * 128;
-constexpr int kCtasPerSm = 4 / kGroups;
 constexpr int kGThreads = 128;
 constexpr int kBK = 16;
 constexpr int kLD = 64 + 4;
@@ -47,8 +56,37 @@ static_assert(kRedFloats + kMirFloats <= kRingFloats,
               "partial tiles and mirror staging must fit in the ring region");
 static_assert(kPairFloats <= kSmemFloats, "symmetrising job staging must fit");
 constexpr int kSmemBytes = kSmemFloats * 4;
-static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 227 * 1024, "shared memory per SM");
-constexpr int kPT = 64, kPLD = 65, kPRows = kThreads / kPT;  // 64 x 64 tile-pair jobs
+static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory per SM");
+constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
+
+// ---- 128 x 128 items ----------------------------------------------------------------
+constexpr int k2Threads = 256;  // 16 x 16 threads, 8 x 8 outputs each
+constexpr int k2BK = 16;
+constexpr int k2LD = 128 + 4;  // row stride of a staged k slice (16-byte aligned rows)
+constexpr int k2Stages = 4;
+constexpr int k2StageFloats = 2 * k2BK * k2LD;
+constexpr int k2RingFloats = k2Stages * k2StageFloats;  // 66 KB
+// epilogue operands (the adds and the skew term, <= 3 tiles) of one 64 x 64 quadrant are
+// staged in shared memory, two quadrants in flight (reusing the ring after the main loop)
+constexpr int k2QLD = 64 + 4;
+constexpr int k2QOpFloats = 64 * k2QLD;
+constexpr int k2QBufFloats = 3 * k2QOpFloats;
+constexpr int k2EpiFloats = 2 * k2QBufFloats;  // 102 KB
+constexpr int k2MaxFloats = k2RingFloats > k2EpiFloats ? k2RingFloats : k2EpiFloats;
+constexpr int k2SmemFloats = k2MaxFloats > kPairFloats ? k2MaxFloats : kPairFloats;
+constexpr int k2SmemBytes = k2SmemFloats * 4;
+static_assert(2 * (k2SmemBytes + 1024) <= 227 * 1024, "two CTAs per SM");
+
+template <int TILE>
+struct GraphCfg;
+template <>
+struct GraphCfg<64> {
+  static constexpr int threads = kThreads, ctas_per_sm = 1, smem = kSmemBytes;
+};
+template <>
+struct GraphCfg<128> {
+  static constexpr int threads = k2Threads, ctas_per_sm = 2, smem = k2SmemBytes;
+};
 
 __device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
@@ -100,7 +138,7 @@ __device__ __forceinline__ int64_t tri_idx(int i, int j, int b) {
 // ------------------------------------------------------------------ product tile
 // C-tile (64 x 64) of one block: acc = op(A1) B1 (+ alpha2 op(A2) B2), every A read by rows
 // (symmetric, skew, or given transposed), then the structured epilogue.
-__device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+__device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem) {
   const int tid = threadIdx.x;
   const int grp = tid >> 7, gtid = tid & (kGThreads - 1);
   const int tx = gtid & 15, ty = gtid >> 4;
@@ -372,21 +410,247 @@ __device__ void product_tile(const CnpJob& J, int z, int t, int b, float* smem) 
   }
 }
 
+// ------------------------------------------------------------------ 128 x 128 product tile
+// The same product and epilogue as product_tile64 on a 128 x 128 output tile, for 256
+// threads: thread (tx, ty) = (tid & 15, tid >> 4) owns rows {4 ty .. 4 ty + 3} and
+// {64 + 4 ty .. 64 + 4 ty + 3} and the same two column quads from 4 tx, so each k step
+// reads four 16-byte shared-memory vectors (conflict-free: a quarter warp reads 128
+// contiguous bytes or one broadcast address) for 64 FMAs.  The whole K runs in one
+// thread (no split, no partial-tile reduction); the epilogue works quadrant by quadrant
+// from the accumulator registers: operand rows are read as 16-byte vectors, the tile is
+// stored with 16-byte row stores, and the mirror of a symmetric (or symmetric + skew)
+// result is stored from the same registers as 16-byte column segments (four consecutive
+// rows of the thread become four consecutive columns of the mirrored row).
+__device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* smem) {
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int nt = b / 128;
+  int I, Jt;
+  if (J.mode == SG_FULL) {
+    I = t / nt;
+    Jt = t - I * nt;
+  } else {
+    tile_pair(nt, t, I, Jt);
+  }
+  const int m0 = I * 128, n0 = Jt * 128;
+  const int64_t boff = (int64_t)z * b * b;
+  const float* A1 = J.A + boff;
+  const float* B1 = J.B + boff;
+  const float* A2 = J.A2 ? J.A2 + boff : nullptr;
+  const float* B2 = J.B2 ? J.B2 + boff : nullptr;
+  const int nk1 = b / k2BK;
+  const int nkt = nk1 + (A2 ? b / k2BK : 0);
+  const float s1 = J.a_sym < 0 ? -1.f : 1.f;
+  const float s2 = J.a2_sym < 0 ? -1.f : 1.f;
+  // raw sums run over A read by rows; the first part is rescaled at the boundary so that
+  // one final factor gives op(A1) B1 + alpha2 op(A2) B2 (alpha2 = +-1 in every job)
+  const float boundary = s1 * s2 * J.alpha2;
+  const float scale = A2 ? s2 * J.alpha2 : s1;
+
+  float acc[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+
+  auto As_ = [&](int st) { return smem + st * k2StageFloats; };
+  auto Bs_ = [&](int st) { return smem + st * k2StageFloats + k2BK * k2LD; };
+  auto issue = [&](int kt) {
+    if (kt < nkt) {
+      const bool first = kt < nk1;
+      const float* A = first ? A1 : A2;
+      const float* B = first ? B1 : B2;
+      const int k0 = (first ? kt : kt - nk1) * k2BK;
+      float* As = As_(kt % k2Stages);
+      float* Bs = Bs_(kt % k2Stages);
+#pragma unroll
+      for (int l = 0; l < 2; ++l) {
+        const int f = tid + l * k2Threads;
+        const int r = f >> 5, c4 = (f & 31) * 4;
+        cp_async16(As + r * k2LD + c4, A + (int64_t)(k0 + r) * b + m0 + c4);
+        cp_async16(Bs + r * k2LD + c4, B + (int64_t)(k0 + r) * b + n0 + c4);
+      }
+    }
+    cp_commit();
+  };
+#pragma unroll
+  for (int st = 0; st < k2Stages - 1; ++st) issue(st);
+  for (int kt = 0; kt < nkt; ++kt) {
+    cp_wait<k2Stages - 2>();
+    __syncthreads();  // k tile kt landed for every thread; tile kt - 1 fully consumed
+    issue(kt + k2Stages - 1);
+    if (kt == nk1) {  // only with a second product
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] *= boundary;
+    }
+    const float* As = As_(kt % k2Stages);
+    const float* Bs = Bs_(kt % k2Stages);
+#pragma unroll
+    for (int k = 0; k < k2BK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(As + k * k2LD + ty * 4);
+      const float4 a1 = *reinterpret_cast<const float4*>(As + k * k2LD + 64 + ty * 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * k2LD + tx * 4);
+      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * k2LD + 64 + tx * 4);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+    }
+  }
+  cp_wait<0>();
+
+  // ---- epilogue from the registers, quadrant by quadrant
+  // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
+  float* const C = J.C + boff;
+  __nv_bfloat16* const Cb = J.Cb ? J.Cb + boff : nullptr;
+  float* const C2 = J.C2 ? J.C2 + boff : nullptr;
+  const int mode = J.mode;
+  const bool structured = mode != SG_FULL;
+  const float alpha = J.alpha * scale, alpha_c2 = J.alpha_c2 * scale;
+  const float diag = J.diag, diag2 = J.diag2, skew_c = J.skew_c;
+  const int nadd = J.nadd;
+  const float* ops[3] = {nadd > 0 ? J.add[0] + boff : nullptr,
+                         nadd > 1 ? J.add[1] + boff : nullptr,
+                         J.skew_add ? J.skew_add + boff : nullptr};
+  const float ac0 = nadd > 0 ? J.addc[0] : 0.f, ac1 = nadd > 1 ? J.addc[1] : 0.f;
+  const float bc0 = nadd > 0 ? J.addc2[0] : 0.f, bc1 = nadd > 1 ? J.addc2[1] : 0.f;
+  const bool has_ops = nadd > 0 || J.skew_add;
+  const bool diag_tile = structured && I == Jt;
+  // quadrants that produce output (q = 2 qr + qc): a diagonal tile keeps i <= j, so its
+  // quadrant below the diagonal (q = 2: rows 64.., columns ..63) holds nothing to store
+  const int nq = diag_tile ? 3 : 4;
+  auto quad = [&](int qi) { return (diag_tile && qi == 2) ? 3 : qi; };
+  // the ring is free: every thread passed the last k tile's barrier and its loads landed
+  __syncthreads();
+  auto stage_ops = [&](int qi) {  // coalesced 16-byte copies of the quadrant's operands
+    if (has_ops && qi < nq) {
+      const int qr = quad(qi) >> 1, qc = quad(qi) & 1;
+      float* buf = smem + (qi & 1) * k2QBufFloats;
+#pragma unroll
+      for (int o = 0; o < 3; ++o) {
+        if (!ops[o]) continue;
+        const float* src = ops[o] + (int64_t)(m0 + qr * 64) * b + n0 + qc * 64;
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+          const int f = tid + l * k2Threads;
+          const int r = f >> 4, c4 = (f & 15) * 4;
+          cp_async16(buf + o * k2QOpFloats + r * k2QLD + c4, src + (int64_t)r * b + c4);
+        }
+      }
+    }
+    cp_commit();
+  };
+  stage_ops(0);
+  stage_ops(1);
+  // the quadrant loop is unrolled so that the accumulators are indexed by constants
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (diag_tile && q == 2) continue;
+    const int qi = (diag_tile && q == 3) ? 2 : q;  // position in the staging order
+    cp_wait<1>();
+    __syncthreads();  // quadrant qi's operands are in shared memory for every thread
+    const int qr = q >> 1, qc = q & 1;
+    const bool dq = diag_tile && qr == qc;  // element-wise i <= j / i < j masks
+    const int i0 = m0 + qr * 64 + ty * 4, j0 = n0 + qc * 64 + tx * 4;
+    const float* buf = smem + (qi & 1) * k2QBufFloats;
+    // element (rr, c) of the quadrant: acc and the staged operands give the direct value
+    // v (at (i, j)), the mirrored value vm (at (j, i)) and the second output v2
+    auto values = [&](int rr, int c, float& v, float& vm, float& v2) {
+      const int i = i0 + rr, j = j0 + c;
+      const int so = (ty * 4 + rr) * k2QLD + tx * 4 + c;
+      const float e0 = ops[0] ? buf[so] : 0.f;
+      const float e1 = ops[1] ? buf[k2QOpFloats + so] : 0.f;
+      const float es = ops[2] ? buf[2 * k2QOpFloats + so] : 0.f;
+      const float a = acc[qr * 4 + rr][qc * 4 + c];
+      const float sym = (i == j ? diag : 0.f) + ac0 * e0 + ac1 * e1;
+      const float sym2 = (i == j ? diag2 : 0.f) + bc0 * e0 + bc1 * e1;
+      const float skew = alpha * a + skew_c * es;
+      if (mode == SG_SYMSKEW) {
+        v = (i == j) ? sym : sym + skew;
+        vm = sym - skew;
+      } else {
+        v = skew + sym;
+        vm = v;
+      }
+      v2 = alpha_c2 * a + sym2;
+    };
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {  // direct: row i, columns j0 .. j0 + 3
+      const int i = i0 + rr;
+      float v[4], vm_[4], v2[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) values(rr, c, v[c], vm_[c], v2[c]);
+      const int64_t row = (int64_t)i * b;
+      if (!dq) {
+        __stcg(reinterpret_cast<float4*>(C + row + j0), make_float4(v[0], v[1], v[2], v[3]));
+        if (Cb)
+          __stcg(reinterpret_cast<uint2*>(Cb + row + j0),
+                 make_uint2(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3])));
+        if (C2)
+          __stcg(reinterpret_cast<float4*>(C2 + row + j0), make_float4(v2[0], v2[1], v2[2], v2[3]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (i > j0 + c) continue;
+          __stcg(C + row + j0 + c, v[c]);
+          if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + j0 + c), bf16_bits(v[c]));
+          if (C2) __stcg(C2 + row + j0 + c, v2[c]);
+        }
+      }
+    }
+    if (structured) {  // mirror: row j, columns i0 .. i0 + 3
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = j0 + c;
+        float v[4], vm[4], v2[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) values(rr, c, v[rr], vm[rr], v2[rr]);
+        const int64_t row = (int64_t)j * b;
+        if (!dq) {
+          __stcg(reinterpret_cast<float4*>(C + row + i0), make_float4(vm[0], vm[1], vm[2], vm[3]));
+          if (Cb)
+            __stcg(reinterpret_cast<uint2*>(Cb + row + i0),
+                   make_uint2(bf16x2_bits(vm[0], vm[1]), bf16x2_bits(vm[2], vm[3])));
+          if (C2)
+            __stcg(reinterpret_cast<float4*>(C2 + row + i0),
+                   make_float4(v2[0], v2[1], v2[2], v2[3]));
+        } else {
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            if (i0 + rr >= j) continue;
+            __stcg(C + row + i0 + rr, vm[rr]);
+            if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + i0 + rr), bf16_bits(vm[rr]));
+            if (C2) __stcg(C2 + row + i0 + rr, v2[rr]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // every thread is done with buffer (qi & 1) before it is refilled
+    stage_ops(qi + 2);
+  }
+  cp_wait<0>();
+}
+
 // ------------------------------------------------------------------ 64 x 64 tile-pair jobs
 // Tile pair (I, J), I <= J, of a block; thread (tx = tid & 63, ty = tid >> 6) walks rows
 // ty, ty + 8, ... of the 64 x 64 tile, so each row is one coalesced 256-byte access.
 
-// A thread handles 4 consecutive columns c4.. of rows r = (tid >> 4) + 32 u (u < 2) of a
-// tile: every global access is a 16-byte vector of a coalesced row (the number of
-// requests, not the bytes, bounds these small jobs), and all of a thread's loads are
-// issued before any of them is used, so a tile costs one L2 round trip.
-constexpr int kQuadRows = kThreads / 16;           // rows covered per sweep
-constexpr int kQuadSweeps = kPT / kQuadRows;        // sweeps per 64-row tile
-static_assert(kQuadRows * kQuadSweeps == kPT, "tile sweep");
+// With NT threads, a thread handles 4 consecutive columns c4.. of rows
+// r = (tid >> 4) + (NT / 16) u of a tile: every global access is a 16-byte vector of a
+// coalesced row (the number of requests, not the bytes, bounds these small jobs), and all
+// of a thread's loads are issued before any of them is used, so a tile costs one L2 round
+// trip.
 
 
 // theta -> Q: Q_ij = theta, Q_ji = -theta
+template <int NT>
 __device__ void expand_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  constexpr int kQuadRows = NT / 16, kQuadSweeps = kPT / kQuadRows;
+  static_assert(kQuadRows * kQuadSweeps == kPT, "tile sweep");
   float (*tt)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
   int I, Jt;
   tile_pair(b / kPT, t, I, Jt);
@@ -427,7 +691,10 @@ __device__ void expand_tile(const CnpJob& J, int z, int t, int b, float* smem) {
 // out_o = sum_s coef[o][s] (X_s + X_s^T) (symmetric outputs), optional Cb_f = X_0^T.
 // Both tiles (I,J) and (J,I) of every input are staged first; each output element is then
 // formed directly (the sum is commutative, so diagonal tiles come out exactly symmetric).
+template <int NT>
 __device__ void symcomb_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  constexpr int kQuadRows = NT / 16, kQuadSweeps = kPT / kQuadRows;
+  static_assert(kQuadRows * kQuadSweeps == kPT, "tile sweep");
   float (*ta)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem);            // X_s(I,J)
   float (*tb)[kPT][kPLD] = reinterpret_cast<float (*)[kPT][kPLD]>(smem + 2 * kPT * kPLD);  // X_s(J,I)
   int I, Jt;
@@ -502,7 +769,10 @@ __device__ void symcomb_tile(const CnpJob& J, int z, int t, int b, float* smem) 
 }
 
 // dtheta_idx(i, j) = A_ij - A_ji
+template <int NT>
 __device__ void pack_tile(const CnpJob& J, int z, int t, int b, float* smem) {
+  constexpr int kQuadRows = NT / 16, kQuadSweeps = kPT / kQuadRows;
+  static_assert(kQuadRows * kQuadSweeps == kPT, "tile sweep");
   float (*ta)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem);
   float (*tb)[kPLD] = reinterpret_cast<float (*)[kPLD]>(smem + kPT * kPLD);
   int I, Jt;
@@ -525,6 +795,7 @@ __device__ void pack_tile(const CnpJob& J, int z, int t, int b, float* smem) {
   }
   __syncthreads();
   // packed rows are contiguous in j but not 16-byte aligned: scalar stores, tx-major
+  constexpr int kPRows = NT / kPT;
   const int tx = threadIdx.x & (kPT - 1), ty = threadIdx.x / kPT;
 #pragma unroll
   for (int u = 0; u < kPT / kPRows; ++u) {
@@ -539,7 +810,10 @@ __device__ __forceinline__ void red_release_add(int* p, int v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid_constant__ CnpGraph g) {
+template <int TILE>
+__global__ void __launch_bounds__(GraphCfg<TILE>::threads, GraphCfg<TILE>::ctas_per_sm)
+    k_cnp_graph(const __grid_constant__ CnpGraph g) {
+  constexpr int NT = GraphCfg<TILE>::threads;
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_item, s_next;
   __shared__ int s_ok;
@@ -598,10 +872,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_cnp_graph(const __grid
     if (!s_ok) break;
     const CnpJob& J = *reinterpret_cast<const CnpJob*>(s_job);
     switch (J.type) {
-      case JOB_EXPAND: expand_tile(J, z, t, g.b, smem); break;
-      case JOB_PRODUCT: product_tile(J, z, t, g.b, smem); break;
-      case JOB_SYMCOMB: symcomb_tile(J, z, t, g.b, smem); break;
-      default: pack_tile(J, z, t, g.b, smem); break;
+      case JOB_EXPAND: expand_tile<NT>(J, z, t, g.b, smem); break;
+      case JOB_PRODUCT:
+        if (TILE == 64)
+          product_tile64(J, z, t, g.b, smem);
+        else
+          product_tile128(J, z, t, g.b, smem);
+        break;
+      case JOB_SYMCOMB: symcomb_tile<NT>(J, z, t, g.b, smem); break;
+      default: pack_tile<NT>(J, z, t, g.b, smem); break;
     }
     // publish: the barrier orders every thread's stores before thread 0's release
     __syncthreads();
@@ -617,30 +896,68 @@ __global__ void k_zero_ints(int* p, int n, int first) {
     p[i] = i == 0 ? first : 0;
 }
 
-}  // namespace
-
-int cnp_graph_tiles(int type, int mode, int b) {
+// items per block of a job: output tiles of a product (tile x tile; upper tiles only for
+// symmetric results), 64 x 64 tile pairs of an elementwise job
+int cnp_graph_tiles(int type, int mode, int b, int tile) {
   if (type == JOB_PRODUCT) {
-    const int nt = b / 64;
+    const int nt = b / tile;
     return mode == SG_FULL ? nt * nt : nt * (nt + 1) / 2;
   }
-  const int nt = b / 64;  // 64 x 64 tile pairs
+  const int nt = b / 64;
   return nt * (nt + 1) / 2;
 }
 
+template <int TILE>
+cudaError_t launch_graph_t(const CnpGraph& g, cudaStream_t s) {
+  using Cfg = GraphCfg<TILE>;
+  // persistent grid: never more CTAs than can be resident at once
+  static int per_sm_dev[64] = {0};  // once per device, outside any stream capture
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  int& per_sm = per_sm_dev[dev];
+  cudaError_t e;
+  if (per_sm == 0) {
+    int v = 0;
+    e = cudaFuncSetAttribute(k_cnp_graph<TILE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::smem);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k_cnp_graph<TILE>, Cfg::threads,
+                                                      Cfg::smem);
+    if (e != cudaSuccess) return e;
+    per_sm = v > 0 ? v : 1;
+  }
+  int grid = num_sms() * per_sm;
+  const int total = g.item_start[g.njobs];
+  if (grid > total) grid = total;
+  begin_launch("cnp_sgemm", s);
+  e = launch_pdl(k_cnp_graph<TILE>, dim3(grid), dim3(Cfg::threads), Cfg::smem, s, g);
+  end_launch("cnp_sgemm", s);
+  return e;
+}
+
+}  // namespace
+
 cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;
-  g.item_start[0] = 0;
-  for (int j = 0; j < g.njobs; ++j) {
-    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.b);
-    g.item_start[j + 1] = g.item_start[j] + g.job[j].tiles * g.nblk;
-  }
   for (int j = 0; j < g.njobs; ++j) {  // shapes the tile code relies on
     const CnpJob& J = g.job[j];
     if (J.type == JOB_PRODUCT && J.nadd + (J.skew_add ? 1 : 0) > kEpiTiles)
       return cudaErrorInvalidValue;
+    if (J.type == JOB_PRODUCT && J.A2 && J.alpha2 != 1.f && J.alpha2 != -1.f)
+      return cudaErrorInvalidValue;
     if (J.type == JOB_SYMCOMB && (J.nin < 1 || J.nin > 2 || J.nout < 1 || J.nout > 4))
       return cudaErrorInvalidValue;
+  }
+  // 128 x 128 product items when every level of the chain has at least two waves of them
+  // (two CTAs per SM); otherwise 64 x 64 items, which split a block four times finer
+  const int nt128 = g.b % 128 == 0 ? g.b / 128 : 0;
+  const int sym_items = g.nblk * nt128 * (nt128 + 1) / 2;
+  const int tile = (nt128 > 0 && sym_items >= 4 * num_sms()) ? 128 : 64;
+  g.item_start[0] = 0;
+  for (int j = 0; j < g.njobs; ++j) {
+    g.job[j].tiles = cnp_graph_tiles(g.job[j].type, g.job[j].mode, g.b, tile);
+    g.item_start[j + 1] = g.item_start[j] + g.job[j].tiles * g.nblk;
   }
   g.err = device_error_flag();
   if (!g.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
@@ -651,28 +968,7 @@ cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
                              g.counters, ncount, g.first_counter);
   end_launch("cnp_elementwise", s);
   if (e != cudaSuccess) return e;
-  // persistent grid: never more CTAs than can be resident at once
-  static int per_sm_dev[64] = {0};  // once per device, outside any stream capture
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  int& per_sm = per_sm_dev[dev];
-  if (per_sm == 0) {
-    int v = 0;
-    e = cudaFuncSetAttribute(k_cnp_graph, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k_cnp_graph, kThreads, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    per_sm = v > 0 ? v : 1;
-  }
-  int grid = num_sms() * per_sm;
-  const int total = g.item_start[g.njobs];
-  if (grid > total) grid = total;
-  begin_launch("cnp_sgemm", s);
-  e = launch_pdl(k_cnp_graph, dim3(grid), dim3(kThreads), kSmemBytes, s, g);
-  end_launch("cnp_sgemm", s);
-  return e;
+  return tile == 128 ? launch_graph_t<128>(g, s) : launch_graph_t<64>(g, s);
 }
 
 }  // namespace poetx

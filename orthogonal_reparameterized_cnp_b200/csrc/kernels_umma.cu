@@ -17,6 +17,8 @@
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x (M=128, N=BN, K=16) per chunk
 //   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator, convert, stage each 32 x 64
 //               piece in a 128-byte-swizzled 4 KB tile, TMA tensor store
+//   warps 10-11 (SIDE instantiation only): a side job independent of the GEMM -- the
+//               int8 weight's next panel dequantised to bf16 while this one is multiplied
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap the main loop
 // of tile t+1.  The kernel is launched as a programmatic dependent of the previous kernel
 // on the stream: set-up (barriers, TMEM, tensor-map prefetch) runs before
@@ -34,6 +36,7 @@
 
 #include <mutex>
 
+#include "dequant_dev.cuh"
 #include "poetx_internal.h"
 
 namespace poetx {
@@ -71,7 +74,14 @@ struct Params {
   int* err;
   unsigned long long wait_ns;  // bound of every mbarrier wait
   int y_per_bz, y_per_split;  // output tensor rows per batch entry / per split
+  // side job (SIDE instantiation)
+  const int8_t* side_q;
+  long long side_ldq, side_ldd;
+  const float* side_scales;
+  __nv_bfloat16* side_dst;
+  int side_rows, side_cols;
 };
+constexpr int kSideWarps = 2;
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -296,8 +306,8 @@ __device__ __forceinline__ int b_key(const Params& p, int item) {
   return (w.bz * p.ksplit + w.split) * p.tiles_n + w.tn;
 }
 
-template <int BN, bool A_MN, bool B_MN, bool B_RES>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, bool A_MN, bool B_MN, bool B_RES, bool SIDE>
+__global__ void __launch_bounds__(kThreads + (SIDE ? 32 * kSideWarps : 0), 1)
     k_umma_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const Params p) {
   using C = Cfg<BN, B_RES>;
@@ -488,6 +498,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // all MMAs issued by this thread complete before TMEM is released
     umma_commit(drain_bar);
     mbar_drain_wait(drain_bar, 0);
+  } else if (SIDE && warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ side job
+    const int st = threadIdx.x - 32 * (2 + kEpiWarps);
+    dequant_rows2d(p.side_q, p.side_ldq, p.side_scales, p.side_dst, p.side_ldd, p.side_rows,
+                   p.side_cols, (int64_t)blockIdx.x * (32 * kSideWarps) + st,
+                   (int64_t)gridDim.x * (32 * kSideWarps));
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue
     // warp w drains TMEM lane quadrant (w % 4) and column half (w - 2) / 4 of each tile,
@@ -600,10 +616,11 @@ bool make_map(CUtensorMap* map, const UmmaOperand& op, int box_rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, bool A_MN, bool B_MN, bool B_RES>
+template <int BN, bool A_MN, bool B_MN, bool B_RES, bool SIDE = false>
 cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
                      const Params& p, int grid, const char* family, cudaStream_t s) {
-  auto kern = k_umma_gemm<BN, A_MN, B_MN, B_RES>;
+  auto kern = k_umma_gemm<BN, A_MN, B_MN, B_RES, SIDE>;
+  constexpr int threads = kThreads + (SIDE ? 32 * kSideWarps : 0);
   static bool attr_done[64] = {false};  // once per device, outside any stream capture
   int dev = 0;
   cudaGetDevice(&dev);
@@ -615,7 +632,7 @@ cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtenso
     attr_done[dev] = true;
   }
   begin_launch(family, s);
-  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), Cfg<BN, B_RES>::SMEM_BYTES, s,
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), Cfg<BN, B_RES>::SMEM_BYTES, s,
                                    ma, mb, md, p);
   end_launch(family, s);
   return e;
@@ -625,6 +642,11 @@ template <int BN>
 cudaError_t launch_bn(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
                       const Params& p, int grid, bool a_mn, bool b_mn, bool b_res,
                       const char* family, cudaStream_t s) {
+  if (p.side_rows > 0) {  // the merged-weight GEMMs: A K-major, B either way, B streamed
+    if (a_mn || b_res) return cudaErrorInvalidValue;
+    if (!b_mn) return launch_t<BN, false, false, false, true>(ma, mb, md, p, grid, family, s);
+    return launch_t<BN, false, true, false, true>(ma, mb, md, p, grid, family, s);
+  }
   if (b_res) {  // A K-major only
     if (!b_mn) return launch_t<BN, false, false, true>(ma, mb, md, p, grid, family, s);
     return launch_t<BN, false, true, true>(ma, mb, md, p, grid, family, s);
@@ -702,6 +724,18 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   p.d_boff_col = g.d_boff_col;
   p.d_boff = g.d_boff;
   p.d_split = g.d_split;
+  p.side_q = g.side_q;
+  p.side_ldq = g.side_ldq;
+  p.side_scales = g.side_scales;
+  p.side_dst = static_cast<__nv_bfloat16*>(g.side_dst);
+  p.side_ldd = g.side_ldd;
+  p.side_rows = g.side_rows > 0 ? g.side_rows : 0;
+  p.side_cols = g.side_cols;
+  if (p.side_rows > 0 &&
+      (!g.side_q || !g.side_scales || !g.side_dst || g.side_cols <= 0 || g.side_cols % 16 ||
+       g.side_ldq % 16 || g.side_ldd % 8 || (reinterpret_cast<uintptr_t>(g.side_q) & 15) ||
+       (reinterpret_cast<uintptr_t>(g.side_dst) & 15)))
+    return cudaErrorInvalidValue;
   p.err = device_error_flag();
   if (!p.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
   p.wait_ns = wait_limit_ns();
@@ -718,7 +752,7 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   if (grid > p.num_items) grid = p.num_items;
   // keep B resident when one item's whole B (K <= 256) fits and the items share it
   const bool b_res = !g.A.mn_major && p.kcps <= 4 && p.ksplit == 1 &&
-                     p.num_items >= 2 * grid && p.tiles_m >= 2;
+                     p.num_items >= 2 * grid && p.tiles_m >= 2 && p.side_rows == 0;
   if (BN == 256)
     return launch_bn<256>(ma, mb, md, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);
   return launch_bn<128>(ma, mb, md, p, grid, g.A.mn_major, g.B.mn_major, b_res, family, s);

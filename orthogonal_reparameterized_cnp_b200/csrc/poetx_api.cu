@@ -1194,6 +1194,25 @@ int poetx_quantize_rows(const void* W, int8_t* q, float* scales, int32_t m, int3
   return POETX_OK;
 }
 
+int poetx_merge_perm_q8(const void* W0, int8_t* W0q, float* scales, int32_t m, int32_t n,
+                        const int32_t* perm_R, const int32_t* perm_P, int dtype, void* stream) {
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m < 0 || n < 0) return fail(POETX_ERR_INVALID_ARG, "negative size");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!W0 || !W0q || !scales || !perm_R || !perm_P)
+    return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W0) || !aligned16(W0q) || !aligned16(scales) || !aligned16(perm_R) ||
+      !aligned16(perm_P))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const int es = dtype == POETX_BF16 ? 2 : 4;
+  if ((size_t)n * es > 200 * 1024)
+    return fail(POETX_ERR_SHAPE, "rows wider than 200 KB are not supported");
+  POETX_CUDA(launch_merge_quantize(W0, perm_R, perm_P, W0q, scales, m, n, es,
+                                   static_cast<cudaStream_t>(stream)),
+             "merge + quantize");
+  return POETX_OK;
+}
+
 size_t poetx_linear_q8_scratch(const poetx_linear_desc* d) {
   if (!d || d->dtype != POETX_BF16 || d->m <= 0 || d->n <= 0) return 0;
   return align_up((size_t)d->m * d->n * 2);

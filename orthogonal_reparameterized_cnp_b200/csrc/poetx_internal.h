@@ -80,9 +80,17 @@ cudaError_t launch_compose_perm(const int32_t* outer, const int32_t* inner, int3
 // per-row symmetric int8: s_i = max|w_i.| / 127, q = rint(w / s) in [-127, 127]
 cudaError_t launch_quantize_rows(const void* W, int8_t* q, float* s, int m, int n,
                                  int elem_bytes, cudaStream_t st);
+// q, s = per-row int8 codes of the merged weight W0[perm_R][:, perm_P] (no merged copy)
+cudaError_t launch_merge_quantize(const void* W0, const int32_t* perm_R, const int32_t* perm_P,
+                                  int8_t* q, float* s, int m, int n, int elem_bytes,
+                                  cudaStream_t st);
 // out (bf16) = s_i * q_ij
 cudaError_t launch_dequant_rows(const int8_t* q, const float* s, void* out, int m, int n,
                                 cudaStream_t st);
+// out[r][c] (bf16, row stride ldo) = s_r * q[r][c] (row stride ldq) for r < rows, c < cols;
+// cols % 16 == 0, 16-byte aligned rows
+cudaError_t launch_dequant_2d(const int8_t* q, int64_t ldq, const float* s, void* out,
+                              int64_t ldo, int rows, int cols, cudaStream_t st);
 
 // ---- fp32 SIMT batched GEMM (kernels_sgemm.cu) -----------------------------------
 enum SgemmMode { SG_FULL = 0, SG_SYM = 1, SG_SYMSKEW = 2 };
@@ -219,6 +227,15 @@ struct UmmaGemm {
   int64_t d_boff_col = 0;     // per-batch column offset of D
   int64_t d_boff = 0;         // per-batch element offset of D
   int64_t d_split = 0;        // per-split element offset of D
+  // optional side job of two extra warps per CTA, run alongside the GEMM:
+  // side_dst[r][c] = bf16(side_scales[r] * side_q[r][c]) for r < side_rows, c < side_cols
+  // (the int8 weight's next panel while this panel is multiplied); side_rows = 0: none
+  const int8_t* side_q = nullptr;
+  int64_t side_ldq = 0;
+  const float* side_scales = nullptr;
+  void* side_dst = nullptr;
+  int64_t side_ldd = 0;
+  int side_rows = 0, side_cols = 0;
 };
 cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t s);
 // ksplit the launcher would choose for the given problem (used to size scratch).

@@ -72,6 +72,7 @@ SIGNATURES = {
                                              _vp]),
     "poetx_fma_probe": (_c_int, [_vp, _c_i32, _c_i32, _vp]),
     "poetx_quantize_rows": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _c_int, _vp]),
+    "poetx_merge_perm_q8": (_c_int, [_vp, _vp, _vp, _c_i32, _c_i32, _vp, _vp, _c_int, _vp]),
     "poetx_linear_q8_scratch": (_c_size, [ctypes.POINTER(LinearDesc)]),
     "poetx_linear_fwd_q8": (_c_int, [ctypes.POINTER(LinearDesc), _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _vp, _c_size, _vp]),
@@ -320,6 +321,15 @@ def quantize_rows(W, q, scales, stream=None):
                                        _stream(stream)), "poetx_quantize_rows")
 
 
+def merge_perm_q8(W0, q, scales, perm_R, perm_P, stream=None):
+    """Int8 codes and per-row scales of W0' = W0[perm_R][:, perm_P], without forming W0'."""
+    _require_cuda()
+    m, n = W0.shape
+    _check(_load().poetx_merge_perm_q8(_ptr(W0), _ptr(q), _ptr(scales), m, n, _ptr(perm_R),
+                                       _ptr(perm_P), _dtype_code(W0), _stream(stream)),
+           "poetx_merge_perm_q8")
+
+
 def linear_q8_scratch(desc: LinearDesc) -> int:
     return int(_load().poetx_linear_q8_scratch(ctypes.byref(desc)))
 
@@ -447,7 +457,7 @@ class PoetxLinear:
         self.perm_P, self.inv_P = torch.as_tensor(pP, **i32), torch.as_tensor(iP, **i32)
         self.perm_R, self.inv_R = torch.as_tensor(pR, **i32), torch.as_tensor(iR, **i32)
         self.W0 = W0
-        self.W0p = torch.empty_like(W0)
+        self.W0p = None if int8_weight else torch.empty_like(W0)
         if cnp is None:
             cnp = CnpBuffers(nblk, b, k, dev, W0.dtype if self.bf16 else None)
             first_block = 0
@@ -483,8 +493,8 @@ class PoetxLinear:
         elif ws.numel() * ws.element_size() < need:
             raise ValueError("shared layer scratch too small")
         self.ws = ws
-        if int8_weight:  # the bf16 merged weight is only a step of merge(): it lives in scratch
-            self.W0p = self.ws[: self.m * self.n * 2].view(W0.dtype).view(self.m, self.n)
+        if int8_weight:  # the merged weight exists only as int8 codes (merge_perm_q8)
+            self.W0p = None
         self.merge()
 
     def G_ops(self):
@@ -493,9 +503,10 @@ class PoetxLinear:
 
     def merge(self, stream=None):
         """W0' = Pi_R W0 Pi_P^T (and its int8 codes): once per set of permutations."""
-        merge_perm(self.W0, self.W0p, self.perm_R, self.perm_P, stream)
         if self.int8:
-            quantize_rows(self.W0p, self.W0q, self.scales, stream)
+            merge_perm_q8(self.W0, self.W0q, self.scales, self.perm_R, self.perm_P, stream)
+        else:
+            merge_perm(self.W0, self.W0p, self.perm_R, self.perm_P, stream)
 
     def cnp_forward(self, stream=None):
         self.cnp.forward(stream)

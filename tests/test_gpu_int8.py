@@ -44,6 +44,31 @@ def test_quantize_rows_bit_exact(dtype, m, n):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("m,n", [(1, 16), (300, 520), (13824, 5120), (77, 13824), (5, 33)])
+def test_merge_perm_q8_bit_exact(dtype, m, n):
+    """Codes and scales of the merged weight straight from W0 equal the oracle's quantiser
+    applied to the oracle's merged weight W0[p_R][:, p_P] (zero rows included)."""
+    import torch
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    rng = np.random.default_rng(m * 7 + n)
+    W = rng.standard_normal((m, n)) * rng.uniform(1e-3, 5.0, (m, 1))
+    W[min(2, m - 1)] = 0.0
+    W = round_to_bf16(W) if dtype == "bf16" else W.astype(np.float32).astype(np.float64)
+    Wd = tensor(W, torch.bfloat16 if dtype == "bf16" else torch.float32)
+    pR, _ = P.make_perm(m + 1, m)
+    pP, _ = P.make_perm(n + 2, n)
+    q = torch.empty((m, n), dtype=torch.int8, device="cuda")
+    s = torch.empty((m,), dtype=torch.float32, device="cuda")
+    P.merge_perm_q8(Wd, q, s, tensor(pR, torch.int32), tensor(pP, torch.int32))
+    torch.cuda.synchronize()
+    oR, _ = ref.make_perm(m + 1, m)
+    oP, _ = ref.make_perm(n + 2, n)
+    q_ref, s_ref = ref.quantize_rows_int8(ref.merge_perm(W, oR, oP))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
 @pytest.mark.parametrize("T,n,m,b", [(256, 512, 384, 128), (320, 512, 768, 256)])
 def test_int8_layer_matches_oracle(T, n, m, b):
     import torch

@@ -114,14 +114,15 @@ def test_cnp_matches_oracle(b, k):
     assert torch.equal(Gb.cpu(), G.cpu().to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("b,k", [(64, 6), (100, 4), (256, 4), (128, 1)])
-def test_cnp_saved_pair_is_bit_identical(b, k):
+@pytest.mark.parametrize("b,k,nblk", [(64, 6, 3), (100, 4, 3), (256, 4, 3), (128, 1, 3),
+                                      (256, 4, 200), (128, 6, 700)])
+def test_cnp_saved_pair_is_bit_identical(b, k, nblk):
     # the forward keeps Q, S = Q^2 and F'; the backward that reads them must give exactly
     # the dtheta of the recomputing backward (task graph: b % 64 == 0; b = 100 takes the
-    # per-step path), and S must be Q^2
+    # per-step path; 200 blocks of 256 and 700 of 128 take the 128 x 128 product items),
+    # and S must be Q^2
     import torch
     P = _P()
-    nblk = 3
     rng = np.random.default_rng(b * 7 + k)
     theta = (rng.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
     dG = rng.standard_normal((nblk, b, b)).astype(np.float32)
@@ -139,9 +140,14 @@ def test_cnp_saved_pair_is_bit_identical(b, k):
     assert P.device_status() == P.POETX_OK
     assert torch.equal(G2, G)
     assert torch.equal(dth2, dth)
-    Q = np.stack([ref.theta_to_Q(t, b) for t in theta.astype(np.float64)])
-    assert np.array_equal(host(Qs), Q)  # the packing, bit-exact (fp32 theta is exact in fp64)
-    assert np.abs(host(S) - Q @ Q).max() <= CNP_ABS
+    sel = [0, nblk // 2, nblk - 1]
+    Q = np.stack([ref.theta_to_Q(t, b) for t in theta[sel].astype(np.float64)])
+    # the packing, bit-exact (fp32 theta is exact in fp64)
+    assert np.array_equal(host(Qs[sel]), Q)
+    assert np.abs(host(S[sel]) - Q @ Q).max() <= CNP_ABS
+    # G and dtheta of those blocks against the oracle
+    assert np.abs(host(G[sel]) - ref.cnp_forward(theta[sel], b, k)).max() <= CNP_ABS
+    assert np.abs(host(dth[sel]) - ref.cnp_backward(theta[sel], dG[sel], b, k)).max() <= CNP_ABS
 
 
 def test_cnp_zero_theta_is_exact_identity():

@@ -165,6 +165,19 @@ def test_int8_weight_validation_before_launch():
                                    None) == P.POETX_ERR_WORKSPACE
 
 
+def test_merge_perm_q8_validation_before_launch():
+    lib = P.lib()
+    f = ctypes.c_void_p(0xA0000)
+    assert lib.poetx_merge_perm_q8(f, f, f, 4, 8, f, f, 9, None) == P.POETX_ERR_DTYPE
+    assert lib.poetx_merge_perm_q8(None, f, f, 4, 8, f, f, P.POETX_BF16, None) == \
+        P.POETX_ERR_INVALID_ARG
+    assert lib.poetx_merge_perm_q8(f, f, f, 4, 8, ctypes.c_void_p(0xA0004), f, P.POETX_BF16,
+                                   None) == P.POETX_ERR_ALIGN
+    assert lib.poetx_merge_perm_q8(f, f, f, 4, 200000, f, f, P.POETX_F32, None) == \
+        P.POETX_ERR_SHAPE
+    assert lib.poetx_merge_perm_q8(f, f, f, 0, 8, f, f, P.POETX_BF16, None) == P.POETX_OK
+
+
 def test_profile_and_launch_counter_without_launches():
     n0 = P.launch_count()
     assert P.launch_count() == n0
