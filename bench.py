@@ -525,6 +525,29 @@ def family_attribution(P, wl, stream, reps):
     return out
 
 
+def w0_single_cta(P, wl, stream, reps):
+    """The merged-weight GEMMs of one step on single CTAs (128 x 256 tiles) instead of CTA
+    pairs, from CUDA-graph replays with events around each launch (for comparison)."""
+    import torch
+    prev = P.set_gemm_pairs(False)
+    try:
+        P.profile_begin("gemm_w0")
+        g = graph_of(lambda st: wl.step(0, st), stream)
+        P.profile_begin(None)
+        tot, launches = 0.0, 0
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            n, ms = P.profile_end()
+            tot += ms
+            launches = n
+        del g
+    finally:
+        P.set_gemm_pairs(prev)
+    check_status(P, stream, "the single-CTA GEMM replays")
+    return {"launches_per_step": launches, "ms_per_step": tot / reps}
+
+
 def cnp_only(P, wl, stream, reps):
     """CNP forward and backward alone (one call each over every block), CUDA-graph replay."""
     c = wl.group.cnp
@@ -702,10 +725,16 @@ def run_poetx(args):
     # per-family device time and the roofline of the dominant family
     work = family_work(shapes)
     breakdown = family_attribution(P, wl, stream, reps=min(reps, 20))
-    dominant = max(breakdown, key=lambda f: breakdown[f]["ms_per_step"])
+    if wl.bf16:
+        alt = w0_single_cta(P, wl, stream, reps=min(reps, 20))
+        ww = family_work(shapes)["gemm_w0"]
+        alt["achieved_tflops"] = ww["flops"] / (alt["ms_per_step"] / 1e3) / 1e12
+        breakdown["gemm_w0_single_cta"] = alt
+    dominant = max(FAMILIES, key=lambda f: breakdown[f]["ms_per_step"])
     peaks, peak_src = load_peaks()
     wkey = workload_name(args.workload, shapes)
-    for fam, bd in breakdown.items():
+    for fam in FAMILIES:
+        bd = breakdown[fam]
         ww = work.get(fam)
         if ww and bd["ms_per_step"] > 0:
             if "flops" in ww:

@@ -340,6 +340,17 @@ int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* d
 int poetx_set_wait_limit(uint64_t ns, uint64_t* previous);
 
 /*
+ * Kernel choice for the merged-weight GEMMs (W = V W0'^T, dV = dW W0'): 1 (the default)
+ * runs them on CTA pairs (tcgen05 cta_group::2, 256 x 256 tiles shared by two SMs) when the
+ * shape allows (N % 256 == 0, M >= 256), 0 always on single CTAs (128 x 256 tiles).  Both
+ * compute the same products; the switch exists to compare them.  Applies to launches made
+ * after the call.
+ *   previous: receives the setting before this call (may be NULL).
+ *   Errors: POETX_ERR_INVALID_ARG for a value other than 0 or 1.
+ */
+int poetx_set_gemm_pairs(int enable, int* previous);
+
+/*
  * Self-test of the bounded waits (no counterpart in the pages): runs the CNP forward task
  * graph of nblk blocks with the done-counter of block 0's first step started far below
  * reach, so the first item that depends on it waits until the time limit, records

@@ -1,0 +1,453 @@
+// tcgen05 GEMM on CTA pairs (cta_group::2) for the merged-weight products of the layer,
+// W = V W0'^T and dV = dW W0' (POET-X technical summary section 2.1: the dense W0' product
+// of the input-centric layer, the largest contraction of a step).
+//
+//   D[M x N] = A[M x K] . B[N x K]^T      (bf16 operands, fp32 accumulation in TMEM, bf16 out)
+//
+// The two CTAs of a cluster compute one 256 x 256 output tile together.  CTA r of the pair
+// loads, per 64-wide K chunk, rows [128 r, 128 r + 128) of the tile's A and rows
+// [128 r, 128 r + 128) of its B (half of the tile's N) into its own shared memory with
+// TMA; the leader CTA (r = 0) issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16),
+// which reads both CTAs' shared memory and accumulates row half r of the tile in CTA r's
+// TMEM.  Per MAC each SM thus loads half the B bytes of the one-CTA kernel (128 x 256
+// tiles), and the freed shared memory holds six operand stages instead of four.
+//
+// Roles (320 threads per CTA, one CTA per SM, persistent over the tiles of its pair):
+//   warp 0      TMA producer, both CTAs: waits for its own stage to be free, loads its
+//               halves; the completion bytes of both CTAs land on the leader's full barrier
+//   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (leader only):
+//               waits on its full barrier, issues 4 MMAs per chunk, and its commits arrive on
+//               the stage's empty barrier and the accumulator's full barrier of both CTAs
+//   warps 2..9  epilogue, both CTAs: tcgen05.ld of the CTA's 128 accumulator rows, bf16,
+//               TMA tensor stores; then a remote arrive on the leader's accumulator-empty
+//               barrier
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap the main loop
+// of tile t + 1.  Loads carry no cluster multicast: each CTA loads distinct data.
+//
+// Every mbarrier wait is bounded (Params2::wait_ns): on a timeout the waiting role records
+// POETX_ERR_TIMEOUT in the device flag and leaves its loop; the CTAs then drain what they can
+// observe with short bounded waits, meet at a cluster barrier and free TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "poetx_internal.h"
+#include "umma_ptx.cuh"
+
+namespace poetx {
+namespace {
+
+constexpr int kPairBM = 128;   // A rows per CTA (256 per pair)
+constexpr int kPairBN = 256;   // N of the pair tile (128 B rows per CTA)
+constexpr int kPairBK = 64;
+constexpr int kPairStages = 6;
+constexpr int kPairThreads = 320;
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairA = kPairBM * kPairBK * 2;            // 16 KB
+constexpr int kPairB = (kPairBN / 2) * kPairBK * 2;      // 16 KB
+constexpr int kPairRing = kPairStages * (kPairA + kPairB);
+constexpr int kPairEpi = kPairEpiWarps * 4096;
+constexpr int kPairSmem = 1024 + kPairRing + kPairEpi + 256;
+static_assert(kPairSmem <= 227 * 1024, "shared memory per CTA");
+constexpr uint32_t kPairTmemCols = 2 * kPairBN;
+
+struct Params2 {
+  int M, N, K, total_kc, tiles_m, tiles_n, num_items;
+  int* err;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// the address of this CTA's shared variable `a` in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait with cluster-scope acquire (barriers that the peer CTA arrives on)
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int* err,
+                                               unsigned long long limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  unsigned spins = 0;
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if ((++spins & 63u) == 0) {
+      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        atomicCAS(err, 0, (int)POETX_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+// TMA load into this CTA's shared memory whose completion bytes go to `mbar_cluster`, a
+// barrier of either CTA of the pair (no multicast)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t mbar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrives once on the barrier at offset `bar` of every CTA in `mask` when all MMAs issued so
+// far by this thread have completed
+__device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+template <bool B_MN>
+__device__ __forceinline__ uint32_t make_idesc_pair() {
+  return (1u << 4)                              // D format: f32
+         | (1u << 7)                            // A format: bf16
+         | (1u << 10)                           // B format: bf16
+         | (0u << 15)                           // A K-major
+         | ((B_MN ? 1u : 0u) << 16)             // B major
+         | ((uint32_t)(kPairBN >> 3) << 17)     // N = 256
+         | ((uint32_t)(256 >> 4) << 24);        // M = 256 (the pair)
+}
+
+template <bool B_MN>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    k_umma_gemm_pair(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmD, const Params2 p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t sA = base;                                   // stages x 16 KB
+  const uint32_t sB = base + kPairStages * kPairA;            // stages x 16 KB
+  const uint32_t sEpi = base + kPairRing;                     // 1024-aligned staging tiles
+  const uint32_t sBar = sEpi + kPairEpi;
+  auto full_bar = [&](int s) { return sBar + 8u * s; };
+  auto empty_bar = [&](int s) { return sBar + 8u * (kPairStages + s); };
+  auto tfull_bar = [&](int a) { return sBar + 8u * (2 * kPairStages + a); };
+  auto tempty_bar = [&](int a) { return sBar + 8u * (2 * kPairStages + 2 + a); };
+  const uint32_t drain_bar = sBar + 8u * (2 * kPairStages + 4);
+  const uint32_t tmem_slot = sBar + 8u * (2 * kPairStages + 5);
+  unsigned char* generic_base = smem_raw + (base - raw);
+  volatile uint32_t* tmem_slot_ptr =
+      reinterpret_cast<volatile uint32_t*>(generic_base + (tmem_slot - base));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * kPairEpiWarps);  // the epilogue warps of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmD);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kPairTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or TMA completion
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot_ptr;
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    int it = 0;
+    bool ok = true;
+    for (int item = cid; ok && item < p.num_items; item += nclusters) {
+      const int tm = item % p.tiles_m, tn = item / p.tiles_m;
+      const int m0 = tm * 256 + (int)rank * kPairBM;
+      const int n0 = tn * kPairBN + (int)rank * (kPairBN / 2);
+      for (int kc = 0; kc < p.total_kc; ++kc, ++it) {
+        const int s = it % kPairStages, r = it / kPairStages;
+        if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_expect_tx(full_bar(s), 2u * (kPairA + kPairB));
+        const uint32_t fb = map_to_rank(full_bar(s), 0);
+        const int k = kc * kPairBK;
+        tma_load_2d_pair(sA + s * kPairA, &tmA, k, m0, fb);
+        const uint32_t b_dst = sB + s * kPairB;
+        if (!B_MN) {
+          tma_load_2d_pair(b_dst, &tmB, k, n0, fb);
+        } else {
+          tma_load_2d_pair(b_dst, &tmB, n0, k, fb);
+          tma_load_2d_pair(b_dst + 8192, &tmB, n0 + 64, k, fb);
+        }
+      }
+    }
+    if (!ok && leader) {
+      // no TMA write may still be in flight into the leader's stages when it leaves
+      const int last = it;
+      for (int j = (last > kPairStages ? last - kPairStages : 0); j < last; ++j)
+        mbar_drain_wait(full_bar(j % kPairStages), (j / kPairStages) & 1);
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    const uint32_t idesc = make_idesc_pair<B_MN>();
+    int it = 0, tcount = 0;
+    bool ok = true;
+    for (int item = cid; ok && item < p.num_items; item += nclusters, ++tcount) {
+      const int acc = tcount & 1, ra = tcount >> 1;
+      if (!mbar_wait_cluster(tempty_bar(acc), (ra & 1) ^ 1, p.err, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kPairBN);
+      for (int kc = 0; kc < p.total_kc; ++kc, ++it) {
+        const int s = it % kPairStages, r = it / kPairStages;
+        if (!mbar_wait(full_bar(s), r & 1, p.err, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = sA + s * kPairA;
+        const uint32_t b_addr = sB + s * kPairB;
+#pragma unroll
+        for (int kk = 0; kk < kPairBK / 16; ++kk) {
+          const uint64_t adesc = make_desc(a_addr + kk * 32, 16, 1024);
+          const uint64_t bdesc = B_MN ? make_desc(b_addr + kk * 2048, 8192, 1024)
+                                      : make_desc(b_addr + kk * 32, 16, 1024);
+          umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit_pair_mc(empty_bar(s), (uint16_t)0x3);  // both CTAs' stage s is free
+      }
+      if (!ok) break;
+      umma_commit_pair_mc(tfull_bar(acc), (uint16_t)0x3);  // both accumulator halves ready
+    }
+    // every MMA issued here completes before TMEM is released
+    umma_commit_pair(drain_bar);
+    mbar_drain_wait(drain_bar, 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    // warp w drains TMEM lane quadrant (w % 4) and column half (w - 2) / 4 of this CTA's
+    // 128 accumulator rows, 64 columns per tcgen05.ld; each 32-row piece goes through the
+    // warp's 4 KB 128-byte-swizzled staging tile to a TMA tensor store.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int HALF = kPairBN / 2;
+    const uint32_t stage = sEpi + (uint32_t)(warp - 2) * 4096u;
+    const uint32_t my_row = stage + (uint32_t)lane * 128u;
+    const uint32_t sw = (uint32_t)(lane & 7);
+    int tcount = 0;
+    for (int item = cid; item < p.num_items; item += nclusters, ++tcount) {
+      const int tm = item % p.tiles_m, tn = item / p.tiles_m;
+      const int acc = tcount & 1, ra = tcount >> 1;
+      int ready = 0;
+      if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err, p.wait_ns) ? 1 : 0;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (!ready) break;
+      tc_fence_after();
+      const int row0 = tm * 256 + (int)rank * kPairBM + q * 32;
+      const int n0 = tn * kPairBN;
+#pragma unroll 1
+      for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
+        uint32_t v[64];
+        tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kPairBN + c), v);
+        tmem_wait_ld();
+        if (n0 + c >= p.N) continue;  // (uniform across the warp)
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(v[8 * k + 2 * e]),
+                                                      __uint_as_float(v[8 * k + 2 * e + 1]));
+            o[e] = *reinterpret_cast<uint32_t*>(&hh);
+          }
+          sts128(my_row + (((uint32_t)k ^ sw) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmD, n0 + c, row0, stage);
+          bulk_commit();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar(acc), 0));
+    }
+    if (lane == 0) bulk_wait0();  // every store of this warp has landed before exit
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // both CTAs are done with TMEM, shared memory and the barriers
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kPairTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    tried = true;
+  }
+  return fn;
+}
+
+bool map2d(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+           uint32_t box_cols, uint32_t box_rows, bool store) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             store ? CU_TENSOR_MAP_L2_PROMOTION_NONE : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool B_MN>
+cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
+                          const Params2& p, int grid, const char* family, cudaStream_t s) {
+  auto kern = k_umma_gemm_pair<B_MN>;
+  static bool attr_done[64] = {false};  // once per device, outside any stream capture
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPairSmem);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  begin_launch(family, s);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
+  end_launch(family, s);
+  return e;
+}
+
+}  // namespace
+
+bool umma_pair_eligible(const UmmaGemm& g) {
+  return g.batch == 1 && g.ksplit <= 1 && !g.A.mn_major && !g.out_f32 && g.side_rows == 0 &&
+         g.N % kPairBN == 0 && g.M >= 256 && g.K >= kPairBK && g.ldd == g.N &&
+         g.A.boff_k == 0 && g.A.boff_mn == 0 && g.B.boff_k == 0 && g.B.boff_mn == 0 &&
+         g.d_boff == 0 && g.d_boff_col == 0 && g.d_split == 0;
+}
+
+cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStream_t s) {
+  if (!umma_pair_eligible(g)) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb, md;
+  // A K-major: boxes of 128 rows x 64 K.  B K-major: 128 N-rows x 64 K; MN-major: 64 K-rows
+  // x 64 N (two per stage).  Output: 32-row boxes of 64 bf16.
+  if (!map2d(&ma, g.A.ptr, g.A.rows, g.A.cols, g.A.ld, 64u, (uint32_t)kPairBM, false))
+    return cudaErrorInvalidValue;
+  if (!map2d(&mb, g.B.ptr, g.B.rows, g.B.cols, g.B.ld, 64u, g.B.mn_major ? 64u : 128u, false))
+    return cudaErrorInvalidValue;
+  if (!map2d(&md, g.D, g.M, g.N, g.ldd, 64u, 32u, true)) return cudaErrorInvalidValue;
+  Params2 p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.total_kc = (g.K + kPairBK - 1) / kPairBK;
+  p.tiles_m = (g.M + 255) / 256;
+  p.tiles_n = g.N / kPairBN;
+  const long long items = (long long)p.tiles_m * p.tiles_n;
+  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  p.num_items = (int)items;
+  p.err = device_error_flag();
+  if (!p.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
+  p.wait_ns = wait_limit_ns();
+  int grid = (num_sms() / 2) * 2;
+  if (grid > 2 * p.num_items) grid = 2 * p.num_items;
+  if (grid < 2) return cudaErrorInvalidValue;
+  return g.B.mn_major ? launch_pair_t<true>(ma, mb, md, p, grid, family, s)
+                      : launch_pair_t<false>(ma, mb, md, p, grid, family, s);
+}
+
+}  // namespace poetx

@@ -48,6 +48,9 @@ static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};  // 2 s
 
 unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
+static std::atomic<int> g_gemm_pairs{1};
+bool gemm_pairs_enabled() { return g_gemm_pairs.load(std::memory_order_relaxed) != 0; }
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -274,6 +277,13 @@ int poetx_invert_perm(const int32_t* perm, int32_t n, int32_t* inv) {
     seen[(size_t)p] = 1;
   }
   for (int32_t i = 0; i < n; ++i) inv[perm[i]] = i;
+  return POETX_OK;
+}
+
+int poetx_set_gemm_pairs(int enable, int* previous) {
+  if (enable != 0 && enable != 1) return fail(POETX_ERR_INVALID_ARG, "enable must be 0 or 1");
+  const int old = g_gemm_pairs.exchange(enable);
+  if (previous) *previous = old;
   return POETX_OK;
 }
 

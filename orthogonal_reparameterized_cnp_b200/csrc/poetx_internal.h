@@ -238,6 +238,12 @@ struct UmmaGemm {
   int side_rows = 0, side_cols = 0;
 };
 cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t s);
+// The CTA-pair form (kernels_umma2.cu) for the plain merged-weight GEMMs: one batch entry,
+// no K split, A K-major, bf16 output, N % 256 == 0, dense output (ldd == N).
+bool umma_pair_eligible(const UmmaGemm& g);
+cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStream_t s);
+// whether launch_umma_gemm sends eligible GEMMs to the CTA-pair kernel (default: yes)
+bool gemm_pairs_enabled();
 // ksplit the launcher would choose for the given problem (used to size scratch).
 int umma_choose_ksplit(int M, int N, int K, int batch);
 

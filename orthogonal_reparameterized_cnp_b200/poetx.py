@@ -68,6 +68,7 @@ SIGNATURES = {
                                   _vp, _vp, _vp, _c_int, _vp, _c_size, _vp]),
     "poetx_device_status": (_c_int, [_vp]),
     "poetx_set_wait_limit": (_c_int, [_c_u64, ctypes.POINTER(_c_u64)]),
+    "poetx_set_gemm_pairs": (_c_int, [_c_int, ctypes.POINTER(_c_int)]),
     "poetx_selftest_wait_timeout": (_c_int, [_vp, _vp, _c_i32, _c_i32, _c_i32, _vp, _c_size,
                                              _vp]),
     "poetx_fma_probe": (_c_int, [_vp, _c_i32, _c_i32, _vp]),
@@ -176,6 +177,15 @@ def set_wait_limit(ns: int) -> int:
     prev = _c_u64(0)
     _check(_load().poetx_set_wait_limit(int(ns), ctypes.byref(prev)), "poetx_set_wait_limit")
     return int(prev.value)
+
+
+def set_gemm_pairs(enable: bool) -> bool:
+    """Merged-weight GEMMs on CTA pairs (True, the default) or single CTAs; returns the
+    previous setting."""
+    prev = ctypes.c_int(0)
+    _check(_load().poetx_set_gemm_pairs(int(bool(enable)), ctypes.byref(prev)),
+           "poetx_set_gemm_pairs")
+    return bool(prev.value)
 
 
 def cnp_workspace(nblk: int, b: int, k: int) -> int:

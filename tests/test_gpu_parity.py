@@ -241,6 +241,28 @@ def test_layer_bf16_llama1b_full():
     _check_full(out, s, inp, BF16_NORM)
 
 
+@pytest.mark.parametrize("n,m,T", [(1024, 1024, 1000), (512, 1536, 300), (1536, 512, 257)])
+def test_gemm_pairs_and_single_ctas_agree_with_the_oracle(n, m, T):
+    """The merged-weight GEMMs on CTA pairs (256 x 256 tiles over two SMs) and on single CTAs
+    both meet the bar against the oracle, with ragged token counts (M tails)."""
+    P = _P()
+    s = LayerShape(f"pairs-{n}x{m}", T=T, n=n, m=m, b=256, k=4, dtype="bf16", config_id=500)
+    inp = layer_inputs(s)
+    outs = {}
+    prev = P.set_gemm_pairs(True)
+    try:
+        for pairs in (True, False):
+            P.set_gemm_pairs(pairs)
+            out = run_layer(inp)
+            out.pop("layer")
+            outs[pairs] = out
+            _check_full(out, s, inp, BF16_NORM)
+    finally:
+        P.set_gemm_pairs(prev)
+    for key in ["y", "dx", "dG_P", "dG_R"]:
+        assert norm_max_err(outs[True][key], outs[False][key]) <= 1e-2, key
+
+
 def test_recompute_mode_matches_saved_mode():
     s = LayerShape("bf16-recompute", T=777, n=512, m=768, b=256, k=4, dtype="bf16", config_id=300)
     inp = layer_inputs(s)

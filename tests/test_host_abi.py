@@ -226,6 +226,16 @@ class _FakeW0:
     dtype = None
 
 
+def test_gemm_pairs_setter():
+    prev = P.set_gemm_pairs(False)
+    try:
+        assert P.set_gemm_pairs(True) is False
+        assert P.set_gemm_pairs(True) is True
+        assert P.lib().poetx_set_gemm_pairs(2, None) == P.POETX_ERR_INVALID_ARG
+    finally:
+        P.set_gemm_pairs(prev)
+
+
 def test_wait_limit_setter():
     prev = P.set_wait_limit(50_000_000)
     try:
