@@ -181,8 +181,8 @@ int poetx_cnp_fwd(const float* theta, float* G, void* G_bf16, int32_t nblk, int3
  *   Scratch: a fixed 32 MiB array of the library's own device memory, present on every
  *   GPU that loads the library until the process exits.  One block's forward scratch must
  *   fit it: (d + 2) b x b fp32 matrices plus 64 bytes of counters and a fixed 256 bytes,
- *   with d = floor((k + 1) / 2) -- every k <= 16 for b <= 512, k <= 5 for b = 1024;
- *   b = 1024 with k >= 6 returns POETX_ERR_WORKSPACE with a message.  Any number of
+ *   with d = floor((k + 1) / 2) -- every k <= 16 for b <= 512, k <= 10 for b = 1024;
+ *   b = 1024 with k >= 11 returns POETX_ERR_WORKSPACE with a message.  Any number of
  *   blocks is processed in chunks.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before any
