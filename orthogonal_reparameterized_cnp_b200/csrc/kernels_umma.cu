@@ -574,7 +574,8 @@ cudaError_t launch_umma_gemm(const UmmaGemm& g, const char* family, cudaStream_t
   const int64_t out_rows = g.d_split ? (int64_t)p.ksplit * (g.d_split / g.ldd)
                                      : (g.d_boff ? (int64_t)g.batch * (g.d_boff / g.ldd) : g.M);
   CUtensorMap md;
-  if (!make_out_map(&md, g.D, out_rows, g.ldd, g.ldd, g.out_f32 != 0)) return cudaErrorInvalidValue;
+  if (!make_out_map(&md, g.D, out_rows, g.d_cols ? g.d_cols : g.ldd, g.ldd, g.out_f32 != 0))
+    return cudaErrorInvalidValue;
   int grid = num_sms();
   if (grid > p.num_items) grid = p.num_items;
   // keep B resident when one item's whole B (K <= 256) fits and the items share it

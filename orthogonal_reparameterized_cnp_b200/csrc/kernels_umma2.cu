@@ -24,6 +24,15 @@
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of tile t overlap the main loop
 // of tile t + 1.  Loads carry no cluster multicast: each CTA loads distinct data.
 //
+// Int8 merged weight (Q8 instantiation, POET-XQ: the base weight kept in int8 and
+// dequantised where it is used): B is read from two bf16 panel buffers of panel_n rows of
+// N each, filled in turn by two extra warps per CTA.  Panel p + 1 is dequantised (every
+// CTA converts its share, then bumps ready[p + 1]) while the MMAs consume panel p; the
+// producers wait for ready[p] before loading a tile of panel p, and the leader's epilogue
+// counts consumed[p] per finished tile, so panel p + 2 overwrites buffer p & 1 only after
+// every tile of panel p has been multiplied.  The full bf16 weight never exists, and the
+// conversion (once per weight element) runs beside the MMAs.
+//
 // Every mbarrier wait is bounded (Params2::wait_ns): on a timeout the waiting role records
 // POETX_ERR_TIMEOUT in the device flag and leaves its loop; the CTAs then drain what they can
 // observe with short bounded waits, meet at a cluster barrier and free TMEM.
@@ -31,6 +40,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include "dequant_dev.cuh"
 #include "poetx_internal.h"
 #include "umma_ptx.cuh"
 
@@ -55,7 +65,17 @@ struct Params2 {
   int M, N, K, total_kc, tiles_m, tiles_n, num_items;
   int* err;
   unsigned long long wait_ns;
+  // Q8: int8 weight W0q [rows x ldq] with per-row scales; panels of panel_n along N
+  const int8_t* q;
+  long long ldq;
+  const float* scales;
+  __nv_bfloat16* panel[2];
+  long long panel_ld;
+  int panel_n, npanels;
+  int* ready;     // [npanels]: CTAs that finished their share of panel p
+  int* consumed;  // [npanels]: tiles of panel p whose MMAs completed
 };
+constexpr int kSideWarps2 = 2;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -150,6 +170,37 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
                : "memory");
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// orders this thread's generic-proxy global accesses with its async-proxy (TMA) ones
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// bounded wait until *cnt >= need (acquire)
+__device__ __noinline__ bool wait_count(const int* cnt, int need, int* err,
+                                        unsigned long long limit_ns) {
+  if (ld_acquire_gpu(cnt) >= need) return true;
+  const unsigned long long t0 = globaltimer();
+  unsigned spins = 0;
+  while (ld_acquire_gpu(cnt) < need) {
+    if ((++spins & 31u) == 0) {
+      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        atomicCAS(err, 0, (int)POETX_ERR_TIMEOUT);
+        return false;
+      }
+      __nanosleep(128);
+    }
+  }
+  return true;
+}
+
 template <bool B_MN>
 __device__ __forceinline__ uint32_t make_idesc_pair() {
   return (1u << 4)                              // D format: f32
@@ -161,10 +212,11 @@ __device__ __forceinline__ uint32_t make_idesc_pair() {
          | ((uint32_t)(256 >> 4) << 24);        // M = 256 (the pair)
 }
 
-template <bool B_MN>
-__global__ void __launch_bounds__(kPairThreads, 1)
+template <bool B_MN, bool Q8>
+__global__ void __launch_bounds__(kPairThreads + (Q8 ? 32 * kSideWarps2 : 0), 1)
     k_umma_gemm_pair(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmB1,
                      const __grid_constant__ CUtensorMap tmD, const Params2 p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -202,6 +254,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (Q8) prefetch_tmap(&tmB1);
     prefetch_tmap(&tmD);
   }
   if (warp == 1) {
@@ -219,10 +272,25 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // ------------------------------------------------------------ TMA producer (both CTAs)
     int it = 0;
     bool ok = true;
+    int seen = -1;  // highest panel known to be ready (Q8)
     for (int item = cid; ok && item < p.num_items; item += nclusters) {
       const int tm = item % p.tiles_m, tn = item / p.tiles_m;
       const int m0 = tm * 256 + (int)rank * kPairBM;
-      const int n0 = tn * kPairBN + (int)rank * (kPairBN / 2);
+      int n0 = tn * kPairBN + (int)rank * (kPairBN / 2);
+      const CUtensorMap* mapB = &tmB;
+      if (Q8) {
+        const int pan = (tn * kPairBN) / p.panel_n;
+        if (pan > seen) {
+          if (!wait_count(p.ready + pan, (int)gridDim.x, p.err, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // the panel's generic-proxy writes, then TMA reads
+          seen = pan;
+        }
+        n0 -= pan * p.panel_n;
+        mapB = (pan & 1) ? &tmB1 : &tmB;
+      }
       for (int kc = 0; kc < p.total_kc; ++kc, ++it) {
         const int s = it % kPairStages, r = it / kPairStages;
         if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err, p.wait_ns)) {
@@ -235,10 +303,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tma_load_2d_pair(sA + s * kPairA, &tmA, k, m0, fb);
         const uint32_t b_dst = sB + s * kPairB;
         if (!B_MN) {
-          tma_load_2d_pair(b_dst, &tmB, k, n0, fb);
+          tma_load_2d_pair(b_dst, mapB, k, n0, fb);
         } else {
-          tma_load_2d_pair(b_dst, &tmB, n0, k, fb);
-          tma_load_2d_pair(b_dst + 8192, &tmB, n0 + 64, k, fb);
+          tma_load_2d_pair(b_dst, mapB, n0, k, fb);
+          tma_load_2d_pair(b_dst + 8192, mapB, n0 + 64, k, fb);
         }
       }
     }
@@ -285,6 +353,35 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // every MMA issued here completes before TMEM is released
     umma_commit_pair(drain_bar);
     mbar_drain_wait(drain_bar, 0);
+  } else if (Q8 && warp >= 2 + kPairEpiWarps) {
+    // ------------------------------------------------------------ panel dequantisation
+    const int st = threadIdx.x - 32 * (2 + kPairEpiWarps);
+    for (int pan = 0; pan < p.npanels; ++pan) {
+      if (pan >= 2) {  // buffer pan & 1 still holds panel pan - 2 until all its tiles ran
+        const int cols = min(p.panel_n, p.N - (pan - 2) * p.panel_n);
+        const int need = p.tiles_m * (cols / kPairBN);
+        if (st == 0) wait_count(p.consumed + pan - 2, need, p.err, p.wait_ns);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSideWarps2) : "memory");
+        // a failed wait has set the flag: every side thread sees it after the barrier
+        if (*reinterpret_cast<volatile int*>(p.err) != 0) break;
+        fence_proxy_async_global();
+      }
+      const int n_first = pan * p.panel_n;
+      const int width = min(p.panel_n, p.N - n_first);
+      __nv_bfloat16* const dst = (pan & 1) ? p.panel[1] : p.panel[0];
+      const int64_t first = (int64_t)blockIdx.x * (32 * kSideWarps2) + st;
+      const int64_t stride = (int64_t)gridDim.x * (32 * kSideWarps2);
+      if (!B_MN)  // B rows n of W0' (rows of W0q), all K columns
+        dequant_rows2d(p.q + (int64_t)n_first * p.ldq, p.ldq, p.scales + n_first, dst, p.panel_ld,
+                       width, p.K, first, stride);
+      else        // columns n of W0' for every row k of W0q
+        dequant_rows2d(p.q + n_first, p.ldq, p.scales, dst, p.panel_ld, p.K, width, first,
+                       stride);
+      fence_proxy_async_global();
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kSideWarps2) : "memory");
+      if (st == 0) red_release_gpu(p.ready + pan, 1);
+    }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // warp w drains TMEM lane quadrant (w % 4) and column half (w - 2) / 4 of this CTA's
@@ -305,6 +402,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (!ready) break;
       tc_fence_after();
+      if (Q8 && leader && warp == 2 && lane == 0)  // the tile's operands are all consumed
+        red_release_gpu(p.consumed + (tn * kPairBN) / p.panel_n, 1);
       const int row0 = tm * 256 + (int)rank * kPairBM + q * 32;
       const int n0 = tn * kPairBN;
 #pragma unroll 1
@@ -377,10 +476,12 @@ bool map2d(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool B_MN>
-cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
-                          const Params2& p, int grid, const char* family, cudaStream_t s) {
-  auto kern = k_umma_gemm_pair<B_MN>;
+template <bool B_MN, bool Q8>
+cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb1,
+                          const CUtensorMap& md, const Params2& p, int grid, const char* family,
+                          cudaStream_t s) {
+  auto kern = k_umma_gemm_pair<B_MN, Q8>;
+  constexpr int threads = kPairThreads + (Q8 ? 32 * kSideWarps2 : 0);
   static bool attr_done[64] = {false};  // once per device, outside any stream capture
   int dev = 0;
   cudaGetDevice(&dev);
@@ -393,7 +494,7 @@ cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CU
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kPairThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = kPairSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -406,9 +507,44 @@ cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CU
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   begin_launch(family, s);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mb1, md, p);
   end_launch(family, s);
   return e;
+}
+
+// Largest grid (an even number of CTAs) whose clusters are all resident at once: the Q8
+// pipeline's CTAs wait for one another's panel shares, so none may wait for a slot.
+template <bool B_MN, bool Q8>
+int resident_pair_grid() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev]) return cache[dev];
+  int grid = (num_sms() / 2) * 2;
+  if (Q8) {
+    auto kern = k_umma_gemm_pair<B_MN, Q8>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(kPairThreads + 32 * kSideWarps2);
+      cfg.dynamicSmemBytes = kPairSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) == cudaSuccess && nc > 0 &&
+          2 * nc < grid)
+        grid = 2 * nc;
+    }
+  }
+  cache[dev] = grid;
+  return grid;
 }
 
 }  // namespace
@@ -416,8 +552,26 @@ cudaError_t launch_pair_t(const CUtensorMap& ma, const CUtensorMap& mb, const CU
 bool umma_pair_eligible(const UmmaGemm& g) {
   return g.batch == 1 && g.ksplit <= 1 && !g.A.mn_major && !g.out_f32 && g.side_rows == 0 &&
          g.N % kPairBN == 0 && g.M >= 256 && g.K >= kPairBK && g.ldd == g.N &&
+         (g.d_cols == 0 || g.d_cols == g.N) &&
          g.A.boff_k == 0 && g.A.boff_mn == 0 && g.B.boff_k == 0 && g.B.boff_mn == 0 &&
          g.d_boff == 0 && g.d_boff_col == 0 && g.d_split == 0;
+}
+
+static cudaError_t pair_params(const UmmaGemm& g, Params2* p) {
+  *p = Params2{};
+  p->M = g.M;
+  p->N = g.N;
+  p->K = g.K;
+  p->total_kc = (g.K + kPairBK - 1) / kPairBK;
+  p->tiles_m = (g.M + 255) / 256;
+  p->tiles_n = g.N / kPairBN;
+  const long long items = (long long)p->tiles_m * p->tiles_n;
+  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  p->num_items = (int)items;
+  p->err = device_error_flag();
+  if (!p->err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
+  p->wait_ns = wait_limit_ns();
+  return cudaSuccess;
 }
 
 cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStream_t s) {
@@ -431,23 +585,56 @@ cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStr
     return cudaErrorInvalidValue;
   if (!map2d(&md, g.D, g.M, g.N, g.ldd, 64u, 32u, true)) return cudaErrorInvalidValue;
   Params2 p;
-  p.M = g.M;
-  p.N = g.N;
-  p.K = g.K;
-  p.total_kc = (g.K + kPairBK - 1) / kPairBK;
-  p.tiles_m = (g.M + 255) / 256;
-  p.tiles_n = g.N / kPairBN;
-  const long long items = (long long)p.tiles_m * p.tiles_n;
-  if (items > 0x7fffffff) return cudaErrorInvalidValue;
-  p.num_items = (int)items;
-  p.err = device_error_flag();
-  if (!p.err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
-  p.wait_ns = wait_limit_ns();
+  cudaError_t e = pair_params(g, &p);
+  if (e != cudaSuccess) return e;
   int grid = (num_sms() / 2) * 2;
   if (grid > 2 * p.num_items) grid = 2 * p.num_items;
   if (grid < 2) return cudaErrorInvalidValue;
-  return g.B.mn_major ? launch_pair_t<true>(ma, mb, md, p, grid, family, s)
-                      : launch_pair_t<false>(ma, mb, md, p, grid, family, s);
+  return g.B.mn_major ? launch_pair_t<true, false>(ma, mb, mb, md, p, grid, family, s)
+                      : launch_pair_t<false, false>(ma, mb, mb, md, p, grid, family, s);
+}
+
+cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const char* family,
+                                     cudaStream_t s) {
+  // g.B describes the bf16 merged weight the panels come from (its shape and major-ness);
+  // its pointer is not read
+  if (!umma_pair_eligible(g) || !q.q || !q.scales || !q.panel[0] || !q.panel[1] ||
+      !q.counters || q.panel_n <= 0 || q.panel_n % kPairBN != 0)
+    return cudaErrorInvalidValue;
+  const bool b_mn = g.B.mn_major != 0;
+  const int npan = (g.N + q.panel_n - 1) / q.panel_n;
+  // panel layout: K-major B -> [panel_n rows (N) x K], row stride K; MN-major B ->
+  // [K rows x panel_n (N)], row stride panel_n
+  const int64_t prow = b_mn ? g.K : q.panel_n, pcol = b_mn ? q.panel_n : g.K;
+  if (q.ldq % 16 != 0 || pcol % 16 != 0 || (reinterpret_cast<uintptr_t>(q.q) & 15) ||
+      (reinterpret_cast<uintptr_t>(q.panel[0]) & 15) || (reinterpret_cast<uintptr_t>(q.panel[1]) & 15))
+    return cudaErrorInvalidValue;
+  CUtensorMap ma, mb0, mb1, md;
+  if (!map2d(&ma, g.A.ptr, g.A.rows, g.A.cols, g.A.ld, 64u, (uint32_t)kPairBM, false))
+    return cudaErrorInvalidValue;
+  if (!map2d(&mb0, q.panel[0], prow, pcol, pcol, 64u, b_mn ? 64u : 128u, false) ||
+      !map2d(&mb1, q.panel[1], prow, pcol, pcol, 64u, b_mn ? 64u : 128u, false))
+    return cudaErrorInvalidValue;
+  if (!map2d(&md, g.D, g.M, g.N, g.ldd, 64u, 32u, true)) return cudaErrorInvalidValue;
+  Params2 p;
+  cudaError_t e = pair_params(g, &p);
+  if (e != cudaSuccess) return e;
+  p.q = q.q;
+  p.ldq = q.ldq;
+  p.scales = q.scales;
+  p.panel[0] = static_cast<__nv_bfloat16*>(q.panel[0]);
+  p.panel[1] = static_cast<__nv_bfloat16*>(q.panel[1]);
+  p.panel_ld = pcol;
+  p.panel_n = q.panel_n;
+  p.npanels = npan;
+  p.ready = q.counters;
+  p.consumed = q.counters + npan;
+  const int grid = b_mn ? resident_pair_grid<true, true>() : resident_pair_grid<false, true>();
+  if (grid < 2) return cudaErrorInvalidValue;
+  e = cudaMemsetAsync(q.counters, 0, sizeof(int) * 2 * (size_t)npan, s);
+  if (e != cudaSuccess) return e;
+  return b_mn ? launch_pair_t<true, true>(ma, mb0, mb1, md, p, grid, family, s)
+              : launch_pair_t<false, true>(ma, mb0, mb1, md, p, grid, family, s);
 }
 
 }  // namespace poetx

@@ -984,17 +984,103 @@ cudaError_t bf16_w0(const void* in, const void* W0p, void* out, int T, int n, in
   return launch_umma_gemm(g, "gemm_w0", s);
 }
 
+// The merged weight of a layer call: bf16 W0' (q == nullptr), or its int8 codes with per-row
+// scales plus two bf16 panel buffers and the pipeline's counters (the int8 layer).
+struct W0Ref {
+  const void* bf16 = nullptr;
+  const int8_t* q = nullptr;
+  const float* s = nullptr;
+  void* panel[2] = {nullptr, nullptr};
+  int* counters = nullptr;
+  int panel_f = 0, panel_b = 0;  // panel widths (along N) of the forward / backward GEMMs
+};
+
+// Panels of the int8 weight along the GEMM's N: a multiple of 256, at most 32 MB of bf16
+// (K x width x 2 bytes), and at most a quarter of N (so two panels never hold more than half
+// of the weight) where N allows.
+constexpr size_t kPanelBytes = 32ull << 20;
+int q8_panel_width(int N, int K) {
+  int64_t w = (int64_t)(kPanelBytes / ((size_t)K * 2)) / 256 * 256;
+  const int64_t quarter = (int64_t)N / 4 / 256 * 256;
+  if (quarter >= 256 && w > quarter) w = quarter;
+  if (w < 256) w = 256;
+  const int64_t nr = ((int64_t)N + 255) / 256 * 256;
+  return (int)(w < nr ? w : nr);
+}
+struct Q8Layout {
+  int panel_f, panel_b;
+  size_t panel_bytes, counter_bytes, total;
+};
+Q8Layout q8_layout(const poetx_linear_desc* d) {
+  Q8Layout L;
+  L.panel_f = q8_panel_width(d->m, d->n);  // forward: N = m rows of W0', K = n
+  L.panel_b = q8_panel_width(d->n, d->m);  // backward: N = n columns of W0', K = m
+  const size_t ef = (size_t)L.panel_f * d->n, eb = (size_t)d->m * L.panel_b;
+  L.panel_bytes = align_up((ef > eb ? ef : eb) * 2);
+  const int np = (d->m + L.panel_f - 1) / L.panel_f, nq = (d->n + L.panel_b - 1) / L.panel_b;
+  L.counter_bytes = align_up(sizeof(int) * 2 * (size_t)(np > nq ? np : nq));
+  L.total = 2 * L.panel_bytes + L.counter_bytes;
+  return L;
+}
+
+// W = V W0'^T (forward) or dV = dW W0' (backward) for either form of the weight.
+cudaError_t w0_gemm(const void* in, const W0Ref& w, void* out, int T, int n, int m, bool forward,
+                    cudaStream_t s) {
+  if (!w.q) return bf16_w0(in, w.bf16, out, T, n, m, forward, s);
+  // the GEMM as it reads the bf16 merged weight (B's pointer is not used)
+  UmmaGemm g;
+  UmmaOperand B;
+  B.rows = m; B.cols = n; B.ld = n; B.mn_major = forward ? 0 : 1;
+  g.A = act_kmajor(in, T, forward ? n : m, 0);
+  g.B = B;
+  g.M = T; g.N = forward ? m : n; g.K = forward ? n : m;
+  g.batch = 1; g.out_f32 = 0;
+  g.D = out; g.ldd = g.N;
+  const int pw = forward ? w.panel_f : w.panel_b;
+  if (gemm_pairs_enabled() && umma_pair_eligible(g)) {
+    PairQ8 q;
+    q.q = w.q; q.ldq = n; q.scales = w.s;
+    q.panel[0] = w.panel[0]; q.panel[1] = w.panel[1];
+    q.panel_n = pw; q.counters = w.counters;
+    return launch_umma_gemm_pair_q8(g, q, "gemm_w0", s);
+  }
+  // other shapes: panel by panel, each dequantised and then multiplied (one panel buffer)
+  for (int p0 = 0; p0 < g.N; p0 += pw) {
+    const int width = g.N - p0 < pw ? g.N - p0 : pw;
+    cudaError_t e;
+    UmmaGemm h = g;
+    UmmaOperand P;
+    if (forward) {  // rows p0.. of W0': [width x n]
+      e = launch_dequant_2d(w.q + (int64_t)p0 * n, n, w.s + p0, w.panel[0], n, width, n, s);
+      P.ptr = w.panel[0]; P.rows = width; P.cols = n; P.ld = n; P.mn_major = 0;
+    } else {        // columns p0.. of W0': [m x width]
+      e = launch_dequant_2d(w.q + p0, n, w.s, w.panel[0], width, m, width, s);
+      P.ptr = w.panel[0]; P.rows = m; P.cols = width; P.ld = width; P.mn_major = 1;
+    }
+    if (e != cudaSuccess) return e;
+    h.B = P;
+    h.N = width;
+    h.D = static_cast<__nv_bfloat16*>(out) + p0;
+    h.ldd = g.N;
+    h.d_cols = width;
+    e = launch_umma_gemm(h, "gemm_w0", s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 // Forward body shared by poetx_linear_fwd and the recompute path of the backward.
 // Writes U (if U != x-gather target), V, W; Z and y only when y != nullptr.
 int forward_body(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
-                 const void* W0p, void* y, void* U, void* V, void* W, void* Z, cudaStream_t s) {
+                 const W0Ref& w0, void* y, void* U, void* V, void* W, void* Z, cudaStream_t s) {
+  const void* W0p = w0.bf16;
   const int T = d->T, n = d->n, m = d->m, b = d->b;
   const bool bf = d->dtype == POETX_BF16;
   const int es = bf ? 2 : 4;
   POETX_CUDA(launch_gather(x, U, nullptr, d->perm_P, T, n, n, n, es, s), "gather x");
   if (bf) {
     POETX_CUDA(bf16_blockdiag(U, G_P, V, T, n, b, false, s), "blockdiag G_P");
-    POETX_CUDA(bf16_w0(V, W0p, W, T, n, m, true, s), "W0' gemm");
+    POETX_CUDA(w0_gemm(V, w0, W, T, n, m, true, s), "W0' gemm");
     if (y) {
       POETX_CUDA(bf16_blockdiag(W, G_R, Z, T, m, b, false, s), "blockdiag G_R");
       POETX_CUDA(launch_gather(Z, y, nullptr, d->inv_R, T, m, m, m, es, s), "scatter y");
@@ -1031,13 +1117,17 @@ size_t poetx_linear_bwd_workspace(const poetx_linear_desc* d, int has_save_u, in
   return bwd_layout(d, has_save_u, has_save_w).total;
 }
 
-int poetx_linear_fwd(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
-                     const void* W0p, void* y, void* save_u, void* save_w, void* ws,
-                     size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+int linear_fwd_impl(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
+                    const W0Ref& w0, void* y, void* save_u, void* save_w, void* ws,
+                    size_t ws_bytes, void* stream) {
   int st = linear_validate(d);
   if (st != POETX_OK) return st;
   if (d->T == 0) return POETX_OK;
-  if ((st = check_ptrs({x, G_P, G_R, W0p, y})) != POETX_OK) return st;
+  if ((st = check_ptrs({x, G_P, G_R, w0.q ? (const void*)w0.q : w0.bf16, y})) != POETX_OK)
+    return st;
   if ((st = check_opt(save_u)) != POETX_OK || (st = check_opt(save_w)) != POETX_OK) return st;
   const FwdLayout L = fwd_layout(d, save_u != nullptr, save_w != nullptr);
   if (ws_bytes < L.total) return fail(POETX_ERR_WORKSPACE, "forward scratch too small");
@@ -1048,13 +1138,14 @@ int poetx_linear_fwd(const poetx_linear_desc* d, const void* x, const void* G_P,
   void* V = cv.take(L.V);
   void* W = save_w ? save_w : cv.take(L.W);
   void* Z = cv.take(L.Z);
-  return forward_body(d, x, G_P, G_R, W0p, y, U, V, W, Z, static_cast<cudaStream_t>(stream));
+  return forward_body(d, x, G_P, G_R, w0, y, U, V, W, Z, static_cast<cudaStream_t>(stream));
 }
 
-int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, const void* G_P,
-                     const void* G_R, const void* W0p, const void* save_u, const void* save_w,
-                     void* dx, float* dG_P, float* dG_R, int accumulate, void* ws,
-                     size_t ws_bytes, void* stream) {
+int linear_bwd_impl(const poetx_linear_desc* d, const void* x, const void* dy, const void* G_P,
+                    const void* G_R, const W0Ref& w0, const void* save_u, const void* save_w,
+                    void* dx, float* dG_P, float* dG_R, int accumulate, void* ws,
+                    size_t ws_bytes, void* stream) {
+  const void* W0p = w0.bf16;
   int st = linear_validate(d);
   if (st != POETX_OK) return st;
   if (accumulate != 0 && accumulate != 1)
@@ -1070,7 +1161,8 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
     }
     return POETX_OK;
   }
-  if ((st = check_ptrs({dy, G_P, G_R, W0p, dx})) != POETX_OK) return st;
+  if ((st = check_ptrs({dy, G_P, G_R, w0.q ? (const void*)w0.q : W0p, dx})) != POETX_OK)
+    return st;
   if ((st = check_opt(save_u)) != POETX_OK || (st = check_opt(save_w)) != POETX_OK) return st;
   if (!save_u || !save_w)
     if ((st = check_ptrs({x})) != POETX_OK) return st;
@@ -1092,7 +1184,7 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
   float* partP = static_cast<float*>(cv.take(L.partP));
   // recompute what the forward did not save (POET-X section 2.5, checkpointing)
   if (!save_w) {
-    st = forward_body(d, x, G_P, G_R, W0p, nullptr, U, Vr, W, nullptr, s);
+    st = forward_body(d, x, G_P, G_R, w0, nullptr, U, Vr, W, nullptr, s);
     if (st != POETX_OK) return st;
   } else if (!save_u) {
     POETX_CUDA(launch_gather(x, U, nullptr, d->perm_P, T, n, n, n, es, s), "gather x");
@@ -1103,7 +1195,7 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
     POETX_CUDA(bf16_blockdiag(dZ, G_R, dW, T, m, b, true, s), "blockdiag G_R^T");
     POETX_CUDA(bf16_block_grad(dZ, W, partR, dG_R, L.ksR, T, m, b, accumulate, s), "dG_R");
     // B2: dV = dW W0'
-    POETX_CUDA(bf16_w0(dW, W0p, dV, T, n, m, false, s), "W0' gemm (backward)");
+    POETX_CUDA(w0_gemm(dW, w0, dV, T, n, m, false, s), "W0' gemm (backward)");
     // B3: dU_j = dV_j G_P,j; dG_P,j = dV_j^T U_j; dX[:, p_P[i]] = dU[:, i]
     POETX_CUDA(bf16_blockdiag(dV, G_P, dU, T, n, b, true, s), "blockdiag G_P^T");
     POETX_CUDA(bf16_block_grad(dV, U, partP, dG_P, L.ksP, T, n, b, accumulate, s), "dG_P");
@@ -1125,6 +1217,27 @@ int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, 
   }
   POETX_CUDA(launch_gather(dU, dx, nullptr, d->inv_P, T, n, n, n, es, s), "scatter dx");
   return POETX_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int poetx_linear_fwd(const poetx_linear_desc* d, const void* x, const void* G_P, const void* G_R,
+                     const void* W0p, void* y, void* save_u, void* save_w, void* ws,
+                     size_t ws_bytes, void* stream) {
+  W0Ref w;
+  w.bf16 = W0p;
+  return linear_fwd_impl(d, x, G_P, G_R, w, y, save_u, save_w, ws, ws_bytes, stream);
+}
+
+int poetx_linear_bwd(const poetx_linear_desc* d, const void* x, const void* dy, const void* G_P,
+                     const void* G_R, const void* W0p, const void* save_u, const void* save_w,
+                     void* dx, float* dG_P, float* dG_R, int accumulate, void* ws,
+                     size_t ws_bytes, void* stream) {
+  W0Ref w;
+  w.bf16 = W0p;
+  return linear_bwd_impl(d, x, dy, G_P, G_R, w, save_u, save_w, dx, dG_P, dG_R, accumulate, ws,
+                         ws_bytes, stream);
 }
 
 size_t poetx_outer_merge_workspace(int32_t m, int32_t n, int dtype) {
@@ -1225,46 +1338,62 @@ int poetx_merge_perm_q8(const void* W0, int8_t* W0q, float* scales, int32_t m, i
 
 size_t poetx_linear_q8_scratch(const poetx_linear_desc* d) {
   if (!d || d->dtype != POETX_BF16 || d->m <= 0 || d->n <= 0) return 0;
-  return align_up((size_t)d->m * d->n * 2);
+  return q8_layout(d).total;
 }
+
+}  // extern "C"
+
+namespace {
+// validates the int8 weight arguments and carves the panels and counters from the front of
+// ws; the rest of ws is the layer call's own scratch
+int q8_weight(const poetx_linear_desc* d, const int8_t* W0q, const float* scales, void* ws,
+              size_t ws_bytes, W0Ref* w, void** rest, size_t* rest_bytes) {
+  int st = linear_validate(d);
+  if (st != POETX_OK) return st;
+  if (d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "int8 base weight needs bf16");
+  if (!W0q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W0q) || !aligned16(scales) || !aligned16(ws))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const Q8Layout L = q8_layout(d);
+  if (!ws || ws_bytes < L.total) return fail(POETX_ERR_WORKSPACE, "scratch too small");
+  Carve cv(ws);
+  w->q = W0q;
+  w->s = scales;
+  w->panel[0] = cv.take(L.panel_bytes);
+  w->panel[1] = cv.take(L.panel_bytes);
+  w->counters = static_cast<int*>(cv.take(L.counter_bytes));
+  w->panel_f = L.panel_f;
+  w->panel_b = L.panel_b;
+  *rest = static_cast<char*>(ws) + L.total;
+  *rest_bytes = ws_bytes - L.total;
+  return POETX_OK;
+}
+}  // namespace
+
+extern "C" {
 
 int poetx_linear_fwd_q8(const poetx_linear_desc* d, const void* x, const void* G_P,
                         const void* G_R, const int8_t* W0q, const float* scales, void* y,
                         void* save_u, void* save_w, void* ws, size_t ws_bytes, void* stream) {
-  int st = linear_validate(d);
+  W0Ref w;
+  void* rest = nullptr;
+  size_t rest_bytes = 0;
+  int st = q8_weight(d, W0q, scales, ws, ws_bytes, &w, &rest, &rest_bytes);
   if (st != POETX_OK) return st;
-  if (d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "int8 base weight needs bf16");
-  if (d->T == 0) return POETX_OK;
-  if (!W0q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(W0q) || !aligned16(scales) || !aligned16(ws))
-    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
-  const size_t q8 = poetx_linear_q8_scratch(d);
-  if (!ws || ws_bytes < q8) return fail(POETX_ERR_WORKSPACE, "scratch too small");
-  // the dequantised weight lives in the first part of the scratch for this call only
-  POETX_CUDA(launch_dequant_rows(W0q, scales, ws, d->m, d->n, static_cast<cudaStream_t>(stream)),
-             "dequantise W0'");
-  return poetx_linear_fwd(d, x, G_P, G_R, ws, y, save_u, save_w,
-                          static_cast<char*>(ws) + q8, ws_bytes - q8, stream);
+  return linear_fwd_impl(d, x, G_P, G_R, w, y, save_u, save_w, rest, rest_bytes, stream);
 }
 
 int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* dy,
                         const void* G_P, const void* G_R, const int8_t* W0q, const float* scales,
                         const void* save_u, const void* save_w, void* dx, float* dG_P,
                         float* dG_R, int accumulate, void* ws, size_t ws_bytes, void* stream) {
-  int st = linear_validate(d);
+  W0Ref w;
+  void* rest = nullptr;
+  size_t rest_bytes = 0;
+  int st = q8_weight(d, W0q, scales, ws, ws_bytes, &w, &rest, &rest_bytes);
   if (st != POETX_OK) return st;
-  if (d->dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "int8 base weight needs bf16");
-  if (!W0q || !scales) return fail(POETX_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(W0q) || !aligned16(scales) || !aligned16(ws))
-    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
-  const size_t q8 = poetx_linear_q8_scratch(d);
-  if (!ws || ws_bytes < q8) return fail(POETX_ERR_WORKSPACE, "scratch too small");
-  if (d->T > 0)
-    POETX_CUDA(launch_dequant_rows(W0q, scales, ws, d->m, d->n,
-                                   static_cast<cudaStream_t>(stream)),
-               "dequantise W0'");
-  return poetx_linear_bwd(d, x, dy, G_P, G_R, ws, save_u, save_w, dx, dG_P, dG_R, accumulate,
-                          static_cast<char*>(ws) + q8, ws_bytes - q8, stream);
+  return linear_bwd_impl(d, x, dy, G_P, G_R, w, save_u, save_w, dx, dG_P, dG_R, accumulate, rest,
+                         rest_bytes, stream);
 }
 
 int poetx_device_status(void* stream) {

@@ -227,6 +227,7 @@ struct UmmaGemm {
   int64_t d_boff_col = 0;     // per-batch column offset of D
   int64_t d_boff = 0;         // per-batch element offset of D
   int64_t d_split = 0;        // per-split element offset of D
+  int64_t d_cols = 0;         // columns of D (0: ldd); D may start inside a wider matrix
   // optional side job of two extra warps per CTA, run alongside the GEMM:
   // side_dst[r][c] = bf16(side_scales[r] * side_q[r][c]) for r < side_rows, c < side_cols
   // (the int8 weight's next panel while this panel is multiplied); side_rows = 0: none
@@ -244,6 +245,20 @@ bool umma_pair_eligible(const UmmaGemm& g);
 cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStream_t s);
 // whether launch_umma_gemm sends eligible GEMMs to the CTA-pair kernel (default: yes)
 bool gemm_pairs_enabled();
+// The CTA-pair GEMM with B from the int8 weight q (per-row scales; row stride ldq): B is the
+// bf16 merged weight that g.B describes, dequantised panel by panel (panel_n along N,
+// a multiple of 256) into two scratch panels while the MMAs run.  counters: 2 * ceil(N /
+// panel_n) ints of scratch (zeroed by the launcher).
+struct PairQ8 {
+  const int8_t* q = nullptr;
+  int64_t ldq = 0;
+  const float* scales = nullptr;
+  void* panel[2] = {nullptr, nullptr};
+  int panel_n = 0;
+  int* counters = nullptr;
+};
+cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const char* family,
+                                     cudaStream_t s);
 // ksplit the launcher would choose for the given problem (used to size scratch).
 int umma_choose_ksplit(int M, int N, int K, int batch);
 

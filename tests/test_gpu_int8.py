@@ -69,6 +69,49 @@ def test_merge_perm_q8_bit_exact(dtype, m, n):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
+@pytest.mark.parametrize("T,n,m", [(300, 512, 384), (600, 1024, 2048), (1000, 2048, 1024)])
+def test_int8_layer_equals_bf16_layer_on_the_dequantised_weight(T, n, m):
+    """The int8 entry points (weight dequantised panel by panel inside the GEMMs) give
+    exactly what the bf16 entry points give on bf16(s * q) as a whole weight: several
+    panels per GEMM, so the two panel buffers are reused."""
+    import torch
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    b = 256 if n % 256 == 0 and m % 256 == 0 else 128
+    s = LayerShape(f"xqeq-{n}x{m}", T=T, n=n, m=m, b=b, k=4, dtype="bf16", config_id=12,
+                   std_theta=0.01)
+    inp = layer_inputs(s)
+    pP, _ = P.make_perm(inp.seed_P, n)
+    pR, _ = P.make_perm(inp.seed_R, m)
+    L = P.PoetxLinear(tensor(inp.W0, torch.bfloat16), tensor(inp.theta_P, torch.float32),
+                      tensor(inp.theta_R, torch.float32), pP, pR, b, 4, T, int8_weight=True)
+    x = tensor(inp.x, torch.bfloat16)
+    dy = tensor(inp.dy, torch.bfloat16)
+    L.cnp_forward()
+    y8 = torch.empty((T, m), dtype=torch.bfloat16, device="cuda")
+    dx8 = torch.empty((T, n), dtype=torch.bfloat16, device="cuda")
+    L.forward(x, y8)
+    L.backward(x, dy, dx8)
+    dG8 = L.dG.clone()
+    # the same layer on the dequantised weight through the bf16 entry points
+    Wdq = (L.scales[:, None] * L.W0q.float()).to(torch.bfloat16).contiguous()
+    GP, GR = L.G_ops()
+    ws = torch.empty(max(P.linear_fwd_workspace(L.desc), P.linear_bwd_workspace(L.desc)),
+                     dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(y8)
+    dx = torch.empty_like(dx8)
+    U = torch.empty_like(L.U)
+    Ws = torch.empty_like(L.Wsave)
+    dG_P = torch.empty_like(L.dG[: L.nP])
+    dG_R = torch.empty_like(L.dG[L.nP:])
+    P.linear_fwd(L.desc, x, GP, GR, Wdq, y, U, Ws, ws)
+    P.linear_bwd(L.desc, x, dy, GP, GR, Wdq, U, Ws, dx, dG_P, dG_R, 0, ws)
+    torch.cuda.synchronize()
+    assert P.device_status() == P.POETX_OK
+    assert torch.equal(y8, y)
+    assert torch.equal(dx8, dx)
+    assert torch.equal(dG8[: L.nP], dG_P) and torch.equal(dG8[L.nP:], dG_R)
+
+
 @pytest.mark.parametrize("T,n,m,b", [(256, 512, 384, 128), (320, 512, 768, 256)])
 def test_int8_layer_matches_oracle(T, n, m, b):
     import torch
