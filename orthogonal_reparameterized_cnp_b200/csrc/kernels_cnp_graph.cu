@@ -60,10 +60,29 @@ static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory per SM");
 constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
 
 // ---- 128 x 128 items ----------------------------------------------------------------
+// Tuning knobs (defaults measured best on B200): k slice depth, cp.async stages, unrolling
+// of the k steps of a slice, CTAs per SM, register double-buffering of the operand
+// fragments.
+#ifndef CNP2_BK
+#define CNP2_BK 16
+#endif
+#ifndef CNP2_STAGES
+#define CNP2_STAGES 4
+#endif
+#ifndef CNP2_KUNROLL
+#define CNP2_KUNROLL CNP2_BK
+#endif
+#ifndef CNP2_CTAS
+#define CNP2_CTAS 2
+#endif
+#ifndef CNP2_DBUF
+#define CNP2_DBUF 0
+#endif
 constexpr int k2Threads = 256;  // 16 x 16 threads, 8 x 8 outputs each
-constexpr int k2BK = 16;
+constexpr int k2BK = CNP2_BK;
 constexpr int k2LD = 128 + 4;  // row stride of a staged k slice (16-byte aligned rows)
-constexpr int k2Stages = 4;
+constexpr int k2Stages = CNP2_STAGES;
+constexpr int k2KUnroll = CNP2_KUNROLL;
 constexpr int k2StageFloats = 2 * k2BK * k2LD;
 constexpr int k2RingFloats = k2Stages * k2StageFloats;  // 66 KB
 // epilogue operands (the adds and the skew term, <= 3 tiles) of one 64 x 64 quadrant are
@@ -75,7 +94,7 @@ constexpr int k2EpiFloats = 2 * k2QBufFloats;  // 102 KB
 constexpr int k2MaxFloats = k2RingFloats > k2EpiFloats ? k2RingFloats : k2EpiFloats;
 constexpr int k2SmemFloats = k2MaxFloats > kPairFloats ? k2MaxFloats : kPairFloats;
 constexpr int k2SmemBytes = k2SmemFloats * 4;
-static_assert(2 * (k2SmemBytes + 1024) <= 227 * 1024, "two CTAs per SM");
+static_assert(CNP2_CTAS * (k2SmemBytes + 1024) <= 228 * 1024, "CTAs per SM");
 
 template <int TILE>
 struct GraphCfg;
@@ -85,7 +104,7 @@ struct GraphCfg<64> {
 };
 template <>
 struct GraphCfg<128> {
-  static constexpr int threads = k2Threads, ctas_per_sm = 2, smem = k2SmemBytes;
+  static constexpr int threads = k2Threads, ctas_per_sm = CNP2_CTAS, smem = k2SmemBytes;
 };
 
 __device__ __forceinline__ void cp_async16(float* smem_dst, const float* gsrc) {
@@ -464,7 +483,7 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
       float* As = As_(kt % k2Stages);
       float* Bs = Bs_(kt % k2Stages);
 #pragma unroll
-      for (int l = 0; l < 2; ++l) {
+      for (int l = 0; l < k2BK * 32 / k2Threads; ++l) {
         const int f = tid + l * k2Threads;
         const int r = f >> 5, c4 = (f & 31) * 4;
         cp_async16(As + r * k2LD + c4, A + (int64_t)(k0 + r) * b + m0 + c4);
@@ -487,7 +506,28 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
     }
     const float* As = As_(kt % k2Stages);
     const float* Bs = Bs_(kt % k2Stages);
+#if CNP2_DBUF
+    float4 a0 = *reinterpret_cast<const float4*>(As + ty * 4);
+    float4 a1 = *reinterpret_cast<const float4*>(As + 64 + ty * 4);
+    float4 b0 = *reinterpret_cast<const float4*>(Bs + tx * 4);
+    float4 b1 = *reinterpret_cast<const float4*>(Bs + 64 + tx * 4);
+#pragma unroll k2KUnroll
+    for (int k = 0; k < k2BK; ++k) {
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      if (k + 1 < k2BK) {  // the next k step's fragments load while this one computes
+        a0 = *reinterpret_cast<const float4*>(As + (k + 1) * k2LD + ty * 4);
+        a1 = *reinterpret_cast<const float4*>(As + (k + 1) * k2LD + 64 + ty * 4);
+        b0 = *reinterpret_cast<const float4*>(Bs + (k + 1) * k2LD + tx * 4);
+        b1 = *reinterpret_cast<const float4*>(Bs + (k + 1) * k2LD + 64 + tx * 4);
+      }
 #pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+    }
+#else
+#pragma unroll k2KUnroll
     for (int k = 0; k < k2BK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(As + k * k2LD + ty * 4);
       const float4 a1 = *reinterpret_cast<const float4*>(As + k * k2LD + 64 + ty * 4);
@@ -500,6 +540,7 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
     }
+#endif
   }
   cp_wait<0>();
 
@@ -937,6 +978,14 @@ cudaError_t launch_graph_t(const CnpGraph& g, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_fill_ints(int* p, int n, int first, const char* family, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  begin_launch(family, s);
+  const cudaError_t e = launch_pdl(k_zero_ints, dim3((n + 255) / 256), dim3(256), 0, s, p, n, first);
+  end_launch(family, s);
+  return e;
+}
 
 cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;

@@ -26,8 +26,9 @@
 //
 // Int8 merged weight (Q8 instantiation, POET-XQ: the base weight kept in int8 and
 // dequantised where it is used): B is read from two bf16 panel buffers of panel_n rows of
-// N each, filled in turn by two extra warps per CTA.  Panel p + 1 is dequantised (every
-// CTA converts its share, then bumps ready[p + 1]) while the MMAs consume panel p; the
+// N each.  Panel 0 is dequantised by a short kernel launched just before; the others by two
+// extra warps per CTA: panel p + 1 is dequantised (every CTA converts its share, then bumps
+// ready[p + 1]) while the MMAs consume panel p; the
 // producers wait for ready[p] before loading a tile of panel p, and the leader's epilogue
 // counts consumed[p] per finished tile, so panel p + 2 overwrites buffer p & 1 only after
 // every tile of panel p has been multiplied.  The full bf16 weight never exists, and the
@@ -74,7 +75,27 @@ struct Params2 {
   int panel_n, npanels;
   int* ready;     // [npanels]: CTAs that finished their share of panel p
   int* consumed;  // [npanels]: tiles of panel p whose MMAs completed
+  int group_m;    // tile raster: groups of group_m M-tiles swept over every N-tile (0: N-major)
 };
+
+// Tile (tm, tn) of the pair's item-th output tile.  group_m > 0: items run through groups of
+// group_m M-tiles, N-tile by N-tile inside a group, so the tiles in flight at one time share
+// a few A row blocks and B column blocks (both stay in L2); group_m = 0: all M-tiles of an
+// N-tile before the next N-tile (the int8 pipeline consumes the weight panel by panel).
+__device__ __forceinline__ void pair_tile(const Params2& p, int item, int& tm, int& tn) {
+  if (p.group_m <= 0) {
+    tm = item % p.tiles_m;
+    tn = item / p.tiles_m;
+    return;
+  }
+  const int per_group = p.group_m * p.tiles_n;
+  const int g = item / per_group;
+  const int first = g * p.group_m;
+  const int gm = min(p.tiles_m - first, p.group_m);
+  const int local = item - g * per_group;
+  tm = first + local % gm;
+  tn = local / gm;
+}
 constexpr int kSideWarps2 = 2;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -274,7 +295,8 @@ __global__ void __launch_bounds__(kPairThreads + (Q8 ? 32 * kSideWarps2 : 0), 1)
     bool ok = true;
     int seen = -1;  // highest panel known to be ready (Q8)
     for (int item = cid; ok && item < p.num_items; item += nclusters) {
-      const int tm = item % p.tiles_m, tn = item / p.tiles_m;
+      int tm, tn;
+      pair_tile(p, item, tm, tn);
       const int m0 = tm * 256 + (int)rank * kPairBM;
       int n0 = tn * kPairBN + (int)rank * (kPairBN / 2);
       const CUtensorMap* mapB = &tmB;
@@ -356,7 +378,7 @@ __global__ void __launch_bounds__(kPairThreads + (Q8 ? 32 * kSideWarps2 : 0), 1)
   } else if (Q8 && warp >= 2 + kPairEpiWarps) {
     // ------------------------------------------------------------ panel dequantisation
     const int st = threadIdx.x - 32 * (2 + kPairEpiWarps);
-    for (int pan = 0; pan < p.npanels; ++pan) {
+    for (int pan = 1; pan < p.npanels; ++pan) {  // panel 0 arrives dequantised
       if (pan >= 2) {  // buffer pan & 1 still holds panel pan - 2 until all its tiles ran
         const int cols = min(p.panel_n, p.N - (pan - 2) * p.panel_n);
         const int need = p.tiles_m * (cols / kPairBN);
@@ -395,7 +417,8 @@ __global__ void __launch_bounds__(kPairThreads + (Q8 ? 32 * kSideWarps2 : 0), 1)
     const uint32_t sw = (uint32_t)(lane & 7);
     int tcount = 0;
     for (int item = cid; item < p.num_items; item += nclusters, ++tcount) {
-      const int tm = item % p.tiles_m, tn = item / p.tiles_m;
+      int tm, tn;
+      pair_tile(p, item, tm, tn);
       const int acc = tcount & 1, ra = tcount >> 1;
       int ready = 0;
       if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err, p.wait_ns) ? 1 : 0;
@@ -571,6 +594,7 @@ static cudaError_t pair_params(const UmmaGemm& g, Params2* p) {
   p->err = device_error_flag();
   if (!p->err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
   p->wait_ns = wait_limit_ns();
+  p->group_m = 8;
   return cudaSuccess;
 }
 
@@ -629,9 +653,15 @@ cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const c
   p.npanels = npan;
   p.ready = q.counters;
   p.consumed = q.counters + npan;
+  p.group_m = 0;  // panel after panel
   const int grid = b_mn ? resident_pair_grid<true, true>() : resident_pair_grid<false, true>();
   if (grid < 2) return cudaErrorInvalidValue;
-  e = cudaMemsetAsync(q.counters, 0, sizeof(int) * 2 * (size_t)npan, s);
+  // counters: ready[0] = grid (panel 0 is filled below), everything else 0
+  e = launch_fill_ints(q.counters, 2 * npan, grid, family, s);
+  if (e != cudaSuccess) return e;
+  const int w0 = npan > 1 ? q.panel_n : g.N;
+  e = b_mn ? launch_dequant_2d(q.q, q.ldq, q.scales, q.panel[0], pcol, g.K, w0, s)
+           : launch_dequant_2d(q.q, q.ldq, q.scales, q.panel[0], pcol, w0, g.K, s);
   if (e != cudaSuccess) return e;
   return b_mn ? launch_pair_t<true, true>(ma, mb0, mb1, md, p, grid, family, s)
               : launch_pair_t<false, true>(ma, mb0, mb1, md, p, grid, family, s);

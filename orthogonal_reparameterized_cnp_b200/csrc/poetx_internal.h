@@ -151,6 +151,9 @@ cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, fl
 // fp32 -> bf16 (round to nearest even)
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s);
 
+// p[0] = first, p[1..n) = 0 (kernels_cnp_graph.cu)
+cudaError_t launch_fill_ints(int* p, int n, int first, const char* family, cudaStream_t s);
+
 // ---- CNP as one persistent task-graph launch (kernels_cnp_graph.cu) -----------------
 // Each job is one step applied to every block of a chunk; an item is one output tile of
 // one job for one block.  Square blocks with b % 64 == 0; products read every A operand
