@@ -525,27 +525,30 @@ def family_attribution(P, wl, stream, reps):
     return out
 
 
-def w0_single_cta(P, wl, stream, reps):
-    """The merged-weight GEMMs of one step on single CTAs (128 x 256 tiles) instead of CTA
-    pairs, from CUDA-graph replays with events around each launch (for comparison)."""
+def single_cta(P, wl, stream, reps, families=("gemm_w0", "gemm_blockdiag")):
+    """The tensor-core families of one step on single CTAs instead of CTA pairs, from
+    CUDA-graph replays with events around each launch (for comparison)."""
     import torch
+    out = {}
     prev = P.set_gemm_pairs(False)
     try:
-        P.profile_begin("gemm_w0")
-        g = graph_of(lambda st: wl.step(0, st), stream)
-        P.profile_begin(None)
-        tot, launches = 0.0, 0
-        for _ in range(reps):
-            g.replay()
-            torch.cuda.synchronize()
-            n, ms = P.profile_end()
-            tot += ms
-            launches = n
-        del g
+        for fam in families:
+            P.profile_begin(fam)
+            g = graph_of(lambda st: wl.step(0, st), stream)
+            P.profile_begin(None)
+            tot, launches = 0.0, 0
+            for _ in range(reps):
+                g.replay()
+                torch.cuda.synchronize()
+                n, ms = P.profile_end()
+                tot += ms
+                launches = n
+            del g
+            out[fam] = {"launches_per_step": launches, "ms_per_step": tot / reps}
     finally:
         P.set_gemm_pairs(prev)
-    check_status(P, stream, "the single-CTA GEMM replays")
-    return {"launches_per_step": launches, "ms_per_step": tot / reps}
+    check_status(P, stream, "the single-CTA replays")
+    return out
 
 
 def cnp_only(P, wl, stream, reps):
@@ -726,10 +729,13 @@ def run_poetx(args):
     work = family_work(shapes)
     breakdown = family_attribution(P, wl, stream, reps=min(reps, 20))
     if wl.bf16:
-        alt = w0_single_cta(P, wl, stream, reps=min(reps, 20))
-        ww = family_work(shapes)["gemm_w0"]
-        alt["achieved_tflops"] = ww["flops"] / (alt["ms_per_step"] / 1e3) / 1e12
-        breakdown["gemm_w0_single_cta"] = alt
+        fw = family_work(shapes)
+        for fam, alt in single_cta(P, wl, stream, reps=min(reps, 20)).items():
+            if "flops" in fw[fam]:
+                alt["achieved_tflops"] = fw[fam]["flops"] / (alt["ms_per_step"] / 1e3) / 1e12
+            if "bytes" in fw[fam]:
+                alt["achieved_gbs"] = fw[fam]["bytes"] / (alt["ms_per_step"] / 1e3) / 1e9
+            breakdown[fam + "_single_cta"] = alt
     dominant = max(FAMILIES, key=lambda f: breakdown[f]["ms_per_step"])
     peaks, peak_src = load_peaks()
     wkey = workload_name(args.workload, shapes)

@@ -75,28 +75,33 @@ struct Params2 {
   int panel_n, npanels;
   int* ready;     // [npanels]: CTAs that finished their share of panel p
   int* consumed;  // [npanels]: tiles of panel p whose MMAs completed
-  int group_m;    // tile raster: groups of group_m M-tiles swept over every N-tile (0: N-major)
+  int group_m;    // tile raster: groups of group_m M-tiles swept over the N-tiles
 };
 
-// Tile (tm, tn) of the pair's item-th output tile.  group_m > 0: items run through groups of
-// group_m M-tiles, N-tile by N-tile inside a group, so the tiles in flight at one time share
-// a few A row blocks and B column blocks (both stay in L2); group_m = 0: all M-tiles of an
-// N-tile before the next N-tile (the int8 pipeline consumes the weight panel by panel).
+constexpr int kSideWarps2 = 2;
+
+// Tile (tm, tn) of the pair's item-th output tile.  Tiles run through groups of group_m
+// M-tiles, N-tile by N-tile inside a group, so the tiles in flight at one time share a few A
+// row blocks and B column blocks (both stay in L2).  With the int8 weight (npanels > 0) the
+// groups are formed inside each weight panel and the panels follow one another, since the
+// pipeline consumes the weight panel by panel.
 __device__ __forceinline__ void pair_tile(const Params2& p, int item, int& tm, int& tn) {
-  if (p.group_m <= 0) {
-    tm = item % p.tiles_m;
-    tn = item / p.tiles_m;
-    return;
+  int tn0 = 0, ntn = p.tiles_n, local = item;
+  if (p.npanels > 0) {
+    const int tpp = p.panel_n / kPairBN;  // N-tiles per full panel
+    const int pan = item / (p.tiles_m * tpp);
+    tn0 = pan * tpp;
+    ntn = min(tpp, p.tiles_n - tn0);
+    local = item - pan * p.tiles_m * tpp;
   }
-  const int per_group = p.group_m * p.tiles_n;
-  const int g = item / per_group;
+  const int per_group = p.group_m * ntn;
+  const int g = local / per_group;
   const int first = g * p.group_m;
   const int gm = min(p.tiles_m - first, p.group_m);
-  const int local = item - g * per_group;
-  tm = first + local % gm;
-  tn = local / gm;
+  const int l2 = local - g * per_group;
+  tm = first + l2 % gm;
+  tn = tn0 + l2 / gm;
 }
-constexpr int kSideWarps2 = 2;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -883,7 +888,6 @@ cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const c
   p.npanels = npan;
   p.ready = q.counters;
   p.consumed = q.counters + npan;
-  p.group_m = 0;  // panel after panel
   const int grid = b_mn ? resident_pair_grid<true, true>() : resident_pair_grid<false, true>();
   if (grid < 2) return cudaErrorInvalidValue;
   // counters: ready[0] = grid (panel 0 is filled below), everything else 0
