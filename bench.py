@@ -525,8 +525,8 @@ def family_attribution(P, wl, stream, reps):
     return out
 
 
-def single_cta(P, wl, stream, reps, families=("gemm_w0", "gemm_blockdiag")):
-    """The tensor-core families of one step on single CTAs instead of CTA pairs, from
+def single_cta(P, wl, stream, reps, families=("gemm_w0",)):
+    """The merged-weight GEMMs of one step on single CTAs instead of CTA pairs, from
     CUDA-graph replays with events around each launch (for comparison)."""
     import torch
     out = {}

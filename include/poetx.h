@@ -347,12 +347,12 @@ int poetx_linear_bwd_q8(const poetx_linear_desc* d, const void* x, const void* d
 int poetx_set_wait_limit(uint64_t ns, uint64_t* previous);
 
 /*
- * Kernel choice for the tensor-core products: 1 (the default) runs the merged-weight GEMMs
- * (W = V W0'^T, dV = dW W0') on CTA pairs (tcgen05 cta_group::2, 256 x 256 tiles shared by
- * two SMs) when the shape allows (N % 256 == 0, M >= 256), and the block-diagonal products
- * with b = 256 on CTA pairs (each SM holding half of G_j); 0 runs all of them on single
- * CTAs (128 x 256 tiles).  Both compute the same products; the switch exists to compare
- * them.  Applies to launches made after the call.
+ * Kernel choice for the merged-weight GEMMs (W = V W0'^T, dV = dW W0'): 1 (the default)
+ * runs them on CTA pairs (tcgen05 cta_group::2, 256 x 256 tiles shared by two SMs) when
+ * the shape allows (N % 256 == 0, M >= 256); 0 runs them on single CTAs (128 x 256 tiles).
+ * The block-diagonal and dG products always run on single CTAs.  Both forms compute the
+ * same products; the switch exists to compare them.  Applies to launches made after the
+ * call.
  *   previous: receives the setting before this call (may be NULL).
  *   Errors: POETX_ERR_INVALID_ARG for a value other than 0 or 1.
  */

@@ -440,6 +440,25 @@ __device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem
 // stored with 16-byte row stores, and the mirror of a symmetric (or symmetric + skew)
 // result is stored from the same registers as 16-byte column segments (four consecutive
 // rows of the thread become four consecutive columns of the mirrored row).
+// One k slice of the 128 x 128 item: acc[r][c] += A[k][row r] B[k][col c] for the thread's
+// rows {4 ty + r} U {64 + 4 ty + r} and columns {4 tx + c} U {64 + 4 tx + c}.
+__device__ __forceinline__ void kslice128(float (&acc)[8][8], const float* As, const float* Bs,
+                                          int tx, int ty) {
+#pragma unroll k2KUnroll
+  for (int k = 0; k < k2BK; ++k) {
+    const float4 a0 = *reinterpret_cast<const float4*>(As + k * k2LD + ty * 4);
+    const float4 a1 = *reinterpret_cast<const float4*>(As + k * k2LD + 64 + ty * 4);
+    const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * k2LD + tx * 4);
+    const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * k2LD + 64 + tx * 4);
+    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
+  }
+}
+
 __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* smem) {
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
@@ -527,19 +546,7 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
         for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
     }
 #else
-#pragma unroll k2KUnroll
-    for (int k = 0; k < k2BK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(As + k * k2LD + ty * 4);
-      const float4 a1 = *reinterpret_cast<const float4*>(As + k * k2LD + 64 + ty * 4);
-      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * k2LD + tx * 4);
-      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * k2LD + 64 + tx * 4);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
-    }
+    kslice128(acc, As, Bs, tx, ty);
 #endif
   }
   cp_wait<0>();

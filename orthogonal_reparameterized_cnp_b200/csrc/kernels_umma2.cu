@@ -474,236 +474,6 @@ __global__ void __launch_bounds__(kPairThreads + (Q8 ? 32 * kSideWarps2 : 0), 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kPairTmemCols);
 }
 
-// ------------------------------------------------------------------ block-diagonal products
-// The batched block-diagonal products of the layer (V_j = U_j G_j^T, Z_j = W_j G_j^T and the
-// backward's dW_j = dZ_j G_j, dU_j = dV_j G_j; technical summary section 2.3) for b = 256 on
-// CTA pairs.  A pair's item is 256 tokens of one block j: D[t, 256 j + n] = sum_k
-// A[t, 256 j + k] B_j[n][k].  Each CTA keeps its half of B_j (128 rows of n, all 256 k:
-// 64 KB) resident while the pair walks consecutive token tiles of the same block, and
-// streams its 128 token rows of A through an 8-stage ring (128 KB in flight per SM, which
-// the HBM latency needs; a single CTA holding all of G_j has room for only 4 stages).
-constexpr int kBdStages = 8;
-constexpr int kBdA = kPairBM * kPairBK * 2;           // 16 KB: 128 token rows x 64 k
-constexpr int kBdB = (kPairBN / 2) * kPairBK * 2;     // 16 KB: one k chunk of B's half
-constexpr int kBdRing = kBdStages * kBdA;
-constexpr int kBdRes = 4 * kBdB;                      // K = 256
-constexpr int kBdSmem = 1024 + kBdRing + kBdRes + kPairEpi + 256;
-static_assert(kBdSmem <= 227 * 1024, "shared memory per CTA");
-
-struct ParamsBd {
-  int T, width, nblk, tiles_m, num_items;
-  int* err;
-  unsigned long long wait_ns;
-};
-
-template <bool B_MN>
-__global__ void __launch_bounds__(kPairThreads, 1)
-    k_umma_blockdiag_pair(const __grid_constant__ CUtensorMap tmA,
-                          const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmD, const ParamsBd p) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sA = base;                        // ring: stages x 16 KB
-  const uint32_t sB = base + kBdRing;              // resident half of B_j: 4 x 16 KB
-  const uint32_t sEpi = sB + kBdRes;
-  const uint32_t sBar = sEpi + kPairEpi;
-  auto full_bar = [&](int s) { return sBar + 8u * s; };
-  auto empty_bar = [&](int s) { return sBar + 8u * (kBdStages + s); };
-  auto tfull_bar = [&](int a) { return sBar + 8u * (2 * kBdStages + a); };
-  auto tempty_bar = [&](int a) { return sBar + 8u * (2 * kBdStages + 2 + a); };
-  const uint32_t bfull_bar = sBar + 8u * (2 * kBdStages + 4);
-  const uint32_t bempty_bar = sBar + 8u * (2 * kBdStages + 5);
-  const uint32_t drain_bar = sBar + 8u * (2 * kBdStages + 6);
-  const uint32_t tmem_slot = sBar + 8u * (2 * kBdStages + 7);
-  unsigned char* generic_base = smem_raw + (base - raw);
-  volatile uint32_t* tmem_slot_ptr =
-      reinterpret_cast<volatile uint32_t*>(generic_base + (tmem_slot - base));
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const bool leader = rank == 0;
-  const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-  // a contiguous range of items per pair, so that consecutive items share B_j
-  const int first = (int)(((long long)cid * p.num_items) / nclusters);
-  const int last = (int)(((long long)(cid + 1) * p.num_items) / nclusters);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kBdStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 2 * kPairEpiWarps);
-    }
-    mbar_init(bfull_bar, 1);
-    mbar_init(bempty_bar, 1);
-    mbar_init(drain_bar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmD);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, kPairTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot_ptr;
-  pdl_trigger();
-  pdl_wait();
-
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    int it = 0, brun = -1, cur = -1;
-    bool ok = true;
-    for (int item = first; ok && item < last; ++item) {
-      const int j = item / p.tiles_m, tm = item - j * p.tiles_m;
-      if (j != cur) {  // this CTA's half of B_j, once the previous block's MMAs are done
-        ++brun;
-        if (!mbar_wait(bempty_bar, (brun & 1) ^ 1, p.err, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        if (leader) mbar_expect_tx(bfull_bar, 2u * kBdRes);
-        const uint32_t fb = map_to_rank(bfull_bar, 0);
-#pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
-          const uint32_t dst = sB + kc * kBdB;
-          if (!B_MN) {  // B_j[n][k] = G_j[n][k]: rows of G
-            tma_load_2d_pair(dst, &tmB, kc * kPairBK, j * 256 + (int)rank * 128, fb);
-          } else {      // B_j[n][k] = G_j[k][n]: columns of G
-            tma_load_2d_pair(dst, &tmB, (int)rank * 128, j * 256 + kc * kPairBK, fb);
-            tma_load_2d_pair(dst + 8192, &tmB, (int)rank * 128 + 64, j * 256 + kc * kPairBK, fb);
-          }
-        }
-        cur = j;
-      }
-      const int row0 = tm * 256 + (int)rank * kPairBM;
-      for (int kc = 0; kc < 4; ++kc, ++it) {
-        const int s = it % kBdStages, r = it / kBdStages;
-        if (!mbar_wait(empty_bar(s), (r & 1) ^ 1, p.err, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        if (leader) mbar_expect_tx(full_bar(s), 2u * kBdA);
-        tma_load_2d_pair(sA + s * kBdA, &tmA, j * 256 + kc * kPairBK, row0,
-                         map_to_rank(full_bar(s), 0));
-      }
-    }
-    if (!ok && leader) {
-      for (int q = (it > kBdStages ? it - kBdStages : 0); q < it; ++q)
-        mbar_drain_wait(full_bar(q % kBdStages), (q / kBdStages) & 1);
-      if (brun >= 0) mbar_drain_wait(bfull_bar, brun & 1);
-    }
-  } else if (warp == 1 && lane == 0 && leader) {
-    // ------------------------------------------------------------ MMA issuer (leader)
-    const uint32_t idesc = make_idesc_pair<B_MN>();
-    int it = 0, tcount = 0, brun = -1, cur = -1;
-    bool ok = true;
-    for (int item = first; ok && item < last; ++item, ++tcount) {
-      const int j = item / p.tiles_m;
-      if (j != cur) {
-        ++brun;
-        if (!mbar_wait(bfull_bar, brun & 1, p.err, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        cur = j;
-      }
-      const int acc = tcount & 1, ra = tcount >> 1;
-      if (!mbar_wait_cluster(tempty_bar(acc), (ra & 1) ^ 1, p.err, p.wait_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kPairBN);
-      for (int kc = 0; kc < 4; ++kc, ++it) {
-        const int s = it % kBdStages, r = it / kBdStages;
-        if (!mbar_wait(full_bar(s), r & 1, p.err, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t a_addr = sA + s * kBdA;
-        const uint32_t b_addr = sB + kc * kBdB;
-#pragma unroll
-        for (int kk = 0; kk < kPairBK / 16; ++kk) {
-          const uint64_t adesc = make_desc(a_addr + kk * 32, 16, 1024);
-          const uint64_t bdesc = B_MN ? make_desc(b_addr + kk * 2048, 8192, 1024)
-                                      : make_desc(b_addr + kk * 32, 16, 1024);
-          umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit_pair_mc(empty_bar(s), (uint16_t)0x3);
-      }
-      if (!ok) break;
-      umma_commit_pair_mc(tfull_bar(acc), (uint16_t)0x3);
-      if (item + 1 >= last || (item + 1) / p.tiles_m != j)
-        umma_commit_pair_mc(bempty_bar, (uint16_t)0x3);  // both halves of B_j reusable
-    }
-    umma_commit_pair(drain_bar);
-    mbar_drain_wait(drain_bar, 0);
-  } else if (warp >= 2) {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
-    constexpr int HALF = kPairBN / 2;
-    const uint32_t stage = sEpi + (uint32_t)(warp - 2) * 4096u;
-    const uint32_t my_row = stage + (uint32_t)lane * 128u;
-    const uint32_t sw = (uint32_t)(lane & 7);
-    int tcount = 0;
-    for (int item = first; item < last; ++item, ++tcount) {
-      const int j = item / p.tiles_m, tm = item - j * p.tiles_m;
-      const int acc = tcount & 1, ra = tcount >> 1;
-      int ready = 0;
-      if (lane == 0) ready = mbar_wait(tfull_bar(acc), ra & 1, p.err, p.wait_ns) ? 1 : 0;
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      if (!ready) break;
-      tc_fence_after();
-      const int row0 = tm * 256 + (int)rank * kPairBM + q * 32;
-#pragma unroll 1
-      for (int c = half * HALF; c < (half + 1) * HALF; c += 64) {
-        uint32_t v[64];
-        tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kPairBN + c), v);
-        tmem_wait_ld();
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          uint32_t o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(v[8 * k + 2 * e]),
-                                                      __uint_as_float(v[8 * k + 2 * e + 1]));
-            o[e] = *reinterpret_cast<uint32_t*>(&hh);
-          }
-          sts128(my_row + (((uint32_t)k ^ sw) << 4), o[0], o[1], o[2], o[3]);
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmD, j * 256 + c, row0, stage);
-          bulk_commit();
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_to_rank(tempty_bar(acc), 0));
-    }
-    if (lane == 0) bulk_wait0();
-    __syncwarp();
-  }
-
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem_base, kPairTmemCols);
-}
-
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -899,67 +669,6 @@ cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const c
   if (e != cudaSuccess) return e;
   return b_mn ? launch_pair_t<true, true>(ma, mb0, mb1, md, p, grid, family, s)
               : launch_pair_t<false, true>(ma, mb0, mb1, md, p, grid, family, s);
-}
-
-cudaError_t launch_blockdiag_pair(const void* in, const void* G, void* out, int T, int width,
-                                  int b, bool transposeG, const char* family, cudaStream_t s) {
-  if (T <= 0 || width <= 0) return cudaSuccess;
-  if (b != 256 || width % 256 != 0) return cudaErrorInvalidValue;
-  const int nblk = width / 256;
-  CUtensorMap ma, mb, md;
-  if (!map2d(&ma, in, T, width, width, 64u, (uint32_t)kPairBM, false)) return cudaErrorInvalidValue;
-  // G as one [nblk * 256, 256] matrix.  transposeG = false: D_j = A_j G_j^T, B_j[n][k] =
-  // G_j[n][k], 64 k x 128 n-row boxes (K-major B); transposeG = true: D_j = A_j G_j,
-  // B_j[n][k] = G_j[k][n], 64 n x 64 k-row boxes (MN-major B)
-  if (!map2d(&mb, G, (int64_t)nblk * 256, 256, 256, 64u, transposeG ? 64u : 128u, false))
-    return cudaErrorInvalidValue;
-  if (!map2d(&md, out, T, width, width, 64u, 32u, true)) return cudaErrorInvalidValue;
-  ParamsBd p;
-  p.T = T;
-  p.width = width;
-  p.nblk = nblk;
-  p.tiles_m = (T + 255) / 256;
-  const long long items = (long long)nblk * p.tiles_m;
-  if (items > 0x7fffffff) return cudaErrorInvalidValue;
-  p.num_items = (int)items;
-  p.err = device_error_flag();
-  if (!p.err) return cudaErrorInvalidDevice;
-  p.wait_ns = wait_limit_ns();
-  int grid = (num_sms() / 2) * 2;
-  if (grid > 2 * p.num_items) grid = 2 * p.num_items;
-  if (grid < 2) return cudaErrorInvalidValue;
-  auto launch = [&](auto kern) -> cudaError_t {
-    static bool attr_done[2][64] = {{false}};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    const int which = transposeG ? 0 : 1;
-    if (!attr_done[which][dev]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kBdSmem);
-      if (e != cudaSuccess) return e;
-      attr_done[which][dev] = true;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kPairThreads);
-    cfg.dynamicSmemBytes = kBdSmem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    begin_launch(family, s);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
-    end_launch(family, s);
-    return e;
-  };
-  return transposeG ? launch(k_umma_blockdiag_pair<true>) : launch(k_umma_blockdiag_pair<false>);
 }
 
 }  // namespace poetx

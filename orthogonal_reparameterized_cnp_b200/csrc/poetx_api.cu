@@ -931,8 +931,6 @@ UmmaOperand act_mnmajor(const void* p, int T, int width, int64_t boff_mn) {
 }
 cudaError_t bf16_blockdiag(const void* in, const void* G, void* out, int T, int width, int b,
                            bool transposeG, cudaStream_t s) {
-  if (b == 256 && gemm_pairs_enabled())
-    return launch_blockdiag_pair(in, G, out, T, width, b, transposeG, "gemm_blockdiag", s);
   const int nblk = width / b;
   UmmaGemm g;
   g.A = act_kmajor(in, T, width, b);

@@ -248,11 +248,7 @@ bool umma_pair_eligible(const UmmaGemm& g);
 cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStream_t s);
 // whether launch_umma_gemm sends eligible GEMMs to the CTA-pair kernel (default: yes)
 bool gemm_pairs_enabled();
-// Block-diagonal products with b = 256 on CTA pairs: out[:, 256 j + n] = sum_k
-// in[:, 256 j + k] (transposeG ? G_j[k][n] : G_j[n][k]); in, out [T, width] row-major bf16,
-// G [width / 256, 256, 256] bf16.
-cudaError_t launch_blockdiag_pair(const void* in, const void* G, void* out, int T, int width,
-                                  int b, bool transposeG, const char* family, cudaStream_t s);
+
 // The CTA-pair GEMM with B from the int8 weight q (per-row scales; row stride ldq): B is the
 // bf16 merged weight that g.B describes, dequantised panel by panel (panel_n along N,
 // a multiple of 256) into two scratch panels while the MMAs run.  counters: 2 * ceil(N /
