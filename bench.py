@@ -501,13 +501,13 @@ def check_status(P, stream, where):
         raise RuntimeError(f"device status not OK after {where}")
 
 
-def family_attribution(P, wl, stream, reps):
+def family_attribution(P, wl, stream, reps, families=None):
     """Per-family device time of one step from CUDA-graph replays: the step is captured
     once per family with CUDA events around that family's launches (event nodes of the
     graph), replayed `reps` times, and the bracketed times of each replay summed."""
     import torch
     out = {}
-    for fam in FAMILIES:
+    for fam in families or FAMILIES:
         P.profile_begin(fam)
         g = graph_of(lambda st: wl.step(0, st), stream)
         P.profile_begin(None)
@@ -857,8 +857,11 @@ def run_poetx(args):
         time_graphs(gq, 3, stream)
         qms = time_graphs(gq, reps, stream) / reps
         check_status(P, stream, "the int8-weight steps")
+        qfam = family_attribution(P, wq, stream, min(reps, 20), families=("gemm_w0",))
         xq = {"ms_per_step": qms, "tokens_per_s": T / (qms / 1e3), "steps": reps,
-              "weight": "int8 W0' (per-row scales)"}
+              "weight": "int8 W0' (per-row scales), converted to bf16 in shared memory "
+                        "inside the W0' GEMMs",
+              "gemm_w0_ms_per_step": qfam["gemm_w0"]["ms_per_step"]}
         del gq, wq
         torch.cuda.empty_cache()
 

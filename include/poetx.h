@@ -313,15 +313,15 @@ int poetx_merge_perm_q8(const void* W0, int8_t* W0q, float* scales, int32_t m, i
 /*
  * The bf16 layer with the int8 merged weight (codes and scales from poetx_merge_perm_q8 or
  * poetx_quantize_rows of W0').  The weight is dequantised where the two W0' GEMMs use it,
- * bf16(scales[i] * q[i, j]) (fp32 product, round to nearest even), panel by panel along the
- * GEMM's N: two bf16 panel buffers of at most 32 MB each (and at most a quarter of the
- * weight when its N allows) are filled in turn by two extra warps of the tensor-core kernel
- * while its MMAs consume the other panel, so the bf16 weight never exists as a whole.
- * Shapes the CTA-pair kernel does not take (N % 256 != 0 or fewer than 256 tokens) run the
- * panels one after another (dequantise, then multiply).  The first
- * poetx_linear_q8_scratch(d) bytes of ws hold the panels and the pipeline's counters; the
- * rest is the layer call's scratch, so ws_bytes must be at least poetx_linear_q8_scratch(d)
- * + poetx_linear_{fwd,bwd}_workspace(d, ...).  Results equal poetx_linear_fwd / _bwd run on
+ * bf16(scales[i] * q[i, j]) (fp32 product, round to nearest even): the tensor-core kernel
+ * loads each weight tile as int8 and converts it in shared memory just before its MMAs, so
+ * no bf16 copy of the weight is written to device memory.  Shapes the CTA-pair kernel does
+ * not take (N % 256 != 0, fewer than 256 tokens, n % 16 != 0, or pairs switched off with
+ * poetx_set_gemm_pairs) instead dequantise one panel of the weight at a time (at most 32 MB
+ * of bf16, at most a quarter of the weight when its N allows) into scratch and multiply it.
+ * The first poetx_linear_q8_scratch(d) bytes of ws hold that panel buffer; the rest is the
+ * layer call's scratch, so ws_bytes must be at least poetx_linear_q8_scratch(d) +
+ * poetx_linear_{fwd,bwd}_workspace(d, ...).  Results equal poetx_linear_fwd / _bwd run on
  * the dequantised weight.
  *   W0q device int8 [m, n], scales device fp32 [m]: read.  Other arguments as the bf16
  *   entry points.  d->dtype must be POETX_BF16 (else DTYPE).

@@ -986,14 +986,6 @@ cudaError_t launch_graph_t(const CnpGraph& g, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_fill_ints(int* p, int n, int first, const char* family, cudaStream_t s) {
-  if (n <= 0) return cudaSuccess;
-  begin_launch(family, s);
-  const cudaError_t e = launch_pdl(k_zero_ints, dim3((n + 255) / 256), dim3(256), 0, s, p, n, first);
-  end_launch(family, s);
-  return e;
-}
-
 cudaError_t launch_cnp_graph(CnpGraph g, cudaStream_t s) {
   if (g.njobs <= 0 || g.nblk <= 0) return cudaSuccess;
   for (int j = 0; j < g.njobs; ++j) {  // shapes the tile code relies on

@@ -985,13 +985,13 @@ cudaError_t bf16_w0(const void* in, const void* W0p, void* out, int T, int n, in
 }
 
 // The merged weight of a layer call: bf16 W0' (q == nullptr), or its int8 codes with per-row
-// scales plus two bf16 panel buffers and the pipeline's counters (the int8 layer).
+// scales (the int8 layer) plus one bf16 panel buffer for the shapes that the CTA-pair kernel
+// does not take.
 struct W0Ref {
   const void* bf16 = nullptr;
   const int8_t* q = nullptr;
   const float* s = nullptr;
-  void* panel[2] = {nullptr, nullptr};
-  int* counters = nullptr;
+  void* panel = nullptr;
   int panel_f = 0, panel_b = 0;  // panel widths (along N) of the forward / backward GEMMs
 };
 
@@ -1009,7 +1009,7 @@ int q8_panel_width(int N, int K) {
 }
 struct Q8Layout {
   int panel_f, panel_b;
-  size_t panel_bytes, counter_bytes, total;
+  size_t panel_bytes, total;
 };
 Q8Layout q8_layout(const poetx_linear_desc* d) {
   Q8Layout L;
@@ -1017,9 +1017,7 @@ Q8Layout q8_layout(const poetx_linear_desc* d) {
   L.panel_b = q8_panel_width(d->n, d->m);  // backward: N = n columns of W0', K = m
   const size_t ef = (size_t)L.panel_f * d->n, eb = (size_t)d->m * L.panel_b;
   L.panel_bytes = align_up((ef > eb ? ef : eb) * 2);
-  const int np = (d->m + L.panel_f - 1) / L.panel_f, nq = (d->n + L.panel_b - 1) / L.panel_b;
-  L.counter_bytes = align_up(sizeof(int) * 2 * (size_t)(np > nq ? np : nq));
-  L.total = 2 * L.panel_bytes + L.counter_bytes;
+  L.total = L.panel_bytes;
   return L;
 }
 
@@ -1036,14 +1034,12 @@ cudaError_t w0_gemm(const void* in, const W0Ref& w, void* out, int T, int n, int
   g.M = T; g.N = forward ? m : n; g.K = forward ? n : m;
   g.batch = 1; g.out_f32 = 0;
   g.D = out; g.ldd = g.N;
-  const int pw = forward ? w.panel_f : w.panel_b;
-  if (gemm_pairs_enabled() && umma_pair_eligible(g)) {
+  if (gemm_pairs_enabled() && umma_pair_eligible(g) && n % 16 == 0) {  // converted on chip
     PairQ8 q;
     q.q = w.q; q.ldq = n; q.scales = w.s;
-    q.panel[0] = w.panel[0]; q.panel[1] = w.panel[1];
-    q.panel_n = pw; q.counters = w.counters;
     return launch_umma_gemm_pair_q8(g, q, "gemm_w0", s);
   }
+  const int pw = forward ? w.panel_f : w.panel_b;
   // other shapes: panel by panel, each dequantised and then multiplied (one panel buffer)
   for (int p0 = 0; p0 < g.N; p0 += pw) {
     const int width = g.N - p0 < pw ? g.N - p0 : pw;
@@ -1051,11 +1047,11 @@ cudaError_t w0_gemm(const void* in, const W0Ref& w, void* out, int T, int n, int
     UmmaGemm h = g;
     UmmaOperand P;
     if (forward) {  // rows p0.. of W0': [width x n]
-      e = launch_dequant_2d(w.q + (int64_t)p0 * n, n, w.s + p0, w.panel[0], n, width, n, s);
-      P.ptr = w.panel[0]; P.rows = width; P.cols = n; P.ld = n; P.mn_major = 0;
+      e = launch_dequant_2d(w.q + (int64_t)p0 * n, n, w.s + p0, w.panel, n, width, n, s);
+      P.ptr = w.panel; P.rows = width; P.cols = n; P.ld = n; P.mn_major = 0;
     } else {        // columns p0.. of W0': [m x width]
-      e = launch_dequant_2d(w.q + p0, n, w.s, w.panel[0], width, m, width, s);
-      P.ptr = w.panel[0]; P.rows = m; P.cols = width; P.ld = width; P.mn_major = 1;
+      e = launch_dequant_2d(w.q + p0, n, w.s, w.panel, width, m, width, s);
+      P.ptr = w.panel; P.rows = m; P.cols = width; P.ld = width; P.mn_major = 1;
     }
     if (e != cudaSuccess) return e;
     h.B = P;
@@ -1344,8 +1340,8 @@ size_t poetx_linear_q8_scratch(const poetx_linear_desc* d) {
 }  // extern "C"
 
 namespace {
-// validates the int8 weight arguments and carves the panels and counters from the front of
-// ws; the rest of ws is the layer call's own scratch
+// validates the int8 weight arguments and carves the panel buffer from the front of ws; the
+// rest of ws is the layer call's own scratch
 int q8_weight(const poetx_linear_desc* d, const int8_t* W0q, const float* scales, void* ws,
               size_t ws_bytes, W0Ref* w, void** rest, size_t* rest_bytes) {
   int st = linear_validate(d);
@@ -1359,9 +1355,7 @@ int q8_weight(const poetx_linear_desc* d, const int8_t* W0q, const float* scales
   Carve cv(ws);
   w->q = W0q;
   w->s = scales;
-  w->panel[0] = cv.take(L.panel_bytes);
-  w->panel[1] = cv.take(L.panel_bytes);
-  w->counters = static_cast<int*>(cv.take(L.counter_bytes));
+  w->panel = cv.take(L.panel_bytes);
   w->panel_f = L.panel_f;
   w->panel_b = L.panel_b;
   *rest = static_cast<char*>(ws) + L.total;

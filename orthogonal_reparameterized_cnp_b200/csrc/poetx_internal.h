@@ -151,9 +151,6 @@ cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, fl
 // fp32 -> bf16 (round to nearest even)
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s);
 
-// p[0] = first, p[1..n) = 0 (kernels_cnp_graph.cu)
-cudaError_t launch_fill_ints(int* p, int n, int first, const char* family, cudaStream_t s);
-
 // ---- CNP as one persistent task-graph launch (kernels_cnp_graph.cu) -----------------
 // Each job is one step applied to every block of a chunk; an item is one output tile of
 // one job for one block.  Square blocks with b % 64 == 0; products read every A operand
@@ -250,16 +247,12 @@ cudaError_t launch_umma_gemm_pair(const UmmaGemm& g, const char* family, cudaStr
 bool gemm_pairs_enabled();
 
 // The CTA-pair GEMM with B from the int8 weight q (per-row scales; row stride ldq): B is the
-// bf16 merged weight that g.B describes, dequantised panel by panel (panel_n along N,
-// a multiple of 256) into two scratch panels while the MMAs run.  counters: 2 * ceil(N /
-// panel_n) ints of scratch (zeroed by the launcher).
+// bf16 merged weight that g.B describes, each tile converted to bf16(s * q) in shared memory
+// between its int8 load and the MMAs (no scratch).
 struct PairQ8 {
-  const int8_t* q = nullptr;
+  const int8_t* q = nullptr;  // W0q, row stride ldq (a multiple of 16)
   int64_t ldq = 0;
   const float* scales = nullptr;
-  void* panel[2] = {nullptr, nullptr};
-  int panel_n = 0;
-  int* counters = nullptr;
 };
 cudaError_t launch_umma_gemm_pair_q8(const UmmaGemm& g, const PairQ8& q, const char* family,
                                      cudaStream_t s);

@@ -69,11 +69,23 @@ def test_merge_perm_q8_bit_exact(dtype, m, n):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
-@pytest.mark.parametrize("T,n,m", [(300, 512, 384), (600, 1024, 2048), (1000, 2048, 1024)])
-def test_int8_layer_equals_bf16_layer_on_the_dequantised_weight(T, n, m):
-    """The int8 entry points (weight dequantised panel by panel inside the GEMMs) give
-    exactly what the bf16 entry points give on bf16(s * q) as a whole weight: several
-    panels per GEMM, so the two panel buffers are reused."""
+@pytest.mark.parametrize("T,n,m,pairs", [(300, 512, 384, True), (600, 1024, 2048, True),
+                                         (1000, 2048, 1024, True), (600, 1024, 2048, False)])
+def test_int8_layer_equals_bf16_layer_on_the_dequantised_weight(T, n, m, pairs):
+    """The int8 entry points give exactly what the bf16 entry points give on bf16(s * q) as a
+    whole weight: the CTA-pair kernel converting int8 tiles in shared memory (both operand
+    layouts, ragged token counts), and the panel-by-panel form that other shapes take (m =
+    384 forward, and every GEMM with pairs switched off: several panels per GEMM)."""
+    import torch
+    from orthogonal_reparameterized_cnp_b200 import poetx as P
+    prev = P.set_gemm_pairs(pairs)
+    try:
+        _int8_equals_bf16(T, n, m)
+    finally:
+        P.set_gemm_pairs(prev)
+
+
+def _int8_equals_bf16(T, n, m):
     import torch
     from orthogonal_reparameterized_cnp_b200 import poetx as P
     b = 256 if n % 256 == 0 and m % 256 == 0 else 128
