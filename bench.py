@@ -58,10 +58,13 @@ FAMILIES = ["gemm_w0", "gemm_blockdiag", "gemm_dG", "permute", "cnp_sgemm", "cnp
 WORKLOADS = ["llama13b-block", "llama8b-up", "llama1b-attn", "fp32-small"]
 # kernel source of each family: a committed DRAM-traffic figure applies only while the
 # source it was captured from is unchanged
+# the sources whose kernels a family's launches run (a committed traffic figure is used only
+# while all of them are unchanged)
 FAMILY_SOURCES = {
-    "gemm_w0": "kernels_umma.cu", "gemm_blockdiag": "kernels_umma.cu",
-    "gemm_dG": "kernels_umma.cu", "permute": "kernels_perm.cu",
-    "cnp_sgemm": "kernels_cnp_graph.cu", "reduce": "kernels_sgemm.cu",
+    "gemm_w0": ("kernels_umma2.cu", "kernels_umma.cu", "umma_ptx.cuh"),
+    "gemm_blockdiag": ("kernels_umma.cu", "umma_ptx.cuh"),
+    "gemm_dG": ("kernels_umma.cu", "umma_ptx.cuh"), "permute": ("kernels_perm.cu",),
+    "cnp_sgemm": ("kernels_cnp_graph.cu",), "reduce": ("kernels_sgemm.cu",),
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.md")
 
@@ -110,10 +113,14 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json on this box)"
 
 
-def source_sha(fname: str) -> str:
-    path = os.path.join(ROOT, "orthogonal_reparameterized_cnp_b200", "csrc", fname)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(fnames) -> str:
+    """First 16 hex digits of the SHA-256 of the named kernel sources, concatenated."""
+    h = hashlib.sha256()
+    for fname in ((fnames,) if isinstance(fnames, str) else fnames):
+        with open(os.path.join(ROOT, "orthogonal_reparameterized_cnp_b200", "csrc", fname),
+                  "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def committed_traffic(family: str, workload_key: str):

@@ -102,6 +102,9 @@ static_assert(kConvGroups <= PairCfg<true>::RB, "converter groups");
 static_assert(PairCfg<true>::threads <= 1024, "threads");
 constexpr uint32_t kPairTmemCols = 2 * kPairBN;
 
+#ifndef PAIR_GROUP_M
+#define PAIR_GROUP_M 8  // M-tiles per raster group
+#endif
 struct Params2 {
   int M, N, K, total_kc, tiles_m, tiles_n, num_items;
   int* err;
@@ -169,6 +172,17 @@ __device__ __forceinline__ void q8_chunk_to_bf16(const uint4 w, float s, uint32_
     o[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hi);
   }
 }
+// MN-major int8 tile (64 K rows of 8 chunks of 16 codes): chunk index ch -> (K row kr, chunk
+// c).  Each run of 16 indices covers two rows; its first 8 take chunks 0-3 of the first row
+// and 4-7 of the second, the next 8 the other halves.  Any 8 consecutive indices then read 8
+// different 16-byte bank groups of the staging tile (c differs) and write 8 different ones
+// of the two operand boxes (box c / 4 of either row, whose swizzles differ in bit 0).
+__device__ __forceinline__ void mn_chunk(int ch, int& kr, int& c) {
+  const int j = ch & 15, half = j >> 3, i = j & 7;
+  kr = 2 * (ch >> 4) + (i >> 2);
+  c = (i & 3) | ((((i >> 2) ^ half) & 1) << 2);
+}
+
 // AND of v over the `count` threads meeting at named barrier `id`
 __device__ __forceinline__ bool group_all(bool v, int id, int count) {
   uint32_t r;
@@ -509,12 +523,12 @@ __global__ void __launch_bounds__(PairCfg<Q8>::threads, 1)
     // arrival per CTA on the leader's fullB barrier, and frees the slot.
     //
     // Each 8 KB tile is 512 chunks of 16 codes; group thread gt converts chunks gt +
-    // kGroupThreads * jj.  K-major B (forward): staging rows are N rows of 64 codes, and row n
-    // of the operand is 128 bytes with 16-byte chunk c stored at c ^ (n & 7).  MN-major B
-    // (backward): staging rows are K rows of 128 codes (N), and the operand is two boxes (N
-    // 0-63, 64-127) of 64 K rows of 128 bytes, chunk c of row k stored at c ^ (k & 7).  A
-    // warp's 32 loads cover 512 contiguous staging bytes and its stores spread evenly over the
-    // 32 banks.
+    // kGroupThreads * jj.  K-major B (forward): staging rows are N rows of 64 codes (chunk
+    // ch = 4 n + c), and row n of the operand is 128 bytes with 16-byte chunk c stored at
+    // c ^ (n & 7).  MN-major B (backward): staging rows are K rows of 128 codes (N), chunk ch
+    // mapped to (row, chunk) by mn_chunk, and the operand is two boxes (N 0-63, 64-127) of 64
+    // K rows of 128 bytes, chunk c of row k stored at c ^ (k & 7).  In both layouts every 8
+    // lanes of a warp load from 8 different bank groups and store to 8 different ones.
     const int cw = threadIdx.x - 32 * (3 + EPI);
     const int grp = cw / kGroupThreads, gt = cw % kGroupThreads;
     const int bar_id = 1 + grp;  // named barrier of the group
@@ -545,7 +559,9 @@ __global__ void __launch_bounds__(PairCfg<Q8>::threads, 1)
       } else {      // the scale follows the K row
 #pragma unroll
         for (int jj = 0; jj < kConvChunks; ++jj) {
-          const int o = k + ((gt + kGroupThreads * jj) >> 3);
+          int kr, c;
+          mn_chunk(gt + kGroupThreads * jj, kr, c);
+          const int o = k + kr;
           // rows past K hold zero codes
           sc[jj] = (o < p.K && gt + kGroupThreads * jj < kTileChunks) ? __ldg(p.scales + o) : 0.f;
         }
@@ -573,15 +589,18 @@ __global__ void __launch_bounds__(PairCfg<Q8>::threads, 1)
         const int ch = gt + kGroupThreads * jj;
         if (kTileChunks % kGroupThreads != 0 && ch >= kTileChunks) break;
         uint32_t o[8];
-        q8_chunk_to_bf16(lds128(src + ch * 16), sc[jj], o);
         uint32_t row, c0, c1;
         if (!B_MN) {
+          q8_chunk_to_bf16(lds128(src + ch * 16), sc[jj], o);
           const uint32_t n = (uint32_t)ch >> 2, c = (uint32_t)ch & 3u;
           row = dst + n * 128u;
           c0 = (2u * c) ^ (n & 7u);
           c1 = (2u * c + 1u) ^ (n & 7u);
         } else {
-          const uint32_t kr = (uint32_t)ch >> 3, c = (uint32_t)ch & 7u;
+          int kr_, c_;
+          mn_chunk(ch, kr_, c_);
+          const uint32_t kr = (uint32_t)kr_, c = (uint32_t)c_;
+          q8_chunk_to_bf16(lds128(src + (kr * 8u + c) * 16u), sc[jj], o);
           row = dst + (c >> 2) * 8192u + kr * 128u;
           c0 = (2u * (c & 3u)) ^ (kr & 7u);
           c1 = (2u * (c & 3u) + 1u) ^ (kr & 7u);
@@ -777,7 +796,7 @@ static cudaError_t pair_params(const UmmaGemm& g, Params2* p) {
   p->err = device_error_flag();
   if (!p->err) return cudaErrorInvalidDevice;  // the bounded waits need the flag
   p->wait_ns = wait_limit_ns();
-  p->group_m = 8;
+  p->group_m = PAIR_GROUP_M;
   return cudaSuccess;
 }
 

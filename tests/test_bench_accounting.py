@@ -59,7 +59,9 @@ def test_cnp_flops_per_block(k, fwd, bwd):
 
 def test_committed_traffic_is_tied_to_the_kernel_source(tmp_path, monkeypatch):
     import bench
-    sha = bench.source_sha("kernels_umma.cu")
+    sha = bench.source_sha(bench.FAMILY_SOURCES["gemm_w0"])
+    # a change in any source of the family makes the row stale
+    assert sha != bench.source_sha(bench.FAMILY_SOURCES["gemm_w0"][:1])
     f = tmp_path / "t.md"
     f.write_text(f"| gemm_w0 | wl-a | 1.5e9 | {sha} | note |\n"
                  f"| gemm_w0 | wl-b | 2.0e9 | {'0' * 16} | stale |\n")
