@@ -173,14 +173,24 @@ int cnp_validate(const void* theta, const void* out, int nblk, int b, int k) {
   return POETX_OK;
 }
 
-// Runs fn(first_block, count, scratch) over chunks of blocks that fit in ws.
-template <typename Fn>
-int cnp_chunks(int nblk, int b, int k, bool backward, void* ws, size_t ws_bytes, Fn fn) {
+// The scratch rules every CNP call checks (one block's worth at least, non-null, aligned),
+// also where a path needs none, so that the contract does not depend on the path.
+int cnp_ws_check(int b, int k, bool backward, const void* ws, size_t ws_bytes) {
   const size_t per = cnp_per_block(b, k, backward);
-  size_t cap = ws_bytes > kCnpFixedBytes ? (ws_bytes - kCnpFixedBytes) / per : 0;
+  const size_t cap = ws_bytes > kCnpFixedBytes ? (ws_bytes - kCnpFixedBytes) / per : 0;
   if (cap < 1) return fail(POETX_ERR_WORKSPACE, "CNP scratch smaller than one block needs");
   if (!ws) return fail(POETX_ERR_INVALID_ARG, "null scratch");
   if (!aligned16(ws)) return fail(POETX_ERR_ALIGN, "scratch must be 16-byte aligned");
+  return POETX_OK;
+}
+
+// Runs fn(first_block, count, scratch) over chunks of blocks that fit in ws.
+template <typename Fn>
+int cnp_chunks(int nblk, int b, int k, bool backward, void* ws, size_t ws_bytes, Fn fn) {
+  const int st = cnp_ws_check(b, k, backward, ws, ws_bytes);
+  if (st != POETX_OK) return st;
+  const size_t per = cnp_per_block(b, k, backward);
+  size_t cap = (ws_bytes - kCnpFixedBytes) / per;
   const size_t per_mat_cap = kCnpChunkTarget / ((size_t)b * b * 4);
   if (cap > per_mat_cap && per_mat_cap >= 1) cap = per_mat_cap;
   for (int b0 = 0; b0 < nblk; b0 += (int)cap) {
@@ -576,6 +586,13 @@ static int cnp_fwd_impl(const float* theta, float* G, void* G_bf16, float* Q_sav
       !aligned16(Q_save) || !aligned16(S_save) || !aligned16(F_save))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cnp_fused_ok(b, k)) {  // every block on chip: one launch, the scratch is not used
+    const int wst = cnp_ws_check(b, k, false, ws, ws_bytes);
+    if (wst != POETX_OK) return wst;
+    POETX_CUDA(launch_cnp_fused_fwd(theta, G, G_bf16, Q_save, S_save, F_save, nblk, b, k, s),
+               "cnp fused forward");
+    return POETX_OK;
+  }
   const CnpPoly P = cnp_poly(k);
   const int d = P.d;
   const int64_t bb = (int64_t)b * b, ntri = (int64_t)b * (b - 1) / 2;
@@ -646,6 +663,13 @@ static int cnp_bwd_impl(const float* theta, const float* dG, const float* Q_save
       !aligned16(S_saved) || !aligned16(F_saved))
     return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cnp_fused_ok(b, k)) {
+    const int wst = cnp_ws_check(b, k, true, ws, ws_bytes);
+    if (wst != POETX_OK) return wst;
+    POETX_CUDA(launch_cnp_fused_bwd(theta, dG, Q_saved, S_saved, F_saved, dtheta, nblk, b, k, s),
+               "cnp fused backward");
+    return POETX_OK;
+  }
   const CnpPoly P = cnp_poly(k);
   const int d = P.d;
   const int64_t bb = (int64_t)b * b, ntri = (int64_t)b * (b - 1) / 2;

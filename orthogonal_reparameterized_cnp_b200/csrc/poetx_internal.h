@@ -151,6 +151,18 @@ cudaError_t launch_split_reduce(const float* src, int nsplit, int64_t stride, fl
 // fp32 -> bf16 (round to nearest even)
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, int64_t count, cudaStream_t s);
 
+// ---- CNP for b = 32 or 64, every block's matrices in shared memory (kernels_cnp_fused.cu)
+bool cnp_fused_ok(int b, int k);
+// G (fp32, and its bf16 copy when G_bf16 is given) from theta; Q_save / S_save / F_save
+// (all or none) receive Q, S = Q^2 and F'.  No device scratch.
+cudaError_t launch_cnp_fused_fwd(const float* theta, float* G, void* G_bf16, float* Q_save,
+                                 float* S_save, float* F_save, int nblk, int b, int k,
+                                 cudaStream_t s);
+// dtheta from dG; Q, S, F' read from the *_saved buffers (all or none) or recomputed.
+cudaError_t launch_cnp_fused_bwd(const float* theta, const float* dG, const float* Q_saved,
+                                 const float* S_saved, const float* F_saved, float* dtheta,
+                                 int nblk, int b, int k, cudaStream_t s);
+
 // ---- CNP as one persistent task-graph launch (kernels_cnp_graph.cu) -----------------
 // Each job is one step applied to every block of a chunk; an item is one output tile of
 // one job for one block.  Square blocks with b % 64 == 0; products read every A operand
