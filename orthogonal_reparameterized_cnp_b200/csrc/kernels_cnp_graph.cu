@@ -605,33 +605,39 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
     const bool dq = diag_tile && qr == qc;  // element-wise i <= j / i < j masks
     const int i0 = m0 + qr * 64 + ty * 4, j0 = n0 + qc * 64 + tx * 4;
     const float* buf = smem + (qi & 1) * k2QBufFloats;
-    // element (rr, c) of the quadrant: acc and the staged operands give the direct value
-    // v (at (i, j)), the mirrored value vm (at (j, i)) and the second output v2
-    auto values = [&](int rr, int c, float& v, float& vm, float& v2) {
-      const int i = i0 + rr, j = j0 + c;
-      const int so = (ty * 4 + rr) * k2QLD + tx * 4 + c;
-      const float e0 = ops[0] ? buf[so] : 0.f;
-      const float e1 = ops[1] ? buf[k2QOpFloats + so] : 0.f;
-      const float es = ops[2] ? buf[2 * k2QOpFloats + so] : 0.f;
-      const float a = acc[qr * 4 + rr][qc * 4 + c];
-      const float sym = (i == j ? diag : 0.f) + ac0 * e0 + ac1 * e1;
-      const float sym2 = (i == j ? diag2 : 0.f) + bc0 * e0 + bc1 * e1;
-      const float skew = alpha * a + skew_c * es;
-      if (mode == SG_SYMSKEW) {
-        v = (i == j) ? sym : sym + skew;
-        vm = sym - skew;
-      } else {
-        v = skew + sym;
-        vm = v;
-      }
-      v2 = alpha_c2 * a + sym2;
-    };
+    // Row rr of the thread's 4 x 4 piece: its staged operands (one 16-byte load per operand),
+    // the direct values v (at (i, j)), the mirrored values vm (at (j, i)) and the second
+    // output v2, all from registers; vm and v2 are kept for the mirror's column stores.
+    float vmq[4][4], v2q[4][4];
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {  // direct: row i, columns j0 .. j0 + 3
+    for (int rr = 0; rr < 4; ++rr) {
       const int i = i0 + rr;
-      float v[4], vm_[4], v2[4];
+      const int so = (ty * 4 + rr) * k2QLD + tx * 4;
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 e0v = ops[0] ? *reinterpret_cast<const float4*>(buf + so) : z4;
+      const float4 e1v = ops[1] ? *reinterpret_cast<const float4*>(buf + k2QOpFloats + so) : z4;
+      const float4 esv = ops[2] ? *reinterpret_cast<const float4*>(buf + 2 * k2QOpFloats + so) : z4;
+      const float e0[4] = {e0v.x, e0v.y, e0v.z, e0v.w};
+      const float e1[4] = {e1v.x, e1v.y, e1v.z, e1v.w};
+      const float es[4] = {esv.x, esv.y, esv.z, esv.w};
+      float v[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) values(rr, c, v[c], vm_[c], v2[c]);
+      for (int c = 0; c < 4; ++c) {
+        const int j = j0 + c;
+        const float a = acc[qr * 4 + rr][qc * 4 + c];
+        const float sym = (i == j ? diag : 0.f) + ac0 * e0[c] + ac1 * e1[c];
+        const float sym2 = (i == j ? diag2 : 0.f) + bc0 * e0[c] + bc1 * e1[c];
+        const float skew = alpha * a + skew_c * es[c];
+        if (mode == SG_SYMSKEW) {
+          v[c] = (i == j) ? sym : sym + skew;
+          vmq[rr][c] = sym - skew;
+        } else {
+          v[c] = skew + sym;
+          vmq[rr][c] = v[c];
+        }
+        v2q[rr][c] = alpha_c2 * a + sym2;
+      }
+      // direct: row i, columns j0 .. j0 + 3
       const int64_t row = (int64_t)i * b;
       if (!dq) {
         __stcg(reinterpret_cast<float4*>(C + row + j0), make_float4(v[0], v[1], v[2], v[3]));
@@ -639,14 +645,15 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
           __stcg(reinterpret_cast<uint2*>(Cb + row + j0),
                  make_uint2(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3])));
         if (C2)
-          __stcg(reinterpret_cast<float4*>(C2 + row + j0), make_float4(v2[0], v2[1], v2[2], v2[3]));
+          __stcg(reinterpret_cast<float4*>(C2 + row + j0),
+                 make_float4(v2q[rr][0], v2q[rr][1], v2q[rr][2], v2q[rr][3]));
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           if (i > j0 + c) continue;
           __stcg(C + row + j0 + c, v[c]);
           if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + j0 + c), bf16_bits(v[c]));
-          if (C2) __stcg(C2 + row + j0 + c, v2[c]);
+          if (C2) __stcg(C2 + row + j0 + c, v2q[rr][c]);
         }
       }
     }
@@ -654,25 +661,23 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int j = j0 + c;
-        float v[4], vm[4], v2[4];
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) values(rr, c, v[rr], vm[rr], v2[rr]);
         const int64_t row = (int64_t)j * b;
         if (!dq) {
-          __stcg(reinterpret_cast<float4*>(C + row + i0), make_float4(vm[0], vm[1], vm[2], vm[3]));
+          __stcg(reinterpret_cast<float4*>(C + row + i0),
+                 make_float4(vmq[0][c], vmq[1][c], vmq[2][c], vmq[3][c]));
           if (Cb)
             __stcg(reinterpret_cast<uint2*>(Cb + row + i0),
-                   make_uint2(bf16x2_bits(vm[0], vm[1]), bf16x2_bits(vm[2], vm[3])));
+                   make_uint2(bf16x2_bits(vmq[0][c], vmq[1][c]), bf16x2_bits(vmq[2][c], vmq[3][c])));
           if (C2)
             __stcg(reinterpret_cast<float4*>(C2 + row + i0),
-                   make_float4(v2[0], v2[1], v2[2], v2[3]));
+                   make_float4(v2q[0][c], v2q[1][c], v2q[2][c], v2q[3][c]));
         } else {
 #pragma unroll
           for (int rr = 0; rr < 4; ++rr) {
             if (i0 + rr >= j) continue;
-            __stcg(C + row + i0 + rr, vm[rr]);
-            if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + i0 + rr), bf16_bits(vm[rr]));
-            if (C2) __stcg(C2 + row + i0 + rr, v2[rr]);
+            __stcg(C + row + i0 + rr, vmq[rr][c]);
+            if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + i0 + rr), bf16_bits(vmq[rr][c]));
+            if (C2) __stcg(C2 + row + i0 + rr, v2q[rr][c]);
           }
         }
       }
