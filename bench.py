@@ -784,9 +784,10 @@ def run_poetx(args):
             roof["frac_of_sustained"] = achieved / sus
 
     # end to end through the public API with host buffers (pinned), copies timed: every
-    # step uploads every linear's x and dy and theta, and downloads y, dx and dtheta; the
-    # host pipeline overlaps the uploads of the next step and the downloads of the previous
-    # one with the step's kernels (two copy engines)
+    # step uploads every linear's x and dy and theta and downloads the step's result,
+    # dtheta (y and dx stay on the device, as for layers that feed other layers); the host
+    # pipeline overlaps the uploads of the next step and the downloads of the previous one
+    # with the step's kernels (two copy engines)
     e2e = None
     if args.e2e_steps > 0:
         from orthogonal_reparameterized_cnp_b200.host_pipeline import HostPipeline
@@ -794,8 +795,7 @@ def run_poetx(args):
         hx = [t.cpu().pin_memory() for t in wl.xs[0]]
         hdy = [t.cpu().pin_memory() for t in wl.dys[0]]
         hth = g.cnp.theta.cpu().pin_memory()
-        hy = [torch.empty(t.shape, dtype=wl.act).pin_memory() for t in wl.ys]
-        hdx = [torch.empty(t.shape, dtype=wl.act).pin_memory() for t in wl.dxs]
+        hy = hdx = None  # the step's result is dtheta
         hdth = torch.empty(g.cnp.dtheta.shape, dtype=torch.float32).pin_memory()
         pipe = HostPipeline(g, nbuf=2, exchange=exchange if world > 1 else None)
         for i in range(3):
@@ -814,12 +814,13 @@ def run_poetx(args):
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
         nbytes = lambda ts: sum(t.numel() * t.element_size() for t in ts)  # noqa: E731
         h2d = nbytes(hx) + nbytes(hdy) + hth.numel() * 4
-        d2h = nbytes(hy) + nbytes(hdx) + hdth.numel() * 4
+        d2h = hdth.numel() * 4
         e2e = {"value": job_tokens_per_s(world, T, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps, "copies": "overlapped with compute (2 buffer sets)"}
+               "steps": args.e2e_steps, "copies": "overlapped with compute (2 buffer sets)",
+               "downloaded": "dtheta (the step's result); y and dx stay on the device"}
         check_status(P, stream, "the end-to-end steps")
-        del pipe, hx, hdy, hy, hdx
+        del pipe, hx, hdy
 
     # the merge of the permutations into W0' (S1: once per set of permutations, every
     # linear of the workload), and the outer-loop merge of the first linear (once per

@@ -8,7 +8,9 @@ concurrently: the upload of step i+1 (copy engine, host -> device), the step i k
 and the download of step i-1 (the other copy engine, device -> host).  Each of `nbuf`
 device buffer sets cycles through upload -> compute -> download; events order the three
 streams so that a set is refilled only after its results have left the device.
-Every step still makes its full upload and download.
+Every step still makes its full upload and its download of dtheta.  The downloads of y
+and dx may be left out (pass None): a training loop whose next layers run on the device
+needs only the step's result, dtheta, on the host.
 """
 from __future__ import annotations
 
@@ -58,9 +60,12 @@ class HostPipeline:
         self.used = [False] * nbuf
 
     def submit(self, i: int, hx, hdy, htheta, hy, hdx, hdtheta) -> None:
+        """hy, hdx: host outputs, or None to keep y and dx on the device only."""
         import torch
         s = i % self.nbuf
-        hx, hdy, hy, hdx = _as_list(hx), _as_list(hdy), _as_list(hy), _as_list(hdx)
+        hx, hdy = _as_list(hx), _as_list(hdy)
+        hy = _as_list(hy) if hy is not None else []
+        hdx = _as_list(hdx) if hdx is not None else []
         with torch.cuda.stream(self.h2d):
             if self.used[s]:
                 self.h2d.wait_event(self.computed[s])  # the set's inputs are consumed

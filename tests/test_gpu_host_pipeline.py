@@ -53,3 +53,13 @@ def test_host_pipeline_matches_inline_steps():
     for i in range(steps):
         for got, ref in zip(outs[i], want[i]):
             assert torch.equal(got, ref), f"step {i}"
+    # only the step's result (dtheta) to the host: y and dx stay on the device
+    hdth = [torch.empty(tuple(layer.dtheta.shape), dtype=torch.float32).pin_memory()
+            for _ in range(steps)]
+    pipe = HostPipeline(layer, nbuf=2)
+    for i in range(steps):
+        pipe.submit(i, hx[i], hdy[i], hth[i], None, None, hdth[i])
+    pipe.synchronize()
+    assert P.device_status() == P.POETX_OK
+    for i in range(steps):
+        assert torch.equal(hdth[i], want[i][2]), f"step {i}"
