@@ -32,6 +32,8 @@ namespace poetx {
 namespace {
 
 constexpr int kFzThreads = 256;
+constexpr int kFzFwdMats = 4;  // Q, S, F', one work matrix
+constexpr int kFzBwdMats = 6;  // Q, S, F', dG, U, R^T
 
 template <int B>
 struct Fz {
@@ -145,11 +147,12 @@ __device__ __forceinline__ void fz_expand(float* Qs, const float* __restrict__ t
 }
 
 // S = Q Q and F' = sum_{j>=1} f_j S^j into shared memory (Ss, Fs), with E = e_0 I +
-// sum_{j>=1} e_j S^j returned in registers when want_e.  W0, W1: work matrices.
+// sum_{j>=1} e_j S^j returned in registers when want_e.  W: work matrix (the powers S^j,
+// j >= 2, one after another: each is written only after every thread has read the last).
 template <int B>
-__device__ __forceinline__ void fz_powers(const float* Qs, float* Ss, float* Fs, float* W0,
-                                          float* W1, const FzCoef& P, int tx, int ty,
-                                          float (&E)[4][4], bool want_e) {
+__device__ __forceinline__ void fz_powers(const float* Qs, float* Ss, float* Fs, float* W,
+                                          const FzCoef& P, int tx, int ty, float (&E)[4][4],
+                                          bool want_e) {
   float acc[4][4], F[4][4];
   fz_mm<B>(Qs, Qs, tx, ty, acc);  // rows of Q = columns of Q^T = -columns of Q
 #pragma unroll
@@ -177,9 +180,9 @@ __device__ __forceinline__ void fz_powers(const float* Qs, float* Ss, float* Fs,
         F[r][c] = fmaf(P.f[j], acc[r][c], F[r][c]);
       }
     if (j < P.d) {
-      float* nxt = (j & 1) ? W1 : W0;
-      fz_store<B>(nxt, tx, ty, acc);
-      prev = nxt;
+      if (prev == W) __syncthreads();  // every thread has read S^(j-1) from W
+      fz_store<B>(W, tx, ty, acc);
+      prev = W;
     }
   }
   fz_store<B>(Fs, tx, ty, F);
@@ -194,9 +197,8 @@ __global__ void __launch_bounds__(kFzThreads)
   extern __shared__ __align__(16) float fz_smem[];
   const int sb = threadIdx.x / C::TPB, t = threadIdx.x % C::TPB;
   const int tx = t % (B / 4), ty = t / (B / 4);
-  float* base = fz_smem + sb * 5 * C::MAT;
-  float *Qs = base, *Ss = base + C::MAT, *Fs = base + 2 * C::MAT, *W0 = base + 3 * C::MAT,
-        *W1 = base + 4 * C::MAT;
+  float* base = fz_smem + sb * kFzFwdMats * C::MAT;
+  float *Qs = base, *Ss = base + C::MAT, *Fs = base + 2 * C::MAT, *W = base + 3 * C::MAT;
   const int64_t blk = (int64_t)blockIdx.x * C::BPC + sb;
   const bool live = blk < nblk;  // (every thread still meets every barrier)
   const int64_t bb = (int64_t)B * B;
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kFzThreads)
   if (live) fz_expand<B>(Qs, theta + blk * ((int64_t)B * (B - 1) / 2), tx, ty);
   __syncthreads();
   float E[4][4];
-  fz_powers<B>(Qs, Ss, Fs, W0, W1, P, tx, ty, E, true);
+  fz_powers<B>(Qs, Ss, Fs, W, P, tx, ty, E, true);
   __syncthreads();  // F' is complete
   float acc[4][4], q[4][4];
   fz_mm<B>(Qs, Fs, tx, ty, acc);  // -(Q F')
@@ -247,12 +249,11 @@ __global__ void __launch_bounds__(kFzThreads)
   extern __shared__ __align__(16) float fz_smem[];
   const int sb = threadIdx.x / C::TPB, t = threadIdx.x % C::TPB;
   const int tx = t % (B / 4), ty = t / (B / 4);
-  float* base = fz_smem + sb * 10 * C::MAT;
+  float* base = fz_smem + sb * kFzBwdMats * C::MAT;
+  // Q, S, F', dG, and U and R^T of the recursion (single buffers: each level reads them all
+  // before any thread writes the next level)
   float *Qs = base, *Ss = base + C::MAT, *Fs = base + 2 * C::MAT, *Gs = base + 3 * C::MAT,
-        *Gt = base + 4 * C::MAT, *X2 = base + 5 * C::MAT;
-  // U and R^T in two buffers each (current, next), swapped per level
-  float *Ucur = base + 6 * C::MAT, *Unx = base + 7 * C::MAT;
-  float *Rcur = base + 8 * C::MAT, *Rnx = base + 9 * C::MAT;
+        *Us = base + 4 * C::MAT, *Rs = base + 5 * C::MAT;
   const int64_t blk = (int64_t)blockIdx.x * C::BPC + sb;
   const bool live = blk < nblk;
   const int64_t bb = (int64_t)B * B, ntri = (int64_t)B * (B - 1) / 2;
@@ -270,38 +271,35 @@ __global__ void __launch_bounds__(kFzThreads)
     }
   }
   __syncthreads();
-  if (!Si) {  // the forward's S and F' again (U[0], U[1] as work space)
+  if (!Si) {  // the forward's S and F' again (U as work space)
     float E[4][4];
-    fz_powers<B>(Qs, Ss, Fs, Ucur, Unx, P, tx, ty, E, false);
+    fz_powers<B>(Qs, Ss, Fs, Us, P, tx, ty, E, false);
     __syncthreads();
   }
-  // dG^T, and D = Q dG = -(rows of Q) dG
-  fz_load<B>(Gs, tx, ty, v);
-  fz_store_t<B>(Gt, tx, ty, v);
-  fz_mm<B>(Qs, Gs, tx, ty, acc);
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = -acc[r][c];
-  fz_store<B>(Ucur, tx, ty, acc);  // D (temporarily)
-  __syncthreads();
-  // X2 = D + D^T;  N_j = e_j X1 - f_j X2 with X1 = dG + dG^T
+  // X1 = dG + dG^T, and D = Q dG = -(rows of Q) dG
   float x1[4][4], x2[4][4];
-  fz_load_t<B>(Ucur, tx, ty, v);
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) x2[r][c] = acc[r][c] + v[r][c];
   {
     float g[4][4], gt[4][4];
     fz_load<B>(Gs, tx, ty, g);
-    fz_load<B>(Gt, tx, ty, gt);
+    fz_load_t<B>(Gs, tx, ty, gt);
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
       for (int c = 0; c < 4; ++c) x1[r][c] = g[r][c] + gt[r][c];
   }
-  fz_store<B>(X2, tx, ty, x2);
+  fz_mm<B>(Qs, Gs, tx, ty, acc);
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = -acc[r][c];
+  fz_store<B>(Us, tx, ty, acc);  // D (temporarily)
+  __syncthreads();
+  // X2 = D + D^T;  N_j = e_j X1 - f_j X2
+  fz_load_t<B>(Us, tx, ty, v);
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) x2[r][c] = acc[r][c] + v[r][c];
   __syncthreads();  // D is no longer read
   // U_d = R_d = N_d
   const int d = P.d;
@@ -309,12 +307,12 @@ __global__ void __launch_bounds__(kFzThreads)
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) v[r][c] = P.e[d] * x1[r][c] - P.f[d] * x2[r][c];
-  fz_store<B>(Ucur, tx, ty, v);
-  fz_store_t<B>(Rcur, tx, ty, v);
+  fz_store<B>(Us, tx, ty, v);
+  fz_store_t<B>(Rs, tx, ty, v);
   for (int l = d - 1; l >= 1; --l) {
     __syncthreads();  // U_{l+1}, R_{l+1} are complete
-    fz_mm<B>(Ss, Ucur, tx, ty, acc);   // S U_{l+1}
-    fz_mm<B>(Rcur, Ss, tx, ty, acc2);  // R_{l+1} S
+    fz_mm<B>(Ss, Us, tx, ty, acc);   // S U_{l+1}
+    fz_mm<B>(Rs, Ss, tx, ty, acc2);  // R_{l+1} S
     float u[4][4], rr[4][4];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -324,29 +322,26 @@ __global__ void __launch_bounds__(kFzThreads)
         rr[r][c] = n + acc2[r][c];
         u[r][c] = rr[r][c] + acc[r][c];
       }
-    fz_store<B>(Unx, tx, ty, u);
-    fz_store_t<B>(Rnx, tx, ty, rr);
-    float* t0 = Ucur;
-    Ucur = Unx;
-    Unx = t0;
-    float* t1 = Rcur;
-    Rcur = Rnx;
-    Rnx = t1;
+    __syncthreads();  // every thread has read U_{l+1} and R_{l+1}
+    fz_store<B>(Us, tx, ty, u);
+    fz_store_t<B>(Rs, tx, ty, rr);
   }
-  __syncthreads();  // Y = U_1 is complete
-  // A = f_0 dG + dG F' - Y Q  (dG through its transpose, Y symmetric)
-  fz_mm<B>(Gt, Fs, tx, ty, acc);
-  fz_mm<B>(Ucur, Qs, tx, ty, acc2);
+  __syncthreads();  // Y = U_1 is complete; R is no longer read
+  // dG^T into R's buffer, then A = f_0 dG + dG F' - Y Q  (Y symmetric)
   fz_load<B>(Gs, tx, ty, v);
+  fz_store_t<B>(Rs, tx, ty, v);
+  __syncthreads();
+  fz_mm<B>(Rs, Fs, tx, ty, acc);
+  fz_mm<B>(Us, Qs, tx, ty, acc2);
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) v[r][c] = P.f[0] * v[r][c] + acc[r][c] - acc2[r][c];
-  fz_store<B>(X2, tx, ty, v);  // A (X2 is no longer read)
+  fz_store<B>(Ss, tx, ty, v);  // A (S is no longer read)
   __syncthreads();
   if (!live) return;
   float at[4][4];
-  fz_load_t<B>(X2, tx, ty, at);
+  fz_load_t<B>(Ss, tx, ty, at);
   float* th = dtheta + blk * ntri;
 #pragma unroll
   for (int r = 0; r < 4; ++r)
@@ -389,7 +384,7 @@ template <int B>
 cudaError_t fwd_t(const float* theta, float* G, void* Gb, float* Qo, float* So, float* Fo,
                   int nblk, int k, cudaStream_t s) {
   using C = Fz<B>;
-  const size_t smem = (size_t)C::BPC * 5 * C::MAT * sizeof(float);
+  const size_t smem = (size_t)C::BPC * kFzFwdMats * C::MAT * sizeof(float);
   cudaError_t e = fz_attr<B, true>(k_cnp_fused_fwd<B>, smem);
   if (e != cudaSuccess) return e;
   const int grid = (nblk + C::BPC - 1) / C::BPC;
@@ -404,7 +399,7 @@ template <int B>
 cudaError_t bwd_t(const float* theta, const float* dG, const float* Qi, const float* Si,
                   const float* Fi, float* dtheta, int nblk, int k, cudaStream_t s) {
   using C = Fz<B>;
-  const size_t smem = (size_t)C::BPC * 10 * C::MAT * sizeof(float);
+  const size_t smem = (size_t)C::BPC * kFzBwdMats * C::MAT * sizeof(float);
   cudaError_t e = fz_attr<B, false>(k_cnp_fused_bwd<B>, smem);
   if (e != cudaSuccess) return e;
   const int grid = (nblk + C::BPC - 1) / C::BPC;
