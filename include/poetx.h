@@ -378,8 +378,8 @@ int poetx_selftest_wait_timeout(const float* theta, float* G, int32_t nblk, int3
 /*
  * FP32 FMA throughput probe (no counterpart in the pages; the measured peak of the pipe that
  * bounds the SIMT CNP kernels): one launch of `ctas` CTAs x 512 threads, every thread running
- * 16 independent chains of `iters` fused multiply-adds, i.e. ctas * 512 * 16 * iters * 2
- * FLOPs.  Time it with events on `stream`.
+ * 16 independent chains of `iters` fused multiply-adds (in packed pairs, two FMAs per
+ * instruction), i.e. ctas * 512 * 16 * iters * 2 FLOPs.  Time it with events on `stream`.
  *   out: device fp32 [ctas * 512], written (the chains' sums).
  *   Errors: INVALID_ARG, ALIGN, CUDA.
  */

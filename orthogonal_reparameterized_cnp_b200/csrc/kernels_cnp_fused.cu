@@ -23,7 +23,7 @@
 // threads holds 256 / (B / 4)^2 blocks (1 for b = 64, 4 for b = 32).  Every product reads A
 // through its transpose (At, row k = column k of A): the symmetric and skew operands are
 // their own transposes up to sign, and the general ones are kept transposed.  Per k step a
-// thread issues two 16-byte shared loads and 16 FFMAs.
+// thread issues two 16-byte shared loads and 16 FMAs (as 8 packed pairs).
 #include <cuda_bf16.h>
 
 #include "poetx_internal.h"
@@ -53,11 +53,50 @@ __device__ __forceinline__ int64_t tri_index(int i, int j, int b) {
   return (int64_t)i * b - (int64_t)i * (i + 1) / 2 + (j - i - 1);
 }
 
-// acc = A Bm with At = A^T (row k of At = column k of A); acc is overwritten
+#ifndef FZ_FMA2
+#define FZ_FMA2 1
+#endif
+
+// acc = A Bm with At = A^T (row k of At = column k of A); acc is overwritten.
+// With FZ_FMA2 the 16 FMAs of a k step run as 8 packed pairs (fma.rn.f32x2: two fp32 fused
+// multiply-adds, each rounded once as fmaf, in the same order over k), on the pairs
+//   D[p][q] = (acc[2p][2q],     acc[2p + 1][2q + 1]) += (a[2p], a[2p + 1]) * (b[2q], b[2q + 1])
+//   X[p][q] = (acc[2p][2q + 1], acc[2p + 1][2q])     += (a[2p], a[2p + 1]) * (b[2q + 1], b[2q])
+// whose a and b pairs are halves of the 16-byte loads.
 template <int B>
 __device__ __forceinline__ void fz_mm(const float* __restrict__ At, const float* __restrict__ Bm,
                                       int tx, int ty, float (&acc)[4][4]) {
   constexpr int LD = Fz<B>::LD;
+#if FZ_FMA2
+  unsigned long long D[2][2] = {{0ull, 0ull}, {0ull, 0ull}};  // (+0.f, +0.f)
+  unsigned long long X[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+#pragma unroll 8
+  for (int k = 0; k < B; ++k) {
+    const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(At + k * LD + 4 * ty);
+    const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(Bm + k * LD + 4 * tx);
+    const unsigned long long ap[2] = {a.x, a.y}, bp[2] = {b.x, b.y};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      unsigned long long bs;  // (b[2q + 1], b[2q])
+      asm("{\n\t.reg .b32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tmov.b64 %0, {hi, lo};\n\t}"
+          : "=l"(bs) : "l"(bp[q]));
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(D[p][q]) : "l"(ap[p]), "l"(bp[q]));
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(X[p][q]) : "l"(ap[p]), "l"(bs));
+      }
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 2; ++p)
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * p][2 * q]), "=f"(acc[2 * p + 1][2 * q + 1])
+          : "l"(D[p][q]));
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * p][2 * q + 1]), "=f"(acc[2 * p + 1][2 * q])
+          : "l"(X[p][q]));
+    }
+#else
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -73,6 +112,7 @@ __device__ __forceinline__ void fz_mm(const float* __restrict__ At, const float*
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
   }
+#endif
 }
 
 template <int B>

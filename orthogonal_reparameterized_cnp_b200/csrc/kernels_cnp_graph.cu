@@ -62,7 +62,7 @@ constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
 // ---- 128 x 128 items ----------------------------------------------------------------
 // Tuning knobs (defaults measured best on B200): k slice depth, cp.async stages, unrolling
 // of the k steps of a slice, CTAs per SM, register double-buffering of the operand
-// fragments.
+// fragments (scalar FMAs only), packed-pair FMAs.
 #ifndef CNP2_BK
 #define CNP2_BK 16
 #endif
@@ -77,6 +77,9 @@ constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
 #endif
 #ifndef CNP2_DBUF
 #define CNP2_DBUF 0
+#endif
+#ifndef CNP2_FMA2
+#define CNP2_FMA2 1
 #endif
 constexpr int k2Threads = 256;  // 16 x 16 threads, 8 x 8 outputs each
 constexpr int k2BK = CNP2_BK;
@@ -459,6 +462,51 @@ __device__ __forceinline__ void kslice128(float (&acc)[8][8], const float* As, c
   }
 }
 
+#if CNP2_FMA2
+// The same k slice on packed pairs: fma.rn.f32x2 does two independent fp32 fused
+// multiply-adds (each rounded once, as fmaf), so a k step takes 32 issue slots instead of 64
+// for the same 64 FMAs and the same per-element order over k.  Accumulator pairs:
+//   D[p][q] = (acc[2p][2q],     acc[2p + 1][2q + 1]) += (a[2p], a[2p + 1]) * (b[2q], b[2q + 1])
+//   X[p][q] = (acc[2p][2q + 1], acc[2p + 1][2q])     += (a[2p], a[2p + 1]) * (b[2q + 1], b[2q])
+// so the a and b pairs come straight from the 16-byte shared-memory loads; only the swapped
+// b pairs are built per k step.
+__device__ __forceinline__ void fma2(unsigned long long& d, unsigned long long a,
+                                     unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ unsigned long long swap_pair(unsigned long long v) {
+  unsigned long long r;
+  asm("{\n\t.reg .b32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tmov.b64 %0, {hi, lo};\n\t}"
+      : "=l"(r) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ void kslice128_x2(unsigned long long (&D)[4][4],
+                                             unsigned long long (&X)[4][4], const float* As,
+                                             const float* Bs, int tx, int ty) {
+#pragma unroll k2KUnroll
+  for (int k = 0; k < k2BK; ++k) {
+    const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(As + k * k2LD + ty * 4);
+    const ulonglong2 a1 = *reinterpret_cast<const ulonglong2*>(As + k * k2LD + 64 + ty * 4);
+    const ulonglong2 b0 = *reinterpret_cast<const ulonglong2*>(Bs + k * k2LD + tx * 4);
+    const ulonglong2 b1 = *reinterpret_cast<const ulonglong2*>(Bs + k * k2LD + 64 + tx * 4);
+    const unsigned long long a[4] = {a0.x, a0.y, a1.x, a1.y};
+    const unsigned long long bb[4] = {b0.x, b0.y, b1.x, b1.y};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const unsigned long long bs = swap_pair(bb[q]);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        fma2(D[p][q], a[p], bb[q]);
+        fma2(X[p][q], a[p], bs);
+      }
+    }
+  }
+}
+__device__ __forceinline__ void unpair(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+#endif
+
 __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* smem) {
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
@@ -486,10 +534,18 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
   const float scale = A2 ? s2 * J.alpha2 : s1;
 
   float acc[8][8];
+#if CNP2_FMA2
+  unsigned long long accD[4][4], accX[4][4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) accD[p][q] = accX[p][q] = 0ull;  // (+0.f, +0.f)
+#else
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+#endif
 
   auto As_ = [&](int st) { return smem + st * k2StageFloats; };
   auto Bs_ = [&](int st) { return smem + st * k2StageFloats + k2BK * k2LD; };
@@ -517,14 +573,28 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
     cp_wait<k2Stages - 2>();
     __syncthreads();  // k tile kt landed for every thread; tile kt - 1 fully consumed
     issue(kt + k2Stages - 1);
+    const float* As = As_(kt % k2Stages);
+    const float* Bs = Bs_(kt % k2Stages);
+#if CNP2_FMA2
+    if (kt == nk1) {  // only with a second product
+      unsigned long long bnd;
+      asm("mov.b64 %0, {%1, %1};" : "=l"(bnd) : "f"(boundary));
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(accD[p][q]) : "l"(bnd));
+          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(accX[p][q]) : "l"(bnd));
+        }
+    }
+    kslice128_x2(accD, accX, As, Bs, tx, ty);
+#else
     if (kt == nk1) {  // only with a second product
 #pragma unroll
       for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] *= boundary;
     }
-    const float* As = As_(kt % k2Stages);
-    const float* Bs = Bs_(kt % k2Stages);
 #if CNP2_DBUF
     float4 a0 = *reinterpret_cast<const float4*>(As + ty * 4);
     float4 a1 = *reinterpret_cast<const float4*>(As + 64 + ty * 4);
@@ -548,8 +618,18 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
 #else
     kslice128(acc, As, Bs, tx, ty);
 #endif
+#endif
   }
   cp_wait<0>();
+#if CNP2_FMA2
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      unpair(accD[p][q], acc[2 * p][2 * q], acc[2 * p + 1][2 * q + 1]);
+      unpair(accX[p][q], acc[2 * p][2 * q + 1], acc[2 * p + 1][2 * q]);
+    }
+#endif
 
   // ---- epilogue from the registers, quadrant by quadrant
   // sym = diag*delta + sum addc*add;  skew = alpha*acc + skew_c*skew_add
