@@ -81,6 +81,9 @@ constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
 #ifndef CNP2_FMA2
 #define CNP2_FMA2 1
 #endif
+#ifndef CNP2_DIAGSKIP
+#define CNP2_DIAGSKIP 1
+#endif
 constexpr int k2Threads = 256;  // 16 x 16 threads, 8 x 8 outputs each
 constexpr int k2BK = CNP2_BK;
 constexpr int k2LD = 128 + 4;  // row stride of a staged k slice (16-byte aligned rows)
@@ -157,6 +160,77 @@ __device__ __forceinline__ int64_t tri_idx(int i, int j, int b) {
   return (int64_t)i * b - (int64_t)i * (i + 1) / 2 + (j - i - 1);
 }
 
+#if CNP2_FMA2
+// Product k steps on packed pairs: fma.rn.f32x2 does two independent fp32 fused
+// multiply-adds (each rounded once, as fmaf), so an outer-product step of 2P x 2Q
+// accumulators takes 2PQ issue slots instead of 4PQ, in the same per-element order over k.
+// Accumulator pairs:
+//   D[p][q] = (acc[2p][2q],     acc[2p + 1][2q + 1]) += (a[2p], a[2p + 1]) * (b[2q], b[2q + 1])
+//   X[p][q] = (acc[2p][2q + 1], acc[2p + 1][2q])     += (a[2p], a[2p + 1]) * (b[2q + 1], b[2q])
+// so the a and b pairs are halves of 16-byte shared-memory loads; only the swapped b pairs
+// are built per k step.
+__device__ __forceinline__ void fma2(unsigned long long& d, unsigned long long a,
+                                     unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ unsigned long long swap_pair(unsigned long long v) {
+  unsigned long long r;
+  asm("{\n\t.reg .b32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tmov.b64 %0, {hi, lo};\n\t}"
+      : "=l"(r) : "l"(v));
+  return r;
+}
+template <int NP, int NQ>
+__device__ __forceinline__ void outer2(unsigned long long (&D)[NP][NQ],
+                                       unsigned long long (&X)[NP][NQ],
+                                       const unsigned long long (&a)[NP],
+                                       const unsigned long long (&b)[NQ]) {
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const unsigned long long bs = swap_pair(b[q]);
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      fma2(D[p][q], a[p], b[q]);
+      fma2(X[p][q], a[p], bs);
+    }
+  }
+}
+template <int NP, int NQ>
+__device__ __forceinline__ void zero2(unsigned long long (&D)[NP][NQ],
+                                      unsigned long long (&X)[NP][NQ]) {
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) D[p][q] = X[p][q] = 0ull;  // (+0.f, +0.f)
+}
+template <int NP, int NQ>
+__device__ __forceinline__ void scale2(unsigned long long (&D)[NP][NQ],
+                                       unsigned long long (&X)[NP][NQ], float f) {
+  unsigned long long ff;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(ff) : "f"(f));
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(D[p][q]) : "l"(ff));
+      asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(X[p][q]) : "l"(ff));
+    }
+}
+template <int NP, int NQ>
+__device__ __forceinline__ void unpack2(const unsigned long long (&D)[NP][NQ],
+                                        const unsigned long long (&X)[NP][NQ],
+                                        float (&acc)[2 * NP][2 * NQ]) {
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * p][2 * q]), "=f"(acc[2 * p + 1][2 * q + 1])
+          : "l"(D[p][q]));
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * p][2 * q + 1]), "=f"(acc[2 * p + 1][2 * q])
+          : "l"(X[p][q]));
+    }
+}
+#endif
+
 // ------------------------------------------------------------------ product tile
 // C-tile (64 x 64) of one block: acc = op(A1) B1 (+ alpha2 op(A2) B2), every A read by rows
 // (symmetric, skew, or given transposed), then the structured epilogue.
@@ -191,10 +265,15 @@ __device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem
   const float g_scale = (nk2 > 0 && kt_end > nk1) ? s2 * J.alpha2 : s1;
 
   float acc[8][4];
+#if CNP2_FMA2
+  unsigned long long accD[4][2], accX[4][2];
+  zero2(accD, accX);
+#else
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#endif
 
   float* ring = smem + grp * kStages * kStageFloats;
   auto As_ = [&](int st) { return reinterpret_cast<float (*)[kLD]>(ring + st * kStageFloats); };
@@ -249,15 +328,27 @@ __device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem
     if (kt - kt_begin < kStages - 1) cp_wait<kStages - 1>(); else cp_wait<kStages - 2>();
     group_sync();
     issue(kt + kStages - 1);
+    const int st = (kt - kt_begin) % kStages;
+    float (*As)[kLD] = As_(st);
+    float (*Bs)[kLD] = Bs_(st);
+#if CNP2_FMA2
+    if (nk2 > 0 && kt == nk1 && kt > kt_begin) scale2(accD, accX, boundary);
+#pragma unroll
+    for (int k = 0; k < kBK; ++k) {
+      const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(&As[k][ty * 8]);
+      const ulonglong2 a1 = *reinterpret_cast<const ulonglong2*>(&As[k][ty * 8 + 4]);
+      const ulonglong2 bv = *reinterpret_cast<const ulonglong2*>(&Bs[k][tx * 4]);
+      const unsigned long long a[4] = {a0.x, a0.y, a1.x, a1.y};
+      const unsigned long long bb[2] = {bv.x, bv.y};
+      outer2(accD, accX, a, bb);
+    }
+#else
     if (nk2 > 0 && kt == nk1 && kt > kt_begin) {
 #pragma unroll
       for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[r][c] *= boundary;
     }
-    const int st = (kt - kt_begin) % kStages;
-    float (*As)[kLD] = As_(st);
-    float (*Bs)[kLD] = Bs_(st);
 #pragma unroll
     for (int k = 0; k < kBK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(&As[k][ty * 8]);
@@ -270,7 +361,11 @@ __device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bb[c], acc[r][c]);
     }
+#endif
   }
+#if CNP2_FMA2
+  unpack2(accD, accX, acc);
+#endif
   cp_wait<0>();
   __syncthreads();  // every group is done with its ring: the space becomes red[]
 
@@ -441,8 +536,7 @@ __device__ void product_tile64(const CnpJob& J, int z, int t, int b, float* smem
 // thread (no split, no partial-tile reduction); the epilogue works quadrant by quadrant
 // from the accumulator registers: operand rows are read as 16-byte vectors, the tile is
 // stored with 16-byte row stores, and the mirror of a symmetric (or symmetric + skew)
-// result is stored from the same registers as 16-byte column segments (four consecutive
-// rows of the thread become four consecutive columns of the mirrored row).
+// result is transposed through shared memory and stored as whole rows too.
 // One k slice of the 128 x 128 item: acc[r][c] += A[k][row r] B[k][col c] for the thread's
 // rows {4 ty + r} U {64 + 4 ty + r} and columns {4 tx + c} U {64 + 4 tx + c}.
 __device__ __forceinline__ void kslice128(float (&acc)[8][8], const float* As, const float* Bs,
@@ -462,24 +556,12 @@ __device__ __forceinline__ void kslice128(float (&acc)[8][8], const float* As, c
   }
 }
 
+
 #if CNP2_FMA2
-// The same k slice on packed pairs: fma.rn.f32x2 does two independent fp32 fused
-// multiply-adds (each rounded once, as fmaf), so a k step takes 32 issue slots instead of 64
-// for the same 64 FMAs and the same per-element order over k.  Accumulator pairs:
-//   D[p][q] = (acc[2p][2q],     acc[2p + 1][2q + 1]) += (a[2p], a[2p + 1]) * (b[2q], b[2q + 1])
-//   X[p][q] = (acc[2p][2q + 1], acc[2p + 1][2q])     += (a[2p], a[2p + 1]) * (b[2q + 1], b[2q])
-// so the a and b pairs come straight from the 16-byte shared-memory loads; only the swapped
-// b pairs are built per k step.
-__device__ __forceinline__ void fma2(unsigned long long& d, unsigned long long a,
-                                     unsigned long long b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
-}
-__device__ __forceinline__ unsigned long long swap_pair(unsigned long long v) {
-  unsigned long long r;
-  asm("{\n\t.reg .b32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tmov.b64 %0, {hi, lo};\n\t}"
-      : "=l"(r) : "l"(v));
-  return r;
-}
+// One k slice of the 128 x 128 item on packed pairs.  LOWER_LEFT = false skips the
+// quadrant below the diagonal (rows 64.., columns ..63: pairs p >= 2, q < 2) of a diagonal
+// tile of a symmetric result, which the epilogue never stores.
+template <bool LOWER_LEFT>
 __device__ __forceinline__ void kslice128_x2(unsigned long long (&D)[4][4],
                                              unsigned long long (&X)[4][4], const float* As,
                                              const float* Bs, int tx, int ty) {
@@ -496,14 +578,12 @@ __device__ __forceinline__ void kslice128_x2(unsigned long long (&D)[4][4],
       const unsigned long long bs = swap_pair(bb[q]);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
+        if (!LOWER_LEFT && p >= 2 && q < 2) continue;
         fma2(D[p][q], a[p], bb[q]);
         fma2(X[p][q], a[p], bs);
       }
     }
   }
-}
-__device__ __forceinline__ void unpair(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 #endif
 
@@ -519,6 +599,8 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
     tile_pair(nt, t, I, Jt);
   }
   const int m0 = I * 128, n0 = Jt * 128;
+  // a diagonal tile of a symmetric (or symmetric + skew) result stores only i <= j
+  const bool skip_ll = J.mode != SG_FULL && I == Jt;
   const int64_t boff = (int64_t)z * b * b;
   const float* A1 = J.A + boff;
   const float* B1 = J.B + boff;
@@ -536,10 +618,7 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
   float acc[8][8];
 #if CNP2_FMA2
   unsigned long long accD[4][4], accX[4][4];
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) accD[p][q] = accX[p][q] = 0ull;  // (+0.f, +0.f)
+  zero2(accD, accX);
 #else
 #pragma unroll
   for (int r = 0; r < 8; ++r)
@@ -576,18 +655,11 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
     const float* As = As_(kt % k2Stages);
     const float* Bs = Bs_(kt % k2Stages);
 #if CNP2_FMA2
-    if (kt == nk1) {  // only with a second product
-      unsigned long long bnd;
-      asm("mov.b64 %0, {%1, %1};" : "=l"(bnd) : "f"(boundary));
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(accD[p][q]) : "l"(bnd));
-          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(accX[p][q]) : "l"(bnd));
-        }
-    }
-    kslice128_x2(accD, accX, As, Bs, tx, ty);
+    if (kt == nk1) scale2(accD, accX, boundary);  // only with a second product
+    if (CNP2_DIAGSKIP && skip_ll)
+      kslice128_x2<false>(accD, accX, As, Bs, tx, ty);
+    else
+      kslice128_x2<true>(accD, accX, As, Bs, tx, ty);
 #else
     if (kt == nk1) {  // only with a second product
 #pragma unroll
@@ -622,13 +694,7 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
   }
   cp_wait<0>();
 #if CNP2_FMA2
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      unpair(accD[p][q], acc[2 * p][2 * q], acc[2 * p + 1][2 * q + 1]);
-      unpair(accX[p][q], acc[2 * p][2 * q + 1], acc[2 * p + 1][2 * q]);
-    }
+  unpack2(accD, accX, acc);
 #endif
 
   // ---- epilogue from the registers, quadrant by quadrant
@@ -737,27 +803,47 @@ __device__ void product_tile128(const CnpJob& J, int z, int t, int b, float* sme
         }
       }
     }
-    if (structured) {  // mirror: row j, columns i0 .. i0 + 3
+    if (structured) {
+      // mirror: element (i, j) of the quadrant goes to (j, i).  The thread's 4 x 4 pieces of
+      // the mirrored values are transposed through the quadrant's staging buffer (its
+      // operands are in registers by now), so that the mirror is stored as whole rows.
+      __syncthreads();  // every thread has read its operands from buffer (qi & 1)
+      float* tb = smem + (qi & 1) * k2QBufFloats;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int j = j0 + c;
-        const int64_t row = (int64_t)j * b;
-        if (!dq) {
-          __stcg(reinterpret_cast<float4*>(C + row + i0),
-                 make_float4(vmq[0][c], vmq[1][c], vmq[2][c], vmq[3][c]));
-          if (Cb)
-            __stcg(reinterpret_cast<uint2*>(Cb + row + i0),
-                   make_uint2(bf16x2_bits(vmq[0][c], vmq[1][c]), bf16x2_bits(vmq[2][c], vmq[3][c])));
-          if (C2)
-            __stcg(reinterpret_cast<float4*>(C2 + row + i0),
-                   make_float4(v2q[0][c], v2q[1][c], v2q[2][c], v2q[3][c]));
-        } else {
+        *reinterpret_cast<float4*>(tb + (tx * 4 + c) * k2QLD + ty * 4) =
+            make_float4(vmq[0][c], vmq[1][c], vmq[2][c], vmq[3][c]);
+        if (C2)
+          *reinterpret_cast<float4*>(tb + k2QOpFloats + (tx * 4 + c) * k2QLD + ty * 4) =
+              make_float4(v2q[0][c], v2q[1][c], v2q[2][c], v2q[3][c]);
+      }
+      __syncthreads();
+      // mirrored quadrant: rows n0 + qc 64 .., columns m0 + qr 64 ..; a warp stores two
+      // contiguous 256-byte row segments per instruction
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) {
-            if (i0 + rr >= j) continue;
-            __stcg(C + row + i0 + rr, vmq[rr][c]);
-            if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + i0 + rr), bf16_bits(vmq[rr][c]));
-            if (C2) __stcg(C2 + row + i0 + rr, v2q[rr][c]);
+      for (int l = 0; l < 4; ++l) {
+        const int f = tid + l * k2Threads;
+        const int r = f >> 4, c4 = (f & 15) * 4;
+        const int jg = n0 + qc * 64 + r, ig = m0 + qr * 64 + c4;
+        const float4 w = *reinterpret_cast<const float4*>(tb + r * k2QLD + c4);
+        const float4 w2 = C2 ? *reinterpret_cast<const float4*>(tb + k2QOpFloats + r * k2QLD + c4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int64_t row = (int64_t)jg * b;
+        if (!dq) {
+          __stcg(reinterpret_cast<float4*>(C + row + ig), w);
+          if (Cb)
+            __stcg(reinterpret_cast<uint2*>(Cb + row + ig),
+                   make_uint2(bf16x2_bits(w.x, w.y), bf16x2_bits(w.z, w.w)));
+          if (C2) __stcg(reinterpret_cast<float4*>(C2 + row + ig), w2);
+        } else {  // strictly below the diagonal only: (j, i) with i < j
+          const float wv[4] = {w.x, w.y, w.z, w.w};
+          const float w2v[4] = {w2.x, w2.y, w2.z, w2.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (ig + e >= jg) continue;
+            __stcg(C + row + ig + e, wv[e]);
+            if (Cb) __stcg(reinterpret_cast<unsigned short*>(Cb + row + ig + e), bf16_bits(wv[e]));
+            if (C2) __stcg(C2 + row + ig + e, w2v[e]);
           }
         }
       }
