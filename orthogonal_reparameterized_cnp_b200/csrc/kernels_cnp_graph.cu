@@ -1043,7 +1043,12 @@ __global__ void __launch_bounds__(GraphCfg<TILE>::threads, GraphCfg<TILE>::ctas_
   const int total = g.item_start[g.njobs];
   pdl_trigger();
   pdl_wait();
-  if (threadIdx.x == 0) s_next = atomicAdd(ticket, 1);
+  // three single-thread roles per item, in different warps so that none waits on another:
+  // thread 0 checks the item's dependencies, thread 32 takes the next ticket, thread 64
+  // publishes the previous item's completion
+  constexpr int kTicketThread = 32, kReleaseThread = 64;
+  int done_job = -1, done_z = 0;  // the previous item, published at the next item's start
+  if (threadIdx.x == kTicketThread) s_next = atomicAdd(ticket, 1);
   for (;;) {
     __syncthreads();  // smem of the previous item is free; s_next is visible
     if (threadIdx.x == 0) {
@@ -1051,6 +1056,11 @@ __global__ void __launch_bounds__(GraphCfg<TILE>::threads, GraphCfg<TILE>::ctas_
       s_ok = 1;
     }
     __syncthreads();
+    // publish the previous item: the two barriers order every thread's stores of it before
+    // this release, which waits on nothing, so a published item is never held up by the
+    // next item's dependencies
+    if (threadIdx.x == kReleaseThread && done_job >= 0)
+      red_release_add(g.counters + done_job * g.nblk + done_z, 1);
     const int item = s_item;
     if (item >= total) break;
     int j = 0;
@@ -1064,9 +1074,9 @@ __global__ void __launch_bounds__(GraphCfg<TILE>::threads, GraphCfg<TILE>::ctas_
     const int z = local / tiles;
     const int t = local - z * tiles;
     const unsigned deps = g.job[j].deps;
+    // next ticket in flight while this item runs
+    if (threadIdx.x == kTicketThread) s_next = atomicAdd(ticket, 1);
     if (threadIdx.x == 0) {
-      // next ticket in flight while this item runs
-      s_next = atomicAdd(ticket, 1);
       // wait until every job this one reads has finished for block z
       const unsigned long long t0 = gtimer();
       for (int d = 0; d < j && s_ok; ++d) {
@@ -1101,9 +1111,8 @@ __global__ void __launch_bounds__(GraphCfg<TILE>::threads, GraphCfg<TILE>::ctas_
       case JOB_SYMCOMB: symcomb_tile<NT>(J, z, t, g.b, smem); break;
       default: pack_tile<NT>(J, z, t, g.b, smem); break;
     }
-    // publish: the barrier orders every thread's stores before thread 0's release
-    __syncthreads();
-    if (threadIdx.x == 0) red_release_add(g.counters + j * g.nblk + z, 1);
+    done_job = j;
+    done_z = z;
   }
 }
 
