@@ -15,7 +15,8 @@ Default workload: the Llama-13B-shaped decoder block, all 7 linears as POET-X la
 (q, k, v, o 5120 -> 5120; gate, up 5120 -> 13824; down 13824 -> 5120), b = 256, k = 4,
 T = 8192 tokens, bf16 activations, fp32 theta / CNP, 382 CNP blocks.  The step touches
 several GB, far more than the 126 MB L2, so consecutive steps never find their inputs in
-L2; workloads whose inputs fit in L2 rotate over three input sets instead.
+L2; for workloads whose inputs fit in L2, a buffer of twice the L2 is written before every
+timed step (outside that step's events), so each step starts from a cold L2.
 
 Besides the headline line the run measures: the layer-only figure (forward + backward
 without the CNP), CNP-only forward and backward (blocks/s), per-kernel-family device time
@@ -397,9 +398,22 @@ def graph_of(fn, stream):
     return g
 
 
-def time_graphs(graphs, reps, stream):
-    """Device time (ms) of `reps` back-to-back replays cycling over `graphs`."""
+def time_graphs(graphs, reps, stream, flush=None):
+    """Device time (ms) of `reps` back-to-back replays cycling over `graphs`.  With `flush`
+    (a device buffer larger than L2) the buffer is overwritten before every replay and each
+    replay is timed alone, so that no replay finds its data in L2."""
     import torch
+    if flush is not None:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for i in range(reps):
+                flush.fill_(i & 255)
+                evs[i][0].record(stream)
+                graphs[i % len(graphs)].replay()
+                evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -474,8 +488,12 @@ class Workload:
         self.group = P.PoetxLinearGroup(specs, self.b, self.k, self.T, int8_weight=int8)
         es = 2 if self.bf16 else 4
         in_bytes = sum(s.T * (s.n + s.m) * es for s in self.shapes)
-        # inputs larger than L2 per step need no rotation; small ones rotate over 3 sets
-        self.nsets = 1 if in_bytes > 2 * L2_BYTES else 3
+        # inputs larger than L2 per step leave nothing useful in L2 for the next step; small
+        # ones are evicted by writing a buffer of twice the L2 before every timed step
+        self.nsets = 1
+        self.flush = None
+        if in_bytes <= 2 * L2_BYTES:
+            self.flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
         self.xs, self.dys = [xs], [dys]
         for r in range(1, self.nsets):
             self.xs.append([torch.roll(t, shifts=r, dims=0).contiguous() for t in xs])
@@ -496,11 +514,11 @@ class Workload:
         g.backward(xs, dys, self.dxs, 0, stream)
 
     def l2_note(self):
-        if self.nsets == 1:
+        if self.flush is None:
             return (f"each step reads {self.in_bytes >> 20} MB of inputs and touches several "
                     f"times that (> 126 MB L2): no step finds its inputs in L2")
-        return (f"inputs rotate over {self.nsets} sets "
-                f"({self.nsets * self.in_bytes >> 20} MB > 126 MB L2)")
+        return (f"inputs ({self.in_bytes >> 10} KB) fit in L2: L2 flushed before every timed "
+                f"step by writing {self.flush.numel() >> 20} MB, each step timed alone")
 
 
 def check_status(P, stream, where):
@@ -519,7 +537,9 @@ def family_attribution(P, wl, stream, reps, families=None):
         g = graph_of(lambda st: wl.step(0, st), stream)
         P.profile_begin(None)
         tot, launches = 0.0, 0
-        for _ in range(reps):
+        for i in range(reps):
+            if wl.flush is not None:  # inputs that fit in L2: start every replay cold
+                wl.flush.fill_(i & 255)
             g.replay()
             torch.cuda.synchronize()
             n, ms = P.profile_end()
@@ -544,7 +564,9 @@ def single_cta(P, wl, stream, reps, families=("gemm_w0",)):
             g = graph_of(lambda st: wl.step(0, st), stream)
             P.profile_begin(None)
             tot, launches = 0.0, 0
-            for _ in range(reps):
+            for i in range(reps):
+                if wl.flush is not None:
+                    wl.flush.fill_(i & 255)
                 g.replay()
                 torch.cuda.synchronize()
                 n, ms = P.profile_end()
@@ -564,8 +586,8 @@ def cnp_only(P, wl, stream, reps):
     gf = graph_of(lambda st: c.forward(st), stream)
     gb = graph_of(lambda st: c.backward(st), stream)
     time_graphs([gf, gb], 2, stream)
-    fms = time_graphs([gf], reps, stream) / reps
-    bms = time_graphs([gb], reps, stream) / reps
+    fms = time_graphs([gf], reps, stream, wl.flush) / reps
+    bms = time_graphs([gb], reps, stream, wl.flush) / reps
     check_status(P, stream, "the CNP-only replays")
     cf, cb = cnp_flops_per_block(wl.b, wl.k)
     return {"blocks": c.nblk, "b": wl.b, "k": wl.k, "fwd_ms": fms, "bwd_ms": bms,
@@ -624,8 +646,8 @@ def secondary_step(P, key, dev, stream, reps):
     gs = [graph_of(lambda st, i=i: wl.step(i, st), stream) for i in range(wl.nsets)]
     gl = [graph_of(lambda st, i=i: wl.layer_only(i, st), stream) for i in range(wl.nsets)]
     time_graphs(gs, 3, stream)
-    ms = time_graphs(gs, reps, stream) / reps
-    lms = time_graphs(gl, reps, stream) / reps
+    ms = time_graphs(gs, reps, stream, wl.flush) / reps
+    lms = time_graphs(gl, reps, stream, wl.flush) / reps
     check_status(P, stream, f"the {key} replays")
     out = {"workload": workload_name(key, wl.shapes), "ms_per_step": ms,
            "tokens_per_s": wl.T / (ms / 1e3), "layer_only_tokens_per_s": wl.T / (lms / 1e3),
@@ -702,22 +724,29 @@ def run_poetx(args):
     sampler.start()
     time.sleep(0.3)
     launches0 = P.launch_count()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    # one event pair around all steps; with an L2 flush between steps (inputs that fit in
+    # L2), one pair per step with the flush outside it
+    nev = args.steps if wl.flush is not None else 1
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nev)]
     with torch.cuda.stream(stream):
-        ev0.record(stream)
         for i in range(args.steps):
+            if wl.flush is not None:
+                wl.flush.fill_(i & 255)
+            if wl.flush is not None or i == 0:
+                evs[min(i, nev - 1)][0].record(stream)
             if graphs:
                 graphs[i % wl.nsets].replay()  # the layers' kernels; the collective outside
             else:
                 wl.step(i, stream)
             exchange()
-        ev1.record(stream)
+            if wl.flush is not None or i == args.steps - 1:
+                evs[min(i, nev - 1)][1].record(stream)
     torch.cuda.synchronize(dev)
     launches = graph_launches * args.steps if graphs else P.launch_count() - launches0
     barrier()
     clocks = sampler.stop()
-    elapsed_ms = ev0.elapsed_time(ev1)
+    elapsed_ms = sum(a.elapsed_time(b) for a, b in evs)
     max_ms = max_over_ranks(elapsed_ms, dist if world > 1 else None, dev)
     check_status(P, stream, "the timed region")
     ms_per_step = max_ms / args.steps
@@ -727,7 +756,7 @@ def run_poetx(args):
     # layer-only figure: forward + backward of every linear without the CNP
     gl = [graph_of(lambda st, i=i: wl.layer_only(i, st), stream) for i in range(wl.nsets)]
     time_graphs(gl, 3, stream)
-    lms = time_graphs(gl, reps, stream) / reps
+    lms = time_graphs(gl, reps, stream, wl.flush) / reps
     check_status(P, stream, "the layer-only replays")
     del gl
     cnp = cnp_only(P, wl, stream, reps)
@@ -828,7 +857,7 @@ def run_poetx(args):
     merge = None
     gm = graph_of(lambda st: wl.group.merge(st), stream)
     time_graphs([gm], 2, stream)
-    mms = time_graphs([gm], 10, stream) / 10
+    mms = time_graphs([gm], 10, stream, wl.flush) / 10
     mbytes = sum(2.0 * s.m * s.n * (2 if wl.bf16 else 4) for s in shapes)
     merge = {"ms": mms, "achieved_gbs": mbytes / (mms / 1e3) / 1e9}
     del gm
@@ -847,7 +876,7 @@ def run_poetx(args):
         go = graph_of(lambda st: P.outer_merge(L0.W0p, GP, GR, s.b, L0.inv_P, L0.inv_R, pP2d,
                                                pR2d, W0p_new, mws, st), stream)
         time_graphs([go], 2, stream)
-        oms = time_graphs([go], 10, stream) / 10
+        oms = time_graphs([go], 10, stream, wl.flush) / 10
         mb = 2 * s.m * s.n * 2 + (s.n + s.m) * s.b * 2
         outer = {"linear": [s.n, s.m], "ms": oms, "achieved_gbs": mb / (oms / 1e3) / 1e9,
                  "achieved_tflops": 4.0 * s.m * s.n * s.b / (oms / 1e3) / 1e12}
@@ -863,7 +892,7 @@ def run_poetx(args):
         torch.cuda.synchronize(dev)
         gq = [graph_of(lambda st, i=i: wq.step(i, st), stream) for i in range(wq.nsets)]
         time_graphs(gq, 3, stream)
-        qms = time_graphs(gq, reps, stream) / reps
+        qms = time_graphs(gq, reps, stream, wq.flush) / reps
         check_status(P, stream, "the int8-weight steps")
         qfam = family_attribution(P, wq, stream, min(reps, 20), families=("gemm_w0",))
         xq = {"ms_per_step": qms, "tokens_per_s": T / (qms / 1e3), "steps": reps,

@@ -64,10 +64,10 @@ constexpr int kPT = 64, kPLD = 65;  // 64 x 64 tile-pair jobs
 // of the k steps of a slice, CTAs per SM, register double-buffering of the operand
 // fragments (scalar FMAs only), packed-pair FMAs.
 #ifndef CNP2_BK
-#define CNP2_BK 16
+#define CNP2_BK 32
 #endif
 #ifndef CNP2_STAGES
-#define CNP2_STAGES 4
+#define CNP2_STAGES 3
 #endif
 #ifndef CNP2_KUNROLL
 #define CNP2_KUNROLL CNP2_BK
@@ -90,7 +90,7 @@ constexpr int k2LD = 128 + 4;  // row stride of a staged k slice (16-byte aligne
 constexpr int k2Stages = CNP2_STAGES;
 constexpr int k2KUnroll = CNP2_KUNROLL;
 constexpr int k2StageFloats = 2 * k2BK * k2LD;
-constexpr int k2RingFloats = k2Stages * k2StageFloats;  // 66 KB
+constexpr int k2RingFloats = k2Stages * k2StageFloats;  // 99 KB
 // epilogue operands (the adds and the skew term, <= 3 tiles) of one 64 x 64 quadrant are
 // staged in shared memory, two quadrants in flight (reusing the ring after the main loop)
 constexpr int k2QLD = 64 + 4;

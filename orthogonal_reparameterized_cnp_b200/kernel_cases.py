@@ -90,7 +90,8 @@ def layer32():
 
 
 def cnp(nblk, b, k):
-    """Per call: k_zero_ints then k_cnp_graph (forward, then backward)."""
+    """Per call: k_zero_ints then k_cnp_graph (forward, then backward); for b = 32 or 64 one
+    k_cnp_fused_fwd / k_cnp_fused_bwd launch per call instead."""
     dev = _dev()
     c = P.CnpBuffers(nblk, b, k, dev, torch.bfloat16)
     c.theta.copy_(torch.randn(c.theta.shape, device=dev) * 0.01)
