@@ -34,9 +34,9 @@
 // waits for both rings and frees both; four epilogue warps (instead of eight) drain TMEM.
 // No bf16 copy of the weight exists in global memory, and the operands equal those of the
 // bf16 kernel on the dequantised weight, so the results are the same bit for bit.  Measured
-// rate: about 0.8 of the bf16 kernel's, held by the conversion path (its SIMT work and the
-// latency from a stage's release to its refill); more converter warps, deeper rings and
-// converters reading the codes straight from global memory did not raise it.
+// rate: about 0.8 of the bf16 kernel's.  More converter warps, deeper rings, converters
+// reading the codes straight from global memory (less shared-memory traffic) and a 512 x 128
+// pair tile (half the conversions per FLOP, more shared-memory traffic) did not raise it.
 //
 // Every mbarrier wait is bounded (Params2::wait_ns): on a timeout the waiting role records
 // POETX_ERR_TIMEOUT in the device flag and leaves its loop; the CTAs then drain what they can

@@ -508,20 +508,17 @@ int run_bwd_graph(const float* theta, const float* dg, float* dtheta, const BwdM
   int jY = jN;
   const float* S = M.P[1];
   if (d >= 2) {
-    // T_{d-2} = N_{d-1} + Pm + Pm^T with Pm = N_d S
-    const int jPm = g.njobs;
-    g.job[g.njobs++] = prod_job(M.N[d], 1, S, M.Pm, SG_FULL, (1u << jN) | dS);
+    // T_{d-2} = N_{d-1} + S N_d + N_d S: symmetric (S N_d is the transpose of N_d S), so one
+    // structured job of two products over the upper tiles, mirrored
     const int jT = g.njobs;
-    CnpJob jt;
-    jt.type = JOB_SYMCOMB;
-    jt.A = M.N[d - 1];
-    jt.B = M.Pm;
-    jt.nin = 2;
-    jt.nout = 1;
-    jt.coef[0][0] = 0.5f;  // N_{d-1} is symmetric: 0.5 (N + N^T) = N
-    jt.coef[0][1] = 1.f;
-    jt.C = M.T;
-    jt.deps = (1u << jN) | (1u << jPm);
+    CnpJob jt = prod_job(S, 1, M.N[d], M.T, SG_SYM, (1u << jN) | dS);
+    jt.A2 = M.N[d];
+    jt.a2_sym = 1;
+    jt.B2 = S;
+    jt.alpha2 = 1.f;
+    jt.add[0] = M.N[d - 1];
+    jt.addc[0] = 1.f;
+    jt.nadd = 1;
     g.job[g.njobs++] = jt;
     Y = M.T;
     jY = jT;
