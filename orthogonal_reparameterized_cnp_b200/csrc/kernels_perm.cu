@@ -9,8 +9,8 @@
 // rows written with coalesced 16-byte stores; the random access happens only in shared
 // memory.  HBM traffic is exactly one read and one write of the matrix.  For 2-byte
 // elements (the bf16 layer) k_gather_il8 interleaves 8 rows per shared-memory word so
-// that one access serves a column of 8 rows; the row-staged kernels cover fp32 and rows
-// too wide for its stages.
+// that one access serves a column of 8 rows (rows narrower than 2048); the row-staged
+// kernels cover fp32 and wider rows.
 #include <cuda_bf16.h>
 
 #include "poetx_internal.h"
@@ -388,17 +388,12 @@ cudaError_t gather_impl(const void* in, void* out, const int32_t* row_idx,
                       ((reinterpret_cast<uintptr_t>(in) & 15) == 0) &&
                       ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
   const int nvec = cols / V;
-  // interleaved gather: a 4-deep stage ring where it fits (about 90% of a plain copy's
-  // rate on 8192 x 2048 bf16), else 2-deep
-  if (sizeof(E) == 2 && vec_ok && cols <= 2 * 8 * kIlThreads) {
-    const bool one = cols <= 8 * kIlThreads;
-    if (il_smem(4, cols) <= kIlMaxSmem)
-      return one ? il8_launch<1, 4>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s)
-                 : il8_launch<2, 4>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
-    if (il_smem(2, cols) <= kIlMaxSmem)
-      return one ? il8_launch<1, 2>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s)
-                 : il8_launch<2, 2>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
-  }
+  // interleaved gather (4-deep stage ring) for rows narrower than 2048 bf16, where it
+  // measured 1.1-1.2x the row-batched pipeline (256-1024 columns); from 2048 columns on
+  // the pipeline is as fast or faster (+5% at 2048, +19% at 2560, +10% at 4096 against the
+  // interleaved forms that fit there)
+  if (sizeof(E) == 2 && vec_ok && cols < 8 * kIlThreads && il_smem(4, cols) <= kIlMaxSmem)
+    return il8_launch<1, 4>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);
   if (vec_ok && cols <= 65535 && nvec <= 8 * kPipeThreads && 2 * row_bytes <= 96 * 1024) {
     const int need = (nvec + kPipeThreads - 1) / kPipeThreads;
     if (need <= 1) return pipe_launch<E, 1>(in, out, row_idx, col_idx, rows, cols, ld_in, ld_out, s);

@@ -39,8 +39,9 @@ def _P():
 
 # ------------------------------------------------------------------ index maps
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("rows,cols", [(1, 8), (7, 24), (300, 2048), (9, 2056), (17, 3072),
-                                       (33, 14336), (5, 13824)])
+@pytest.mark.parametrize("rows,cols", [(1, 8), (7, 24), (300, 2048), (9, 2056), (3, 2560),
+                                       (6, 2568), (17, 3072), (11, 4096), (33, 14336),
+                                       (5, 13824)])
 def test_permute_cols_bit_exact(dtype, rows, cols):
     import torch
     P = _P()
