@@ -40,7 +40,7 @@ def _sources():
 
 
 def _headers():
-    return sorted(glob.glob(os.path.join(CSRC, "*.h")) +
+    return sorted(glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
                   glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
