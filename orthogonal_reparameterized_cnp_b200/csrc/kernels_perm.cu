@@ -128,14 +128,23 @@ __global__ void __launch_bounds__(kPipeThreads)
   }
 
   const int nbatch = (rows + R - 1) / R;
+  // the thread's first (row, vector) of a batch and the step between its copies, so that
+  // the copy loop needs no division
+  const int rr_first = threadIdx.x / nvec, vv_first = threadIdx.x - rr_first * nvec;
+  const int rr_step = kPipeThreads / nvec, vv_step = kPipeThreads - rr_step * nvec;
   auto issue = [&](int batch, E* dst) {
     const int r0 = batch * R;
     const int nr = min(R, rows - r0);
-    for (int i = threadIdx.x; i < nr * nvec; i += kPipeThreads) {
-      const int rr = i / nvec, vv = i - rr * nvec;
+    for (int rr = rr_first, vv = vv_first; rr < nr;) {
       int sr = row_idx ? row_idx[r0 + rr] : r0 + rr;
       sr = min(max(sr, 0), rows - 1);
       cp_async16(dst + (size_t)rr * row_elems + vv * V, in + (int64_t)sr * ld_in + vv * V);
+      rr += rr_step;
+      vv += vv_step;
+      if (vv >= nvec) {
+        vv -= nvec;
+        ++rr;
+      }
     }
   };
 
